@@ -1,0 +1,161 @@
+/*
+ * q4_0.h -- C ABI of libq4_0_b200.so, the B200 (sm_100a) Q4_0 weight-only
+ * dequantize-and-matmul library.
+ *
+ * The operation.  The pages run every decoder linear of the Voxtral 4B speech
+ * models on 4-bit weights: "Q4_0 GGUF" weights through a custom fused
+ * dequant+matmul shader (voxtral-mini-realtime-rs (Shannon-Prime fork)
+ * README, "RTF Benchmark Results" and "Architecture Summary" (Q4 matmul
+ * kernel per decoder layer); hakusoku.com story 5135, linear ops and
+ * embeddings), with fused QKV and gate/up projections and batch-2 CFG
+ * (voxtral-mini-realtime-rs README, "TTS (Text-to-Speech)", optimizations).
+ * This library computes
+ *
+ *     Y[M,N] = X[M,K] * dequant(W)^T
+ *
+ * where
+ *   W  is N rows of K weights in Q4_0 blocks: each run of 32 weights of a row
+ *      is 18 bytes = fp16 scale d (little-endian) + 16 bytes qs, byte j of qs
+ *      holding code q[j] (low nibble) and q[j+16] (high nibble); a weight is
+ *      w = (q - 8) * d; blocks of a row are contiguous and rows follow each
+ *      other with no padding (row size K/32*18 bytes);
+ *   X  is bf16, row-major [M,K] (row stride K elements);
+ *   Y  is fp32, row-major [M,N] (row stride N elements), overwritten.
+ * Accumulation is fp32.  Results agree with the exact (float64) product to
+ * |Y - Y_exact| <= 1e-3 * sum_k |X[m,k] * w[n,k]| + 1e-6 per element; pack and
+ * dequant are bit-exact.
+ *
+ * Conventions for every entry point:
+ *   * all data pointers are DEVICE pointers owned by the caller; the library
+ *     never frees, keeps or allocates them, and allocates nothing per call;
+ *   * `stream` is a cudaStream_t (NULL = the legacy default stream); every
+ *     call is asynchronous on it and returns without a host synchronisation;
+ *   * arguments are checked on the host before anything is launched; on a
+ *     failed check nothing is launched and a status != Q4_OK is returned;
+ *   * sizes are element counts; a size of 0 is valid (see each call);
+ *   * the calling thread's current CUDA device must be an sm_100 GPU (compute
+ *     capability 10.0), else Q4_ERR_UNSUPPORTED_DEVICE.
+ * Asynchronous faults surface on the stream as for any CUDA kernel.  Kernels
+ * that wait on on-chip barriers bound every wait; a wait that runs out sets a
+ * device-side error word (q4_0_device_error) and the kernel returns early.
+ */
+#ifndef Q4_0_B200_H
+#define Q4_0_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared here so that this header needs no CUDA
+ * header. */
+typedef struct CUstream_st *q4_0_stream_t;
+
+enum {
+    Q4_OK = 0,
+    Q4_ERR_INVALID_ARG = 1,        /* null pointer, negative size, K % 32 != 0, too large */
+    Q4_ERR_MISALIGNED = 2,         /* a pointer is not 16-byte aligned */
+    Q4_ERR_UNSUPPORTED_DEVICE = 3, /* current device is not compute capability 10.0 */
+    Q4_ERR_CUDA = 4                /* a CUDA runtime call failed; see q4_0_last_cuda_error */
+};
+
+/* Device error bits reported by q4_0_device_error. */
+enum {
+    Q4_DEVERR_WAIT_TIMEOUT = 1u,   /* a bounded on-chip wait gave up; the output is incomplete */
+    Q4_DEVERR_FP16_RANGE = 2u      /* tensor-core path: an operand was beyond the fp16 range */
+};
+
+/* Largest N, K and M accepted (each dimension below 2^31). */
+#define Q4_0_MAX_DIM 2147483647LL
+
+/* Human-readable name of a status code; never NULL. */
+const char *q4_0_status_string(int status);
+
+/* The cudaError_t of the last call that returned Q4_ERR_CUDA on this thread
+ * (0 if none). */
+int q4_0_last_cuda_error(void);
+
+/* Bytes of a Q4_0 matrix of N rows by K weights: N * (K/32) * 18.  Returns -1
+ * if N < 0, K < 0 or K % 32 != 0. */
+int64_t q4_0_bytes(int64_t N, int64_t K);
+
+/* Pack 4-bit codes and fp16 scales into Q4_0 blocks (bit-exact).
+ *   codes  [N,K] uint8, row-major; only the low nibble of each byte is used;
+ *   scales [N,K/32] uint16 fp16 bit patterns, row-major (scale of block
+ *          k/32 of row n at scales[n*(K/32) + k/32]);
+ *   W      output, q4_0_bytes(N,K) bytes, layout as above.
+ * codes, scales and W must be 16-byte aligned.  K % 32 == 0.  N == 0 or
+ * K == 0 writes nothing.  The GGUF Q4_0 packing is the reading taken of the
+ * pages' "Q4_0 GGUF" (voxtral-mini-realtime-rs README, "RTF Benchmark
+ * Results"); codes are given, not derived from float weights. */
+int q4_0_pack(const uint8_t *codes, const uint16_t *scales, void *W,
+              int64_t N, int64_t K, q4_0_stream_t stream);
+
+/* Dequantize Q4_0 blocks to fp32: out[n,k] = (q - 8) * d, exact (bit-exact
+ * against any correct implementation).  W as in q4_0_pack; out [N,K] fp32
+ * row-major.  W and out 16-byte aligned.  N == 0 or K == 0 writes nothing.
+ * This is the dequantization half of the fused shader (hakusoku.com story
+ * 5135, linear ops and embeddings) on its own, for tests and utilities. */
+int q4_0_dequant(const void *W, float *out, int64_t N, int64_t K,
+                 q4_0_stream_t stream);
+
+/* Y[M,N] = X[M,K] * dequant(W)^T with fp32 accumulation, W never written out
+ * dequantized (the fused dequant+matmul of hakusoku.com story 5135, linear
+ * ops and embeddings; one Q4 matmul per decoder linear as in
+ * voxtral-mini-realtime-rs README, "Architecture Summary").
+ *   W  Q4_0 [N, K/32 blocks], X bf16 bit patterns [M,K], Y fp32 [M,N].
+ *   W, X, Y must be 16-byte aligned; K % 32 == 0; X and Y must not overlap W
+ *   or each other.
+ *   M == 0 or N == 0: nothing is done.  K == 0: Y is filled with zeros.
+ * Path: M <= 32 runs the memory-bound decode kernel (dequantization in
+ * registers); M > 32 runs the tcgen05 tensor-core kernel (tiles dequantized
+ * to fp16 in shared memory, fp32 accumulators in tensor memory), whose
+ * operands must lie in the fp16 range (|x| <= 65504, |d| <= 8188); outside
+ * it the result is not within the tolerance and Q4_DEVERR_FP16_RANGE is set
+ * in the device error word. */
+int q4_0_gemm(const void *W, const uint16_t *X, float *Y,
+              int64_t M, int64_t N, int64_t K, q4_0_stream_t stream);
+
+/* One problem of a grouped launch: Y = X * dequant(W)^T, all device
+ * pointers, same rules as q4_0_gemm. */
+typedef struct q4_0_problem {
+    const void *W;
+    const uint16_t *X;
+    float *Y;
+    int64_t M, N, K;
+} q4_0_problem;
+
+/* Largest `count` accepted by q4_0_gemm_grouped. */
+#define Q4_0_MAX_GROUP 256
+
+/* Run `count` independent problems in as few launches as possible (one
+ * persistent launch for all problems with M <= 32), so that a decoder
+ * layer's QKV, O, gate/up and down projections -- or all layers of a decode
+ * step -- stream their weights in one pass without a launch and a tail per
+ * linear (the fused QKV and gate/up projections of voxtral-mini-realtime-rs
+ * README, "TTS (Text-to-Speech)", optimizations, generalised to whole
+ * layers).  `problems` is a HOST array read during the call (it may be
+ * reused as soon as the call returns).  0 <= count <= Q4_0_MAX_GROUP.  All
+ * problems are checked before anything is launched. */
+int q4_0_gemm_grouped(const q4_0_problem *problems, int count,
+                      q4_0_stream_t stream);
+
+/* Read (and, if clear != 0, reset) the device error word of the current
+ * device: an OR of Q4_DEVERR_* bits set by kernels since the last reset.
+ * Synchronises the device.  The pages have no counterpart; this is the
+ * library's failure-detection hook. */
+int q4_0_device_error(uint32_t *flags, int clear);
+
+/* Testing knob, process-wide: force the kernel family used by q4_0_gemm and
+ * q4_0_gemm_grouped.  0 = automatic (default), 1 = portable reference-style
+ * kernel (any shape), 2 = decode kernel (M <= 32 only), 3 = tensor-core
+ * kernel.  A forced family that cannot run a given shape falls back to
+ * automatic.  The pages have no counterpart. */
+int q4_0_force_path(int path);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* Q4_0_B200_H */
