@@ -1,0 +1,220 @@
+// q4_0_api.cu -- the C ABI (include/q4_0.h): argument checks, per-device
+// set-up and the choice of kernel for each problem.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "q4_0_internal.cuh"
+
+// Device error word (one per device that loads the library): kernels OR
+// Q4_DEVERR_* bits into it; q4_0_device_error reads and clears it.
+__device__ unsigned q4_0_device_error_word = 0;
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+std::atomic<int> g_force_path{0};
+
+constexpr int kMaxDevices = 64;
+std::once_flag g_dev_once[kMaxDevices];
+q4::DeviceInfo g_dev[kMaxDevices];
+int g_dev_status[kMaxDevices];
+
+int cuda_fail(cudaError_t e) {
+    g_last_cuda_error = static_cast<int>(e);
+    return Q4_ERR_CUDA;
+}
+
+void init_device(int dev) {
+    q4::DeviceInfo &d = g_dev[dev];
+    d.device = dev;
+    cudaDeviceProp prop;
+    cudaError_t e = cudaGetDeviceProperties(&prop, dev);
+    if (e != cudaSuccess) { g_dev_status[dev] = cuda_fail(e); return; }
+    d.sm_count = prop.multiProcessorCount;
+    d.cc_major = prop.major;
+    d.cc_minor = prop.minor;
+    d.smem_optin = prop.sharedMemPerBlockOptin;
+    if (prop.major != 10 || prop.minor != 0) { g_dev_status[dev] = Q4_ERR_UNSUPPORTED_DEVICE; return; }
+    // The host-side name of a __device__ variable is not a device address:
+    // ask the runtime for this device's address of the error word.
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, q4_0_device_error_word);
+    if (e != cudaSuccess) { g_dev_status[dev] = cuda_fail(e); return; }
+    d.err = static_cast<unsigned *>(p);
+    g_dev_status[dev] = Q4_OK;
+}
+
+// Current device's info, set up once per device.
+int current_device(const q4::DeviceInfo **out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return Q4_ERR_UNSUPPORTED_DEVICE;
+    std::call_once(g_dev_once[dev], init_device, dev);
+    if (g_dev_status[dev] != Q4_OK) return g_dev_status[dev];
+    *out = &g_dev[dev];
+    return Q4_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_dims(int64_t N, int64_t K) {
+    if (N < 0 || K < 0 || N > Q4_0_MAX_DIM || K > Q4_0_MAX_DIM) return Q4_ERR_INVALID_ARG;
+    if (K % 32 != 0) return Q4_ERR_INVALID_ARG;
+    return Q4_OK;
+}
+
+int check_problem(const q4_0_problem &p) {
+    if (p.M < 0 || p.M > Q4_0_MAX_DIM) return Q4_ERR_INVALID_ARG;
+    int st = check_dims(p.N, p.K);
+    if (st != Q4_OK) return st;
+    if (p.M == 0 || p.N == 0) return Q4_OK;
+    if (!p.Y) return Q4_ERR_INVALID_ARG;
+    if (!aligned16(p.Y)) return Q4_ERR_MISALIGNED;
+    if (p.K == 0) return Q4_OK;
+    if (!p.W || !p.X) return Q4_ERR_INVALID_ARG;
+    if (!aligned16(p.W) || !aligned16(p.X)) return Q4_ERR_MISALIGNED;
+    return Q4_OK;
+}
+
+enum Path { kAuto = 0, kGeneric = 1, kDecode = 2, kTensor = 3 };
+
+int run_problems(const q4_0_problem *probs, int count, cudaStream_t s) {
+    int st = Q4_OK;
+    for (int i = 0; i < count; ++i) {
+        st = check_problem(probs[i]);
+        if (st != Q4_OK) return st;
+    }
+    bool any = false;
+    for (int i = 0; i < count; ++i) any = any || (probs[i].M > 0 && probs[i].N > 0);
+    if (!any) return Q4_OK;
+    const q4::DeviceInfo *dev = nullptr;
+    st = current_device(&dev);
+    if (st != Q4_OK) return st;
+    const int force = g_force_path.load(std::memory_order_relaxed);
+    std::vector<q4::Problem> dec, gen, ten;
+    for (int i = 0; i < count; ++i) {
+        const q4_0_problem &a = probs[i];
+        if (a.M == 0 || a.N == 0) continue;
+        if (a.K == 0) {
+            cudaError_t e = q4::launch_zero(a.Y, a.M * a.N, s);
+            if (e != cudaSuccess) return cuda_fail(e);
+            continue;
+        }
+        q4::Problem p{static_cast<const uint8_t *>(a.W), a.X, a.Y, a.M, a.N, a.K};
+        const bool dec_ok = q4::decode_supports(p);
+        const bool ten_ok = q4::prefill_supports(p);
+        if (force == kGeneric) gen.push_back(p);
+        else if (force == kDecode && dec_ok) dec.push_back(p);
+        else if (force == kTensor && ten_ok) ten.push_back(p);
+        else if (p.M <= 32 && dec_ok) dec.push_back(p);
+        else if (p.M > 32 && ten_ok) ten.push_back(p);
+        else gen.push_back(p);
+    }
+    cudaError_t e = cudaSuccess;
+    if (!dec.empty()) e = q4::launch_decode(dec.data(), static_cast<int>(dec.size()), *dev, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    for (const q4::Problem &p : ten) {
+        e = q4::launch_prefill(p, *dev, s);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    if (!gen.empty()) e = q4::launch_generic(gen.data(), static_cast<int>(gen.size()), *dev, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return Q4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *q4_0_status_string(int status) {
+    switch (status) {
+        case Q4_OK: return "Q4_OK";
+        case Q4_ERR_INVALID_ARG: return "Q4_ERR_INVALID_ARG: invalid argument (null pointer, bad size, K % 32 != 0)";
+        case Q4_ERR_MISALIGNED: return "Q4_ERR_MISALIGNED: a pointer is not 16-byte aligned";
+        case Q4_ERR_UNSUPPORTED_DEVICE: return "Q4_ERR_UNSUPPORTED_DEVICE: current device is not sm_100 (CC 10.0)";
+        case Q4_ERR_CUDA: return "Q4_ERR_CUDA: a CUDA runtime call failed";
+        default: return "unknown q4_0 status";
+    }
+}
+
+int q4_0_last_cuda_error(void) { return g_last_cuda_error; }
+
+int64_t q4_0_bytes(int64_t N, int64_t K) {
+    if (N < 0 || K < 0 || K % 32 != 0) return -1;
+    return N * (K / 32) * 18;
+}
+
+int q4_0_pack(const uint8_t *codes, const uint16_t *scales, void *W, int64_t N, int64_t K,
+              q4_0_stream_t stream) {
+    int st = check_dims(N, K);
+    if (st != Q4_OK) return st;
+    if (N == 0 || K == 0) return Q4_OK;
+    if (!codes || !scales || !W) return Q4_ERR_INVALID_ARG;
+    if (!aligned16(codes) || !aligned16(scales) || !aligned16(W)) return Q4_ERR_MISALIGNED;
+    const q4::DeviceInfo *dev = nullptr;
+    st = current_device(&dev);
+    if (st != Q4_OK) return st;
+    cudaError_t e = q4::launch_pack(codes, scales, static_cast<uint8_t *>(W), N, K,
+                                    reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? Q4_OK : cuda_fail(e);
+}
+
+int q4_0_dequant(const void *W, float *out, int64_t N, int64_t K, q4_0_stream_t stream) {
+    int st = check_dims(N, K);
+    if (st != Q4_OK) return st;
+    if (N == 0 || K == 0) return Q4_OK;
+    if (!W || !out) return Q4_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(out)) return Q4_ERR_MISALIGNED;
+    const q4::DeviceInfo *dev = nullptr;
+    st = current_device(&dev);
+    if (st != Q4_OK) return st;
+    cudaError_t e = q4::launch_dequant(static_cast<const uint8_t *>(W), out, N, K,
+                                       reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? Q4_OK : cuda_fail(e);
+}
+
+int q4_0_gemm(const void *W, const uint16_t *X, float *Y, int64_t M, int64_t N, int64_t K,
+              q4_0_stream_t stream) {
+    q4_0_problem p{W, X, Y, M, N, K};
+    return run_problems(&p, 1, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int q4_0_gemm_grouped(const q4_0_problem *problems, int count, q4_0_stream_t stream) {
+    if (count < 0 || count > Q4_0_MAX_GROUP) return Q4_ERR_INVALID_ARG;
+    if (count == 0) return Q4_OK;
+    if (!problems) return Q4_ERR_INVALID_ARG;
+    return run_problems(problems, count, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int q4_0_device_error(uint32_t *flags, int clear) {
+    if (!flags) return Q4_ERR_INVALID_ARG;
+    const q4::DeviceInfo *dev = nullptr;
+    int st = current_device(&dev);
+    if (st != Q4_OK) return st;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e);
+    unsigned v = 0;
+    e = cudaMemcpy(&v, dev->err, sizeof(v), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e);
+    *flags = v;
+    if (clear) {
+        e = cudaMemset(dev->err, 0, sizeof(unsigned));
+        if (e != cudaSuccess) return cuda_fail(e);
+        e = cudaDeviceSynchronize();
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return Q4_OK;
+}
+
+int q4_0_force_path(int path) {
+    if (path < 0 || path > 3) return Q4_ERR_INVALID_ARG;
+    g_force_path.store(path, std::memory_order_relaxed);
+    return Q4_OK;
+}
+
+}  // extern "C"

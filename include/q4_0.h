@@ -48,6 +48,12 @@
 extern "C" {
 #endif
 
+#if defined(__GNUC__)
+#define Q4_0_API __attribute__((visibility("default")))
+#else
+#define Q4_0_API
+#endif
+
 /* Same type as cudaStream_t, declared here so that this header needs no CUDA
  * header. */
 typedef struct CUstream_st *q4_0_stream_t;
@@ -70,15 +76,15 @@ enum {
 #define Q4_0_MAX_DIM 2147483647LL
 
 /* Human-readable name of a status code; never NULL. */
-const char *q4_0_status_string(int status);
+Q4_0_API const char *q4_0_status_string(int status);
 
 /* The cudaError_t of the last call that returned Q4_ERR_CUDA on this thread
  * (0 if none). */
-int q4_0_last_cuda_error(void);
+Q4_0_API int q4_0_last_cuda_error(void);
 
 /* Bytes of a Q4_0 matrix of N rows by K weights: N * (K/32) * 18.  Returns -1
  * if N < 0, K < 0 or K % 32 != 0. */
-int64_t q4_0_bytes(int64_t N, int64_t K);
+Q4_0_API int64_t q4_0_bytes(int64_t N, int64_t K);
 
 /* Pack 4-bit codes and fp16 scales into Q4_0 blocks (bit-exact).
  *   codes  [N,K] uint8, row-major; only the low nibble of each byte is used;
@@ -89,7 +95,7 @@ int64_t q4_0_bytes(int64_t N, int64_t K);
  * K == 0 writes nothing.  The GGUF Q4_0 packing is the reading taken of the
  * pages' "Q4_0 GGUF" (voxtral-mini-realtime-rs README, "RTF Benchmark
  * Results"); codes are given, not derived from float weights. */
-int q4_0_pack(const uint8_t *codes, const uint16_t *scales, void *W,
+Q4_0_API int q4_0_pack(const uint8_t *codes, const uint16_t *scales, void *W,
               int64_t N, int64_t K, q4_0_stream_t stream);
 
 /* Dequantize Q4_0 blocks to fp32: out[n,k] = (q - 8) * d, exact (bit-exact
@@ -97,7 +103,7 @@ int q4_0_pack(const uint8_t *codes, const uint16_t *scales, void *W,
  * row-major.  W and out 16-byte aligned.  N == 0 or K == 0 writes nothing.
  * This is the dequantization half of the fused shader (hakusoku.com story
  * 5135, linear ops and embeddings) on its own, for tests and utilities. */
-int q4_0_dequant(const void *W, float *out, int64_t N, int64_t K,
+Q4_0_API int q4_0_dequant(const void *W, float *out, int64_t N, int64_t K,
                  q4_0_stream_t stream);
 
 /* Y[M,N] = X[M,K] * dequant(W)^T with fp32 accumulation, W never written out
@@ -114,7 +120,7 @@ int q4_0_dequant(const void *W, float *out, int64_t N, int64_t K,
  * operands must lie in the fp16 range (|x| <= 65504, |d| <= 8188); outside
  * it the result is not within the tolerance and Q4_DEVERR_FP16_RANGE is set
  * in the device error word. */
-int q4_0_gemm(const void *W, const uint16_t *X, float *Y,
+Q4_0_API int q4_0_gemm(const void *W, const uint16_t *X, float *Y,
               int64_t M, int64_t N, int64_t K, q4_0_stream_t stream);
 
 /* One problem of a grouped launch: Y = X * dequant(W)^T, all device
@@ -138,21 +144,21 @@ typedef struct q4_0_problem {
  * layers).  `problems` is a HOST array read during the call (it may be
  * reused as soon as the call returns).  0 <= count <= Q4_0_MAX_GROUP.  All
  * problems are checked before anything is launched. */
-int q4_0_gemm_grouped(const q4_0_problem *problems, int count,
+Q4_0_API int q4_0_gemm_grouped(const q4_0_problem *problems, int count,
                       q4_0_stream_t stream);
 
 /* Read (and, if clear != 0, reset) the device error word of the current
  * device: an OR of Q4_DEVERR_* bits set by kernels since the last reset.
  * Synchronises the device.  The pages have no counterpart; this is the
  * library's failure-detection hook. */
-int q4_0_device_error(uint32_t *flags, int clear);
+Q4_0_API int q4_0_device_error(uint32_t *flags, int clear);
 
 /* Testing knob, process-wide: force the kernel family used by q4_0_gemm and
  * q4_0_gemm_grouped.  0 = automatic (default), 1 = portable reference-style
  * kernel (any shape), 2 = decode kernel (M <= 32 only), 3 = tensor-core
  * kernel.  A forced family that cannot run a given shape falls back to
  * automatic.  The pages have no counterpart. */
-int q4_0_force_path(int path);
+Q4_0_API int q4_0_force_path(int path);
 
 #ifdef __cplusplus
 }

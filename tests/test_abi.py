@@ -1,0 +1,101 @@
+"""The C-ABI library loads and exports every symbol include/q4_0.h declares,
+and its host-side argument checks answer without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "q4_0.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"Q4_0_API\s+[\w\s\*]*?\b(q4_0_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def q4():
+    import bit_weight_only_matmul_b200 as q4
+    return q4
+
+
+def test_header_lists_the_entry_points():
+    syms = declared_symbols()
+    assert "q4_0_gemm" in syms and "q4_0_pack" in syms and "q4_0_dequant" in syms
+    assert "q4_0_gemm_grouped" in syms
+
+
+def test_every_declared_symbol_is_exported(q4):
+    lib = ctypes.CDLL(q4.LIB_PATH)
+    missing = [s for s in declared_symbols() if not hasattr(lib, s)]
+    assert not missing, missing
+    assert sorted(q4.EXPORTS) == declared_symbols()
+
+
+def test_status_strings(q4):
+    for st in range(5):
+        assert q4.lib.q4_0_status_string(st)
+    assert b"unknown" in q4.lib.q4_0_status_string(99)
+
+
+def test_bytes(q4):
+    assert q4.q4_0_bytes(3072, 3072) == 5308416
+    assert q4.q4_0_bytes(1, 32) == 18
+    assert q4.q4_0_bytes(0, 64) == 0
+    assert q4.q4_0_bytes(4, 33) == -1
+    assert q4.q4_0_bytes(-1, 32) == -1
+
+
+def test_force_path_range(q4):
+    assert q4.lib.q4_0_force_path(4) == q4.Q4_ERR_INVALID_ARG
+    assert q4.lib.q4_0_force_path(-1) == q4.Q4_ERR_INVALID_ARG
+    assert q4.lib.q4_0_force_path(0) == q4.Q4_OK
+
+
+# argument checks happen before any CUDA call, so they work without a GPU
+A = 1 << 20   # a fake, 16-byte aligned address that is never dereferenced
+
+
+def test_gemm_argument_checks(q4):
+    g = q4.lib.q4_0_gemm
+    assert g(A, A, A, 1, 8, 48, None) == q4.Q4_ERR_INVALID_ARG       # K % 32
+    assert g(A, A, A, -1, 8, 64, None) == q4.Q4_ERR_INVALID_ARG      # M < 0
+    assert g(A, A, A, 1, -8, 64, None) == q4.Q4_ERR_INVALID_ARG      # N < 0
+    assert g(A, A, A, 1, 8, 1 << 31, None) == q4.Q4_ERR_INVALID_ARG  # K too large
+    assert g(None, A, A, 1, 8, 64, None) == q4.Q4_ERR_INVALID_ARG
+    assert g(A, None, A, 1, 8, 64, None) == q4.Q4_ERR_INVALID_ARG
+    assert g(A, A, None, 1, 8, 64, None) == q4.Q4_ERR_INVALID_ARG
+    assert g(A + 2, A, A, 1, 8, 64, None) == q4.Q4_ERR_MISALIGNED
+    assert g(A, A + 8, A, 1, 8, 64, None) == q4.Q4_ERR_MISALIGNED
+    assert g(A, A, A + 4, 1, 8, 64, None) == q4.Q4_ERR_MISALIGNED
+    # empty problems are valid no-ops and need no device
+    assert g(None, None, None, 0, 8, 64, None) == q4.Q4_OK
+    assert g(None, None, None, 4, 0, 64, None) == q4.Q4_OK
+
+
+def test_pack_dequant_argument_checks(q4):
+    p, d = q4.lib.q4_0_pack, q4.lib.q4_0_dequant
+    assert p(A, A, A, 4, 40, None) == q4.Q4_ERR_INVALID_ARG
+    assert p(None, A, A, 4, 64, None) == q4.Q4_ERR_INVALID_ARG
+    assert p(A + 1, A, A, 4, 64, None) == q4.Q4_ERR_MISALIGNED
+    assert p(A, A, A + 2, 4, 64, None) == q4.Q4_ERR_MISALIGNED
+    assert p(None, None, None, 0, 64, None) == q4.Q4_OK
+    assert p(None, None, None, 4, 0, None) == q4.Q4_OK
+    assert d(A, A, 4, 31, None) == q4.Q4_ERR_INVALID_ARG
+    assert d(A, None, 4, 64, None) == q4.Q4_ERR_INVALID_ARG
+    assert d(A, A + 8, 4, 64, None) == q4.Q4_ERR_MISALIGNED
+    assert d(None, None, 0, 64, None) == q4.Q4_OK
+
+
+def test_grouped_argument_checks(q4):
+    gg = q4.lib.q4_0_gemm_grouped
+    probs = q4.make_problems([(A, A, A, 1, 8, 64), (A, A, A, 1, 8, 40)])
+    assert gg(probs, 2, None) == q4.Q4_ERR_INVALID_ARG        # second problem bad: nothing launched
+    assert gg(probs, -1, None) == q4.Q4_ERR_INVALID_ARG
+    assert gg(probs, q4.Q4_0_MAX_GROUP + 1, None) == q4.Q4_ERR_INVALID_ARG
+    assert gg(None, 3, None) == q4.Q4_ERR_INVALID_ARG
+    assert gg(None, 0, None) == q4.Q4_OK
+    empty = q4.make_problems([(None, None, None, 0, 8, 64)])
+    assert gg(empty, 1, None) == q4.Q4_OK

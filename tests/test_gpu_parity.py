@@ -1,0 +1,219 @@
+"""GPU parity: the CUDA library, called through its C ABI, against the
+float64 oracle on the same seeded inputs.
+
+Bars: pack and dequant bit-exact; GEMM within |Y - Y_exact| <= 1e-3 *
+sum_k |x_k w_k| + 1e-6 per element (the method's stated tolerance)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests.gpu_helpers import (build_workload, check_built, check_gemm, dev, host_u16, no_device_error,
+                               pack_on_gpu)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def q4():
+    import bit_weight_only_matmul_b200 as q4
+    torch.cuda.init()
+    q4.q4_0_force_path(0)
+    yield q4
+    q4.q4_0_force_path(0)
+
+
+@pytest.fixture(autouse=True)
+def _clean_error_word(q4):
+    q4.q4_0_device_error(clear=True)
+    yield
+    no_device_error(q4)
+
+
+def rand_inputs(rng, M, N, K, x_sigma=1.0):
+    codes = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
+    scales = (np.abs(rng.standard_normal(size=(N, K // 32))) * 0.002 + 1e-4).astype(np.float16).view(np.uint16)
+    X = workloads.fp32_to_bf16_bits(rng.standard_normal(size=(M, K)).astype(np.float32) * np.float32(x_sigma))
+    return codes, scales, X
+
+
+# --------------------------------------------------------------------------- pack / dequant
+
+@pytest.mark.parametrize("N,K", [(1, 32), (3, 64), (5, 96), (64, 3072), (17, 8192), (33, 5120), (7, 288)])
+def test_pack_bit_exact(q4, N, K):
+    rng = np.random.default_rng(N * 131 + K)
+    codes = rng.integers(0, 256, size=(N, K), dtype=np.uint8)     # high nibble must be ignored
+    scales = rng.integers(0, 65536, size=(N, K // 32), dtype=np.uint16)
+    W = pack_on_gpu(q4, codes, scales).cpu().numpy()
+    assert np.array_equal(W, oracle.get().pack(codes & 15, scales).reshape(-1))
+
+
+@pytest.mark.parametrize("N,K", [(1, 32), (4, 64), (9, 160), (64, 3072), (5, 8192)])
+def test_dequant_bit_exact(q4, N, K):
+    rng = np.random.default_rng(N * 7 + K)
+    W = rng.integers(0, 256, size=(N, K // 32 * 18), dtype=np.uint8)   # every scale bit pattern, NaN/Inf too
+    out = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    q4.q4_0_dequant(dev(W), out, N, K)
+    got = out.cpu().numpy()
+    ref = oracle.get().dequant_f32(W, N, K)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+
+
+def test_pack_dequant_roundtrip_config_shape(q4):
+    lin = workloads.workload("gemv").linears[0]
+    codes, scales = lin.codes(), lin.scales()
+    W = pack_on_gpu(q4, codes, scales)
+    out = torch.empty((lin.N, lin.K), dtype=torch.float32, device="cuda")
+    q4.q4_0_dequant(W, out, lin.N, lin.K)
+    ref = oracle.get().dequant_f32(oracle.get().pack(codes, scales), lin.N, lin.K)
+    assert np.array_equal(out.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+# --------------------------------------------------------------------------- GEMM, small shapes
+
+def run_gemm(q4, M, N, K, seed=0, path=0, x_sigma=1.0):
+    rng = np.random.default_rng(seed * 1000003 + M * 10007 + N * 101 + K)
+    codes, scales, X = rand_inputs(rng, M, N, K, x_sigma)
+    W = pack_on_gpu(q4, codes, scales)
+    Y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    q4.q4_0_force_path(path)
+    try:
+        q4.q4_0_gemm(W, dev(X), Y, M, N, K)
+    finally:
+        q4.q4_0_force_path(0)
+    Y_or, B_or = oracle.get().gemm(oracle.get().pack(codes, scales), X, M, N, K)
+    return check_gemm(Y.cpu().numpy(), Y_or, B_or, f"M={M} N={N} K={K} path={path}")
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 7, 8, 9, 16, 17, 31, 32])
+@pytest.mark.parametrize("N,K", [(17, 256), (100, 1280), (129, 3072)])
+def test_decode_path(q4, M, N, K):
+    run_gemm(q4, M, N, K)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 256), (2, 16, 512), (1, 3, 8192), (32, 33, 2048), (5, 257, 768)])
+def test_decode_path_ragged(q4, M, N, K):
+    run_gemm(q4, M, N, K)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 5, 32), (3, 9, 96), (2, 31, 160), (8, 64, 288), (33, 40, 64),
+                                   (64, 17, 256), (100, 24, 320)])
+def test_generic_shapes(q4, M, N, K):
+    run_gemm(q4, M, N, K)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 100, 1024), (4, 65, 3072), (32, 48, 512)])
+def test_forced_generic_matches(q4, M, N, K):
+    run_gemm(q4, M, N, K, path=q4.PATH_GENERIC)
+
+
+@pytest.mark.parametrize("M,N,K", [(33, 64, 512), (64, 128, 1024), (128, 256, 3072), (200, 96, 320)])
+def test_prefill_shapes(q4, M, N, K):
+    run_gemm(q4, M, N, K, x_sigma=0.5)
+
+
+def test_outlier_rows_decode(q4):
+    # 3 of 32 rows of X scaled x8, as in the concurrent-decode workload
+    M, N, K = 32, 96, 1024
+    rng = np.random.default_rng(5)
+    codes, scales, _ = rand_inputs(rng, M, N, K)
+    X = workloads.gen_x(M, K, seed=77, outlier_rows=3)
+    W = pack_on_gpu(q4, codes, scales)
+    Y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    q4.q4_0_gemm(W, dev(X), Y, M, N, K)
+    Y_or, B_or = oracle.get().gemm(oracle.get().pack(codes, scales), X, M, N, K)
+    check_gemm(Y.cpu().numpy(), Y_or, B_or, "outliers")
+
+
+def test_special_structures(q4):
+    """All-8 codes give exactly zero; one off-centre nibble gives (c-8)*d*x."""
+    M, N, K = 2, 40, 512
+    o = oracle.get()
+    rng = np.random.default_rng(9)
+    X = workloads.fp32_to_bf16_bits(rng.standard_normal(size=(M, K)).astype(np.float32) * 50)
+    scales = np.full((N, K // 32), np.float16(3.5).view(np.uint16), np.uint16)
+    codes = np.full((N, K), 8, np.uint8)
+    for path in (0, q4.PATH_GENERIC):
+        Y = torch.full((M, N), 1.0, dtype=torch.float32, device="cuda")
+        q4.q4_0_force_path(path)
+        q4.q4_0_gemm(pack_on_gpu(q4, codes, scales), dev(X), Y, M, N, K)
+        q4.q4_0_force_path(0)
+        assert torch.count_nonzero(Y).item() == 0
+    codes[7, 300] = 13
+    codes[39, 511] = 0
+    Y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    q4.q4_0_gemm(pack_on_gpu(q4, codes, scales), dev(X), Y, M, N, K)
+    Y_or, B_or = o.gemm(o.pack(codes, scales), X, M, N, K)
+    check_gemm(Y.cpu().numpy(), Y_or, B_or, "single nibble")
+
+
+# --------------------------------------------------------------------------- empty inputs
+
+def test_empty_problems(q4):
+    Y = torch.full((3, 5), 7.0, device="cuda")
+    q4.q4_0_gemm(None, None, Y, 0, 5, 64)
+    q4.q4_0_gemm(None, None, Y, 3, 0, 64)
+    assert torch.all(Y == 7.0)
+    q4.q4_0_gemm(None, None, Y, 3, 5, 0)      # empty sum: zeros
+    torch.cuda.synchronize()
+    assert torch.all(Y == 0.0)
+
+
+# --------------------------------------------------------------------------- grouped launch
+
+def test_grouped_mixed_shapes(q4):
+    o = oracle.get()
+    rng = np.random.default_rng(21)
+    shapes = [(1, 70, 512), (2, 33, 3072), (32, 40, 1024), (1, 5, 96), (48, 64, 256), (0, 5, 64), (3, 9, 0),
+              (9, 300, 2048)]
+    probs, refs, Ys = [], [], []
+    for (M, N, K) in shapes:
+        if M == 0 or K == 0:
+            Y = torch.full((max(M, 1), N), 5.0, device="cuda")
+            probs.append((None, None, Y, M, N, K))
+            refs.append(None)
+            Ys.append(Y)
+            continue
+        codes, scales, X = rand_inputs(rng, M, N, K)
+        Y = torch.full((M, N), float("nan"), device="cuda")
+        probs.append((pack_on_gpu(q4, codes, scales), dev(X), Y, M, N, K))
+        refs.append(o.gemm(o.pack(codes, scales), X, M, N, K))
+        Ys.append(Y)
+    q4.q4_0_gemm_grouped(probs)
+    for (M, N, K), Y, ref in zip(shapes, Ys, refs):
+        if ref is None:
+            assert torch.all(Y == (5.0 if M == 0 else 0.0))
+        else:
+            check_gemm(Y.cpu().numpy(), ref[0], ref[1], f"grouped {M}x{N}x{K}")
+
+
+def test_non_default_stream(q4):
+    M, N, K = 2, 64, 1024
+    rng = np.random.default_rng(3)
+    codes, scales, X = rand_inputs(rng, M, N, K)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        W = pack_on_gpu(q4, codes, scales)
+        Y = torch.empty((M, N), device="cuda")
+        q4.q4_0_gemm(W, dev(X), Y, M, N, K)
+    s.synchronize()
+    o = oracle.get()
+    Y_or, B_or = o.gemm(o.pack(codes, scales), X, M, N, K)
+    check_gemm(Y.cpu().numpy(), Y_or, B_or, "side stream")
+
+
+# --------------------------------------------------------------------------- workload shapes
+
+def test_gemv_workload_full(q4):
+    b = build_workload(q4, workloads.workload("gemv"), full_oracle=True)
+    q4.q4_0_gemm_grouped(b.problems())
+    check_built(b, "gemv")
+
+
+def test_layer_workload_full(q4):
+    b = build_workload(q4, workloads.workload("layer"), full_oracle=True)
+    q4.q4_0_gemm_grouped(b.problems())
+    check_built(b, "layer")
