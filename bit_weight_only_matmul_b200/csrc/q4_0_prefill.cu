@@ -1,13 +1,503 @@
-// q4_0_prefill.cu -- tensor-core path for M > 32 (placeholder until the
-// tcgen05 kernel lands: no problem is routed here).
+// q4_0_prefill.cu -- the tensor-core path for M > 32 (prefill, the adapter,
+// batched requests): a persistent, warp-specialised tcgen05 kernel.
+//
+// The pages run the adapter (reshape to width 5120, then 3072) and the
+// decoder linears over all prompt/audio frames at once
+// (voxtral-mini-realtime-rs (Shannon-Prime fork) README, "Architecture";
+// hakusoku.com story 5135, architecture); with thousands of rows of X this
+// is a dense contraction, so it belongs on the 5th-generation tensor cores.
+//
+// Tile: 128 weight rows (n) x 256 activation rows (m), D = W_tile * X_tile^T
+// accumulated in fp32 in tensor memory (128 lanes x 256 columns).
+//   * A operand = the weight tile, dequantized by four warps straight into
+//     tensor memory as fp16 (q - 8) * d: the raw Q4_0 bytes arrive by TMA
+//     (128 rows x 144 bytes = 256 k per load), each thread turns its row's
+//     blocks into fp16 pairs and writes them with tcgen05.st;
+//   * B operand = the activation tile, loaded by TMA as bf16 into the
+//     128-byte-swizzled K-major layout the MMA reads, then converted to fp16
+//     in place by eight warps;
+//   * one thread issues tcgen05.mma (kind::f16, M=128, N=256, K=16), four per
+//     64-k stage, and signals stage release with tcgen05.commit;
+//   * four epilogue warps drain the accumulator with tcgen05.ld; lane = weight
+//     row, column = activation row, so each store of a column is one
+//     contiguous 128-byte run of Y[m, n0..n0+31].
+// fp16 operands: a weight (q - 8) * d is rounded once to fp16 (relative error
+// <= 2^-11, inside the 1e-3 tolerance of the method); X is exact in fp16 in
+// the normal range.  Both must lie within the fp16 range (|x| <= 65504,
+// |d| <= 8188): beyond it the products overflow to +-inf.  Inside each block
+// of 32 the k order is permuted identically for both operands (positions 1
+// and 2 of every 4 swapped), which lets the dequantization emit the nibble
+// pairs in the order the packed bytes hold them.
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include <cstring>
+#include <mutex>
+
 #include "q4_0_internal.cuh"
+
+namespace {
+
+using namespace q4dev;
+
+constexpr int kTileN = 128;                    // weight rows per tile (MMA M)
+constexpr int kTileM = 256;                    // activation rows per tile (MMA N)
+constexpr int kStageK = 64;                    // k per operand stage (one 128-byte swizzle row)
+constexpr int kRawK = 256;                     // k per raw weight load (8 blocks = 144 bytes)
+static_assert(kRawK == 4 * kStageK, "a raw weight load feeds four operand stages");
+constexpr int kXStages = 4;
+constexpr int kRawStages = 2;
+constexpr int kAStages = 4;                    // A buffers in tensor memory
+constexpr int kXStageBytes = kTileM * 128;     // 32 KB
+constexpr int kRawRowBytes = 144;
+constexpr int kRawStageBytes = kTileN * kRawRowBytes;   // 18 KB
+constexpr int kTmemCols = 512;
+constexpr int kDCol = 0;                       // accumulator columns [0, 256)
+constexpr int kACol = 256;                     // A buffers: 32 columns each
+
+constexpr int kWarpTMA = 0, kWarpMMA = 1;
+constexpr int kWarpDeq0 = 2, kNumDeq = 4;      // warps 2..5
+constexpr int kWarpCvt0 = 6, kNumCvt = 8;      // warps 6..13
+constexpr int kWarpEpi0 = 14, kNumEpi = 4;     // warps 14..17
+constexpr int kThreads = 32 * (kWarpEpi0 + kNumEpi);   // 576
+
+struct alignas(64) PrefillParams {
+    CUtensorMap tmap_x;    // bf16 [M, K], box 64 x 256, 128-byte swizzle
+    CUtensorMap tmap_w;    // uint8 [N, K/32*18], box 144 x 128
+    float *Y;
+    unsigned *err;
+    int M, N, K;
+    int tiles_n, tiles_m;
+};
+
+struct Smem {
+    uint8_t x[kXStages][kXStageBytes];        // 1024-byte aligned (swizzle atoms)
+    uint8_t raw[kRawStages][kRawStageBytes];
+    uint64_t x_full[kXStages], x_conv[kXStages], x_empty[kXStages];
+    uint64_t raw_full[kRawStages], raw_empty[kRawStages];
+    uint64_t a_full[kAStages], a_empty[kAStages];
+    uint64_t d_full, d_empty, mma_done;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+// ---------------------------------------------------------------- PTX wrappers
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16, fp32 accumulate.
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_st_32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+        "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+        "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_ld_32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    #pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row atoms of
+// 1024 bytes stacked along the row dimension.
+__device__ __forceinline__ uint64_t sw128_desc(const void *base) {
+    const uint64_t addr = smem_addr(base);
+    return ((addr >> 4) & 0x3FFFull) | (1ull << 16) | (uint64_t(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor: fp16 x fp16 -> fp32, both K-major, M=128, N=256.
+constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | (uint32_t(kTileM >> 3) << 17) |
+                            (uint32_t(kTileN >> 4) << 24);
+
+// Bounded wait that also gives up when another role has aborted.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, Smem &S, unsigned *err) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 0) {
+            if (*reinterpret_cast<volatile int *>(&S.abort_flag)) return false;
+            if (global_ns() - t0 > kWaitLimitNs) {
+                atomicOr(err, (unsigned)Q4_DEVERR_WAIT_TIMEOUT);
+                *reinterpret_cast<volatile int *>(&S.abort_flag) = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- dequantization
+
+// fp16 pairs of (q - 8) * d for one qs word v (bytes 4w .. 4w+3 of a block):
+//   c[0] = elements (4w, 4w+2), c[1] = (4w+1, 4w+3)        (low nibbles)
+//   c[2] = elements (4w+16, 4w+18), c[3] = (4w+17, 4w+19)  (high nibbles)
+// 0x6400 is fp16 1024 (10 fraction bits): 1024 + q and 1024 + 16q are exact,
+// and so are (1024 + q) - 1032 and (1024 + 16q) / 16 - 72 = q - 8; the only
+// rounding is the final product with d.
+__device__ __forceinline__ void dequant_word(uint32_t v, uint32_t d2, uint32_t (&c)[4]) {
+    const uint32_t v8 = v >> 8;
+    const __half2 k1032 = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
+    const __half2 k16th = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
+    const __half2 km72 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));
+    const __half2 d = *reinterpret_cast<const __half2 *>(&d2);
+    uint32_t t[4] = {and_or(v, 0x000F000Fu, 0x64006400u), and_or(v8, 0x000F000Fu, 0x64006400u),
+                     and_or(v, 0x00F000F0u, 0x64006400u), and_or(v8, 0x00F000F0u, 0x64006400u)};
+    __half2 r0 = __hmul2(__hsub2(*reinterpret_cast<__half2 *>(&t[0]), k1032), d);
+    __half2 r1 = __hmul2(__hsub2(*reinterpret_cast<__half2 *>(&t[1]), k1032), d);
+    __half2 r2 = __hmul2(__hfma2(*reinterpret_cast<__half2 *>(&t[2]), k16th, km72), d);
+    __half2 r3 = __hmul2(__hfma2(*reinterpret_cast<__half2 *>(&t[3]), k16th, km72), d);
+    c[0] = *reinterpret_cast<uint32_t *>(&r0);
+    c[1] = *reinterpret_cast<uint32_t *>(&r1);
+    c[2] = *reinterpret_cast<uint32_t *>(&r2);
+    c[3] = *reinterpret_cast<uint32_t *>(&r3);
+}
+
+// Block i (0..7) of a 144-byte raw row held in 36 registers: the fp16 scale
+// bits and the four qs words.
+__device__ __forceinline__ void block_words(const uint32_t (&raw)[36], int i, uint32_t &dbits, uint32_t (&q)[4]) {
+    const int b = 18 * i;          // byte offset of the block
+    const int w = b >> 2;
+    if ((i & 1) == 0) {            // block starts 4-byte aligned: d = low half of raw[w]
+        dbits = raw[w] & 0xFFFFu;
+        #pragma unroll
+        for (int j = 0; j < 4; ++j) q[j] = prmt(raw[w + j], raw[w + j + 1], 0x5432u);
+    } else {                       // block starts at 2 mod 4: d = high half, qs aligned
+        dbits = raw[w] >> 16;
+        #pragma unroll
+        for (int j = 0; j < 4; ++j) q[j] = raw[w + 1 + j];
+    }
+}
+
+// ---------------------------------------------------------------- the kernel
+
+__global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ PrefillParams P) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem &S = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tiles = P.tiles_n * P.tiles_m;
+    const int ksteps = P.K / kStageK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kXStages; ++s) {
+            mbar_init(&S.x_full[s], 1);
+            mbar_init(&S.x_conv[s], kNumCvt);
+            mbar_init(&S.x_empty[s], 1);
+        }
+        for (int s = 0; s < kRawStages; ++s) {
+            mbar_init(&S.raw_full[s], 1);
+            mbar_init(&S.raw_empty[s], kNumDeq);
+        }
+        for (int s = 0; s < kAStages; ++s) {
+            mbar_init(&S.a_full[s], kNumDeq);
+            mbar_init(&S.a_empty[s], 1);
+        }
+        mbar_init(&S.d_full, 1);
+        mbar_init(&S.d_empty, kNumEpi);
+        mbar_init(&S.mma_done, 1);
+        S.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kWarpMMA) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&S.tmem_base)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+
+    if (warp == kWarpTMA) {
+        if (lane == 0) {
+            uint32_t xc = 0, rc = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                const int n0 = (t % P.tiles_n) * kTileN, m0 = (t / P.tiles_n) * kTileM;
+                for (int ks = 0; ks < ksteps && ok; ++ks) {
+                    if ((ks & 3) == 0) {
+                        const int s = rc % kRawStages;
+                        if (!(ok = wait_or_abort(&S.raw_empty[s], ((rc / kRawStages) & 1) ^ 1, S, P.err))) break;
+                        mbar_arrive_expect_tx(&S.raw_full[s], kRawStageBytes);
+                        tma_load_2d(S.raw[s], &P.tmap_w, (ks >> 2) * kRawRowBytes, n0, &S.raw_full[s]);
+                        ++rc;
+                    }
+                    const int s = xc % kXStages;
+                    if (!(ok = wait_or_abort(&S.x_empty[s], ((xc / kXStages) & 1) ^ 1, S, P.err))) break;
+                    mbar_arrive_expect_tx(&S.x_full[s], kXStageBytes);
+                    tma_load_2d(S.x[s], &P.tmap_x, ks * kStageK, m0, &S.x_full[s]);
+                    ++xc;
+                }
+            }
+            if (!ok) {   // let the loads already issued land (bounded) before the CTA can exit
+                for (uint32_t i = 0; i < kXStages && i < xc; ++i) {
+                    const uint32_t c = xc - 1 - i;
+                    mbar_wait(&S.x_full[c % kXStages], (c / kXStages) & 1, P.err);
+                }
+                for (uint32_t i = 0; i < kRawStages && i < rc; ++i) {
+                    const uint32_t c = rc - 1 - i;
+                    mbar_wait(&S.raw_full[c % kRawStages], (c / kRawStages) & 1, P.err);
+                }
+            }
+        }
+    } else if (warp == kWarpMMA) {
+        if (lane == 0) {
+            uint32_t xc = 0, ac = 0, dc = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++dc) {
+                if (!(ok = wait_or_abort(&S.d_empty, (dc & 1) ^ 1, S, P.err))) break;
+                tc_fence_after();
+                for (int ks = 0; ks < ksteps; ++ks) {
+                    const int sx = xc % kXStages, sa = ac % kAStages;
+                    if (!(ok = wait_or_abort(&S.x_conv[sx], (xc / kXStages) & 1, S, P.err))) break;
+                    if (!(ok = wait_or_abort(&S.a_full[sa], (ac / kAStages) & 1, S, P.err))) break;
+                    tc_fence_after();
+                    const uint64_t bdesc = sw128_desc(S.x[sx]);
+                    #pragma unroll
+                    for (int j = 0; j < 4; ++j)   // K = 16 per MMA: +8 tensor-memory columns, +32 bytes
+                        tc_mma_ts(tmem + kDCol, tmem + kACol + 32 * sa + 8 * j, bdesc + 2 * j, kIdesc,
+                                  (ks | j) != 0);
+                    tc_commit(&S.x_empty[sx]);
+                    tc_commit(&S.a_empty[sa]);
+                    ++xc;
+                    ++ac;
+                }
+                if (ok) tc_commit(&S.d_full);
+            }
+            // every MMA issued so far has completed once this commit arrives
+            tc_commit(&S.mma_done);
+            wait_or_abort(&S.mma_done, 0, S, P.err) || mbar_wait(&S.mma_done, 0, P.err);
+        }
+    } else if (warp >= kWarpDeq0 && warp < kWarpDeq0 + kNumDeq) {
+        const int quad = warp & 3;   // tensor-memory lanes [32*quad, 32*quad + 32)
+        const int row = 32 * quad + lane;
+        uint32_t rc = 0, ac = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            for (int ks = 0; ks < ksteps && ok; ks += 4) {
+                const int s = rc % kRawStages;
+                if (!(ok = wait_or_abort(&S.raw_full[s], (rc / kRawStages) & 1, S, P.err))) break;
+                uint32_t raw[36];
+                const uint4 *src = reinterpret_cast<const uint4 *>(S.raw[s] + row * kRawRowBytes);
+                #pragma unroll
+                for (int i = 0; i < 9; ++i) {
+                    const uint4 v = src[i];
+                    raw[4 * i] = v.x; raw[4 * i + 1] = v.y; raw[4 * i + 2] = v.z; raw[4 * i + 3] = v.w;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.raw_empty[s]);
+                ++rc;
+                #pragma unroll
+                for (int sub = 0; sub < 4; ++sub) {      // 64 k = blocks 2*sub, 2*sub+1
+                    const int sa = ac % kAStages;
+                    if (!(ok = wait_or_abort(&S.a_empty[sa], ((ac / kAStages) & 1) ^ 1, S, P.err))) break;
+                    tc_fence_after();
+                    uint32_t cols[32];
+                    #pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t dbits, q[4];
+                        block_words(raw, 2 * sub + h, dbits, q);
+                        const uint32_t d2 = dbits | (dbits << 16);
+                        #pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            uint32_t c[4];
+                            dequant_word(q[w], d2, c);
+                            cols[16 * h + 2 * w] = c[0];
+                            cols[16 * h + 2 * w + 1] = c[1];
+                            cols[16 * h + 8 + 2 * w] = c[2];
+                            cols[16 * h + 8 + 2 * w + 1] = c[3];
+                        }
+                    }
+                    tc_st_32(tmem + (uint32_t(32 * quad) << 16) + kACol + 32 * sa, cols);
+                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.a_full[sa]);
+                    ++ac;
+                }
+            }
+        }
+    } else if (warp >= kWarpCvt0 && warp < kWarpCvt0 + kNumCvt) {
+        const int row = 32 * (warp - kWarpCvt0) + lane;   // activation row within the tile
+        uint32_t xc = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            for (int ks = 0; ks < ksteps; ++ks) {
+                const int s = xc % kXStages;
+                if (!(ok = wait_or_abort(&S.x_full[s], (xc / kXStages) & 1, S, P.err))) break;
+                uint8_t *rp = S.x[s] + row * 128;
+                #pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    // rotate the chunk order by row so that 8 consecutive rows hit 8 different bank groups
+                    uint4 *p = reinterpret_cast<uint4 *>(rp + 16 * ((c + row) & 7));
+                    const uint4 v = *p;
+                    // bf16 (x0..x7) -> fp16 pairs (x0,x2) (x1,x3) (x4,x6) (x5,x7)
+                    const float f0 = __uint_as_float(v.x << 16), f1 = __uint_as_float(v.x & 0xFFFF0000u);
+                    const float f2 = __uint_as_float(v.y << 16), f3 = __uint_as_float(v.y & 0xFFFF0000u);
+                    const float f4 = __uint_as_float(v.z << 16), f5 = __uint_as_float(v.z & 0xFFFF0000u);
+                    const float f6 = __uint_as_float(v.w << 16), f7 = __uint_as_float(v.w & 0xFFFF0000u);
+                    __half2 h0 = __floats2half2_rn(f0, f2), h1 = __floats2half2_rn(f1, f3);
+                    __half2 h2 = __floats2half2_rn(f4, f6), h3 = __floats2half2_rn(f5, f7);
+                    uint4 o;
+                    o.x = *reinterpret_cast<uint32_t *>(&h0);
+                    o.y = *reinterpret_cast<uint32_t *>(&h1);
+                    o.z = *reinterpret_cast<uint32_t *>(&h2);
+                    o.w = *reinterpret_cast<uint32_t *>(&h3);
+                    *p = o;
+                }
+                // make the generic-proxy writes visible to the tensor core (async proxy)
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.x_conv[s]);
+                ++xc;
+            }
+        }
+    } else {   // epilogue warps
+        const int quad = warp & 3;
+        uint32_t dc = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++dc) {
+            if (!wait_or_abort(&S.d_full, dc & 1, S, P.err)) break;
+            tc_fence_after();
+            const int n0 = (t % P.tiles_n) * kTileN, m0 = (t / P.tiles_n) * kTileM;
+            const int n = n0 + 32 * quad + lane;
+            #pragma unroll 1
+            for (int c = 0; c < kTileM / 32; ++c) {
+                float v[32];
+                tc_ld_32(tmem + (uint32_t(32 * quad) << 16) + kDCol + 32 * c, v);
+                const int mb = m0 + 32 * c;
+                if (n < P.N) {
+                    #pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (mb + j < P.M) P.Y[static_cast<int64_t>(mb + j) * P.N + n] = v[j];
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.d_empty);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMMA) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                 const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled get_encoder() {
+    static EncodeTiled fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(p);
+    });
+    return fn;
+}
+
+constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+
+}  // namespace
 
 namespace q4 {
 
-bool prefill_supports(const Problem &) { return false; }
+bool prefill_supports(const Problem &p) {
+    return p.M >= 1 && p.N >= 1 && p.K >= 256 && p.K % 256 == 0 && p.M < (1LL << 31) && p.N < (1LL << 31) &&
+           p.K < (1LL << 31) && (reinterpret_cast<uintptr_t>(p.W) & 15) == 0 &&
+           (reinterpret_cast<uintptr_t>(p.X) & 15) == 0 && get_encoder() != nullptr;
+}
 
-cudaError_t launch_prefill(const Problem &, const DeviceInfo &, cudaStream_t) {
-    return cudaErrorNotSupported;
+cudaError_t launch_prefill(const Problem &p, const DeviceInfo &dev, cudaStream_t s) {
+    EncodeTiled enc = get_encoder();
+    if (!enc) return cudaErrorNotSupported;
+    PrefillParams local;
+    std::memset(&local, 0, sizeof(local));
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.K), static_cast<cuuint64_t>(p.M)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.K) * 2};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(kStageK), static_cast<cuuint32_t>(kTileM)};
+        const cuuint32_t estr[2] = {1, 1};
+        if (enc(&local.tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(p.X), dims, strides, box,
+                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    {
+        const int64_t row_bytes = p.K / 32 * 18;
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(p.N)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(kRawRowBytes), static_cast<cuuint32_t>(kTileN)};
+        const cuuint32_t estr[2] = {1, 1};
+        if (enc(&local.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(p.W), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    local.Y = p.Y;
+    local.err = dev.err;
+    local.M = static_cast<int>(p.M);
+    local.N = static_cast<int>(p.N);
+    local.K = static_cast<int>(p.K);
+    local.tiles_n = static_cast<int>((p.N + kTileN - 1) / kTileN);
+    local.tiles_m = static_cast<int>((p.M + kTileM - 1) / kTileM);
+    static int configured_device = -1;
+    if (configured_device != dev.device) {
+        cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kSmemBytes));
+        if (e != cudaSuccess) return e;
+        configured_device = dev.device;
+    }
+    const int tiles = local.tiles_n * local.tiles_m;
+    const int grid = tiles < dev.sm_count ? tiles : dev.sm_count;
+    prefill_kernel<<<grid, kThreads, kSmemBytes, s>>>(local);
+    return cudaGetLastError();
 }
 
 }  // namespace q4

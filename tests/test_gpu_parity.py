@@ -217,3 +217,15 @@ def test_layer_workload_full(q4):
     b = build_workload(q4, workloads.workload("layer"), full_oracle=True)
     q4.q4_0_gemm_grouped(b.problems())
     check_built(b, "layer")
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 128, 256), (300, 200, 512), (33, 1, 256), (512, 384, 2048)])
+def test_tensor_core_path(q4, M, N, K):
+    run_gemm(q4, M, N, K, x_sigma=0.5)
+
+
+@pytest.mark.parametrize("name", ["adapter", "qkv_prefill"])
+def test_prefill_workload_sampled(q4, name):
+    b = build_workload(q4, workloads.workload(name), samples=2000)
+    q4.q4_0_gemm_grouped(b.problems())
+    check_built(b, name)
