@@ -1,0 +1,466 @@
+"""Benchmark of the Q4_0 dequant-matmul hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One JSON line on rank 0.  A *step* is one pass of the hot path over one batch
+of synthetic input.  The default workload is one synthetic decoder layer of
+the Voxtral 4B decoder at M=1 (fused QKV N=5120, O N=3072, fused gate/up
+N=16384, all K=3072, and down K=8192, N=3072): the four Q4_0 GEMMs of a token
+step, issued as one grouped launch.  Five independently seeded copies of the
+layer's weights (283 MB, more than twice the 126 MB L2) rotate from step to
+step, so every step streams its weights from HBM.
+
+The metric is effective HBM bandwidth: algorithmic bytes (every Q4_0 weight
+byte once + X and Y once) / time.  Other workloads (--workload): gemv, layer,
+cfg_decode (M=2, 26 layers), concurrent (M=32, 26 layers) in GB/s; adapter,
+qkv_prefill (M=4096) in TFLOP/s.
+
+N > 1 (torchrun, one process per GPU): every rank runs an independent
+replica of the workload (the path has no exchange step); time is the max over
+ranks and the value is the work of all ranks over that time (weak scaling).
+
+--impl reference times the float64 CPU oracle on the same workload (a
+bounded sample of each step, scaled to the metric's unit) on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "Q4_0 dequant-matmul HBM GB/s (M=1,2) and TFLOP/s (M>=64), % of B200 roofline"
+L2_BYTES = 126 * 2**20
+DEFAULT_WORKLOAD = "layer"
+
+# kernel that dominates each workload, and the source file it lives in
+DOMINANT = {
+    "gemv": ("decode_kernel", "q4_0_decode.cu"),
+    "layer": ("decode_kernel", "q4_0_decode.cu"),
+    "cfg_decode": ("decode_kernel", "q4_0_decode.cu"),
+    "concurrent": ("decode_kernel", "q4_0_decode.cu"),
+    "adapter": ("prefill_kernel", "q4_0_prefill.cu"),
+    "qkv_prefill": ("prefill_kernel", "q4_0_prefill.cu"),
+}
+TENSOR_WORKLOADS = ("adapter", "qkv_prefill")
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# --------------------------------------------------------------------------- helpers
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def source_sha(fname: str) -> str:
+    with open(os.path.join(ROOT, "bit_weight_only_matmul_b200", "csrc", fname), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, or None when absent or when the kernel source changed since."""
+    kernel, src = DOMINANT[workload]
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("source_sha256") != source_sha(src):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+# --------------------------------------------------------------------------- our implementation
+
+class GpuWorkload:
+    """A workload resident in HBM: packed Q4_0 weights (packed on the GPU by
+    q4_0_pack from seeded codes and scales), activations and outputs, in
+    `copies` independently seeded replicas."""
+
+    def __init__(self, q4, wl: workloads.Workload, copies: int, seed: int):
+        import torch
+        self.wl = wl
+        self.sets = []
+        for c in range(copies):
+            probs = []
+            for lin in wl.linears:
+                s = seed + 7919 * c
+                codes = torch.from_numpy(lin.codes(s)).cuda()
+                scales = torch.from_numpy(lin.scales(s).view(np.int16)).cuda()
+                W = torch.empty(q4.q4_0_bytes(lin.N, lin.K), dtype=torch.uint8, device="cuda")
+                q4.q4_0_pack(codes, scales, W, lin.N, lin.K)
+                del codes, scales
+                X = torch.from_numpy(lin.x(s).view(np.int16)).cuda()
+                Y = torch.empty((lin.M, lin.N), dtype=torch.float32, device="cuda")
+                probs.append((W, X, Y, lin.M, lin.N, lin.K))
+            self.sets.append((probs, q4.make_problems(probs)))
+        torch.cuda.synchronize()
+
+    def launch(self, q4, step: int):
+        probs, arr = self.sets[step % len(self.sets)]
+        q4.q4_0_gemm_grouped(arr, len(probs))
+
+
+def run_ours(args, rank: int, world: int):
+    import torch
+    import torch.distributed as dist
+    import bit_weight_only_matmul_b200 as q4
+
+    wl = workloads.workload(args.workload)
+    tensor = args.workload in TENSOR_WORKLOADS
+    step_bytes = wl.hbm_bytes
+    step_flops = wl.flops
+    copies = max(1, -(-2 * L2_BYTES // max(1, wl.weight_bytes + sum(l.act_bytes for l in wl.linears))))
+    copies = min(copies, 8)
+    if tensor:
+        copies = 1   # a 4096-row GEMM is compute-bound; its operands stay L2-resident by design
+    log(f"[rank {rank}] building {wl.name}: {len(wl.linears)} GEMMs x {copies} copies, "
+        f"{step_bytes / 1e6:.1f} MB per step")
+    G = GpuWorkload(q4, wl, copies, workloads.SEED + 1000 * rank)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    q4.q4_0_device_error(clear=True)
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        # warm-up: W untimed steps, then an untimed soak of about a second so
+        # that the clock sampler sees the GPU under this load
+        for i in range(args.warmup):
+            G.launch(q4, i)
+        barrier()
+        t_end = time.time() + 1.0
+        i = 0
+        while time.time() < t_end:
+            for _ in range(16):
+                G.launch(q4, i)
+                i += 1
+            torch.cuda.synchronize()
+        barrier()
+        # timed region: exactly K steps, one event pair around each launch
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        t0.record(stream)
+        for k in range(args.steps):
+            ev[k][0].record(stream)
+            G.launch(q4, k)
+            ev[k][1].record(stream)
+        t1.record(stream)
+        barrier()
+    ms_total = t0.elapsed_time(t1)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    dev_err = q4.q4_0_device_error(clear=True)
+    if dev_err:
+        raise RuntimeError(f"device error word {dev_err:#x} after the timed region")
+
+    # end to end through the public API: host X -> device, grouped GEMM, Y -> host
+    probs0 = G.sets[0][0]
+    hx = [torch.empty(p[1].shape, dtype=p[1].dtype, pin_memory=True).copy_(p[1].cpu()) for p in probs0]
+    hy = [torch.empty(p[2].shape, dtype=p[2].dtype, pin_memory=True) for p in probs0]
+    h2d = sum(t.numel() * t.element_size() for t in hx)
+    d2h = sum(t.numel() * t.element_size() for t in hy)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+
+    def e2e_step(k):
+        probs, arr = G.sets[k % len(G.sets)]
+        for (W, X, Y, *_), h in zip(probs, hx):
+            X.copy_(h, non_blocking=True)
+        q4.q4_0_gemm_grouped(arr, len(probs))
+        for (W, X, Y, *_), h in zip(probs, hy):
+            h.copy_(Y, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    barrier()
+    e0.record(stream)
+    for k in range(args.steps):
+        e2e_step(k)
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+
+    # max over ranks
+    t = torch.tensor([ms_total, e2e_ms, statistics.mean(launch_ms)], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total, e2e_ms, launch_avg_ms = (float(v) for v in t.tolist())
+    clock = clocks.summary()
+
+    if rank != 0:
+        return None
+    peaks = measured_peaks()
+    kernel, src = DOMINANT[args.workload]
+    if tensor:
+        unit = "TFLOP/s"
+        value = world * args.steps * step_flops / (ms_total * 1e-3) / 1e12
+        e2e_value = world * args.steps * step_flops / (e2e_ms * 1e-3) / 1e12
+        achieved = step_flops / (launch_avg_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        bound = "tensor"
+    else:
+        unit = "GB/s"
+        value = world * args.steps * step_bytes / (ms_total * 1e-3) / 1e9
+        e2e_value = world * args.steps * step_bytes / (e2e_ms * 1e-3) / 1e9
+        achieved = step_bytes / (launch_avg_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        bound = "hbm"
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": unit,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_total / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16 x q4_0 -> fp32" if not tensor else "fp16 x fp16(q4_0) -> fp32",
+        "data": "synthetic (seeded Philox; codes U{0..15}, d = fp16(|N(0,1)|*0.002+1e-4), X bf16 N(0,1))",
+        "config": {
+            "workload": f"{wl.name}: {wl.description}",
+            "gemms_per_step": len(wl.linears),
+            "bytes_per_step": step_bytes,
+            "flops_per_step": step_flops,
+            "weight_copies": len(G.sets),
+            "l2": (f"{len(G.sets)} rotating weight copies = {len(G.sets) * step_bytes / 1e6:.0f} MB > L2 "
+                   f"({L2_BYTES / 2**20:.0f} MiB)") if not tensor else "compute-bound; operands L2-resident",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        },
+        "roofline": {
+            "bound": bound,
+            "kernel": kernel,
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "unit": unit,
+            "frac": round(achieved / peak, 4),
+            "peak_source": peaks["source"],
+            "traffic": recorded_traffic(args.workload),
+            "algorithmic_per_launch": step_flops if tensor else step_bytes,
+        },
+        "e2e": {"value": round(e2e_value, 2), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * launches_per_step(args.workload, wl),
+        "clocks": clock,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(wl, tensor, budget_s=args.cpu_seconds)
+    return line
+
+
+def launches_per_step(name, wl) -> int:
+    # all M <= 32 problems of a step share one launch; each M > 32 problem is one launch
+    small = any(l.M <= 32 for l in wl.linears)
+    return int(small) + sum(1 for l in wl.linears if l.M > 32)
+
+
+# --------------------------------------------------------------------------- the oracle as a baseline
+
+def oracle_step_sample(o, wl, packed, row_stride: int):
+    """The oracle on every `row_stride`-th output column of every GEMM of
+    the step (all rows of X).  Returns the fraction of the step covered."""
+    covered = 0
+    for lin, (W, X) in zip(wl.linears, packed):
+        ns = np.arange(0, lin.N, row_stride)
+        ms = np.repeat(np.arange(lin.M), len(ns))
+        o.gemm_sampled(W, X, lin.M, lin.N, lin.K, ms, np.tile(ns, lin.M))
+        covered += len(ns) * lin.M * lin.K
+    total = sum(l.M * l.N * l.K for l in wl.linears)
+    return covered / total
+
+
+def pack_on_host(wl, seed):
+    import oracle
+    o = oracle.get()
+    return o, [(o.pack(l.codes(seed), l.scales(seed)), l.x(seed)) for l in wl.linears]
+
+
+def cpu_baseline(wl, tensor: bool, budget_s: float):
+    o, packed = pack_on_host(wl, workloads.SEED)
+    total_macs = sum(l.M * l.N * l.K for l in wl.linears)
+    # choose a column stride so one sampled pass is about budget/3 seconds (46 M MAC/s measured on one core)
+    est_rate = 4.5e7
+    stride = max(1, int(round(total_macs / (est_rate * budget_s / 3))))
+    frac_total, t0 = 0.0, time.perf_counter()
+    reps = 0
+    while True:
+        frac_total += oracle_step_sample(o, wl, packed, stride)
+        reps += 1
+        if time.perf_counter() - t0 > budget_s * 0.66 or reps >= 50:
+            break
+    dt = time.perf_counter() - t0
+    if tensor:
+        value, unit = frac_total * wl.flops / dt / 1e12, "TFLOP/s"
+    else:
+        value, unit = frac_total * wl.hbm_bytes / dt / 1e9, "GB/s"
+    return {"value": value, "unit": unit, "cores": 1, "kind": "oracle",
+            "sample": f"{reps} pass(es) over every {stride}th output column of all {len(wl.linears)} GEMMs "
+                      f"({frac_total / reps:.4f} of a step each), {dt:.1f} s, scaled to whole steps"}
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return None
+    wl = workloads.workload(args.workload)
+    tensor = args.workload in TENSOR_WORKLOADS
+    o, packed = pack_on_host(wl, workloads.SEED)
+    total_macs = sum(l.M * l.N * l.K for l in wl.linears)
+    # each step: a sample of about 1 s of oracle work
+    stride = max(1, int(round(total_macs / 4.5e7)))
+    for _ in range(args.warmup):
+        oracle_step_sample(o, wl, packed, stride)
+    t0 = time.perf_counter()
+    frac = 0.0
+    for _ in range(args.steps):
+        frac += oracle_step_sample(o, wl, packed, stride)
+    dt = time.perf_counter() - t0
+    if tensor:
+        value, unit = frac * wl.flops / dt / 1e12, "TFLOP/s"
+    else:
+        value, unit = frac * wl.hbm_bytes / dt / 1e9, "GB/s"
+    sample = (f"each step = every {stride}th output column of all {len(wl.linears)} GEMMs "
+              f"({frac / args.steps:.4f} of a step), scaled to whole steps")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": unit,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded Philox, same workload recipe)",
+        "config": {"workload": f"{wl.name}: {wl.description}", "bytes_per_step": wl.hbm_bytes,
+                   "flops_per_step": wl.flops, "parallelism": "one host core"},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# --------------------------------------------------------------------------- main
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=workloads.WORKLOADS)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline budget (rank 0, N=1)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        log(f"note: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE")
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+    torch.cuda.set_device(local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    try:
+        line = run_ours(args, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
