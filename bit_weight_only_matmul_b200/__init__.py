@@ -28,7 +28,7 @@ Q4_DEVERR_FP16_RANGE = 2
 
 Q4_0_MAX_GROUP = 256
 
-PATH_AUTO, PATH_GENERIC, PATH_DECODE, PATH_TENSOR = 0, 1, 2, 3
+PATH_AUTO, PATH_GENERIC, PATH_DECODE, PATH_TENSOR, PATH_DECODE_MMA = 0, 1, 2, 3, 4
 
 # every symbol include/q4_0.h declares
 EXPORTS = (

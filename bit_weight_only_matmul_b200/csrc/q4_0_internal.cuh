@@ -32,9 +32,14 @@ cudaError_t launch_pack(const uint8_t *codes, const uint16_t *scales, uint8_t *W
 cudaError_t launch_dequant(const uint8_t *W, float *out, int64_t N, int64_t K, cudaStream_t s);
 cudaError_t launch_zero(float *Y, int64_t count, cudaStream_t s);
 cudaError_t launch_generic(const Problem *probs, int count, const DeviceInfo &dev, cudaStream_t s);
-// Decode kernel: every problem must satisfy decode_supports().
+// Decode kernel on warp-level mma.sync (M <= 32): every problem must satisfy
+// decode_supports().
 bool decode_supports(const Problem &p);
 cudaError_t launch_decode(const Problem *probs, int count, const DeviceInfo &dev, cudaStream_t s);
+// Decode kernel on tcgen05 with weights in tensor memory (M <= 16): every
+// problem must satisfy decode_tmem_supports().
+bool decode_tmem_supports(const Problem &p);
+cudaError_t launch_decode_tmem(const Problem *probs, int count, const DeviceInfo &dev, cudaStream_t s);
 // Tensor-core kernel: every problem must satisfy prefill_supports().
 bool prefill_supports(const Problem &p);
 cudaError_t launch_prefill(const Problem &p, const DeviceInfo &dev, cudaStream_t s);

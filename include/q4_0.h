@@ -154,10 +154,11 @@ Q4_0_API int q4_0_gemm_grouped(const q4_0_problem *problems, int count,
 Q4_0_API int q4_0_device_error(uint32_t *flags, int clear);
 
 /* Testing knob, process-wide: force the kernel family used by q4_0_gemm and
- * q4_0_gemm_grouped.  0 = automatic (default), 1 = portable reference-style
- * kernel (any shape), 2 = decode kernel (M <= 32 only), 3 = tensor-core
- * kernel.  A forced family that cannot run a given shape falls back to
- * automatic.  The pages have no counterpart. */
+ * q4_0_gemm_grouped.  0 = automatic (default), 1 = portable kernel (any
+ * shape), 2 = decode kernels (M <= 32 only), 3 = tensor-core kernel, 4 =
+ * the warp-level mma.sync decode kernel (M <= 32).  A forced family that
+ * cannot run a given shape falls back to automatic.  The pages have no
+ * counterpart. */
 Q4_0_API int q4_0_force_path(int path);
 
 #ifdef __cplusplus

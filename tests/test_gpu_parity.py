@@ -229,3 +229,15 @@ def test_prefill_workload_sampled(q4, name):
     b = build_workload(q4, workloads.workload(name), samples=2000)
     q4.q4_0_gemm_grouped(b.problems())
     check_built(b, name)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 100, 1024), (2, 129, 3072), (8, 64, 512), (16, 33, 2048)])
+def test_forced_warp_mma_decode(q4, M, N, K):
+    run_gemm(q4, M, N, K, path=q4.PATH_DECODE_MMA)
+
+
+@pytest.mark.parametrize("name,layers", [("cfg_decode", [0, 13, 25]), ("concurrent", [0, 25])])
+def test_decode_workloads_sampled(q4, name, layers):
+    b = build_workload(q4, workloads.workload(name, layers=layers), samples=400)
+    q4.q4_0_gemm_grouped(b.problems())
+    check_built(b, name)
