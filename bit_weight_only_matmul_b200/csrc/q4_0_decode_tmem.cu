@@ -20,8 +20,10 @@
 //  * item = 128 weight rows x all of K of one problem; items are sorted by K
 //    (largest first) on the host and dealt to the CTAs in boustrophedon order;
 //  * stage = 256 k of the item (8 Q4_0 blocks, 144 contiguous bytes per row)
-//    plus the same 256 k of every row of X, fetched with 1-D bulk copies
-//    (cp.async.bulk, completion on an mbarrier) into a 4-deep ring;
+//    plus the same 256 k of every row of X, in a 4-deep ring: the weights as
+//    one TMA box (128 rows x 144 bytes) per stage, the few X rows as 1-D bulk
+//    copies (one issue per byte run costs ~60 cycles per SM, so the weights
+//    must not come row by row);
 //  * worker warp (quadrant q, half h) owns tensor-memory lanes 32q..32q+31 =
 //    weight rows, and blocks 4h..4h+3 of each stage: it turns the 4-bit codes
 //    into exact bf16 (q - 8) and writes them to tensor memory (A operand,
@@ -45,6 +47,7 @@
 
 #include "q4_0_internal.cuh"
 #include "q4_0_tcgen05.cuh"
+#include "q4_0_tmap.cuh"
 
 namespace {
 
@@ -75,11 +78,14 @@ struct TProblem {
     int item_begin;    // first item index of this problem
 };
 
-struct TParams {
+// CAP problems per launch (the tensor maps live in the kernel parameters).
+template <int CAP>
+struct alignas(64) TParams {
+    CUtensorMap wmap[CAP];   // Q4_0 bytes [N, K/32*18], box 144 x 128
     int count;
     int total_items;
     unsigned *err;
-    TProblem p[Q4_0_MAX_GROUP];
+    TProblem p[CAP];
 };
 
 struct Smem {
@@ -94,7 +100,8 @@ struct Smem {
     int abort_flag;
 };
 
-__device__ __forceinline__ int find_problem(const TParams &P, int item) {
+template <class TP>
+__device__ __forceinline__ int find_problem(const TP &P, int item) {
     int lo = 0, hi = P.count - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -106,7 +113,8 @@ __device__ __forceinline__ int find_problem(const TParams &P, int item) {
 // One CTA's sequence of (item, stage).
 struct Seq {
     int round, item, prob, row0, stage, nstages;
-    __device__ __forceinline__ void load(const TParams &P) {
+    template <class TP>
+    __device__ __forceinline__ void load(const TP &P) {
         const int G = gridDim.x;
         const int pos = (round & 1) ? (G - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
         item = round * G + pos;
@@ -116,8 +124,10 @@ struct Seq {
         stage = 0;
         nstages = P.p[prob].stages;
     }
-    __device__ __forceinline__ void start(const TParams &P) { round = 0; load(P); }
-    __device__ __forceinline__ void next(const TParams &P) {
+    template <class TP>
+    __device__ __forceinline__ void start(const TP &P) { round = 0; load(P); }
+    template <class TP>
+    __device__ __forceinline__ void next(const TP &P) {
         if (++stage < nstages) return;
         ++round;
         load(P);
@@ -189,8 +199,8 @@ __device__ __forceinline__ void dequant_half(const uint32_t (&w)[20], uint32_t (
     }
 }
 
-template <int MP>
-__global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_constant__ TParams P) {
+template <int MP, int CAP>
+__global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_constant__ TParams<CAP> P) {
     extern __shared__ uint8_t smem_raw[];
     Smem &S = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -227,14 +237,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
             const uint32_t g = prod_issued;
             const bool ok = wait_or_abort(&S.raw_empty[slot], ((g / kRS) & 1) ^ 1, S, P.err);
             if (!__all_sync(0xffffffffu, ok)) break;
-            const int rows = min(kRows, pr.N - q.row0);
-            if (lane == 0) mbar_arrive_expect_tx(&S.raw_full[slot], rows * kRawRow + pr.M * kXRow);
+            // weights: one TMA box (rows past N are zero-filled and still counted)
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&S.raw_full[slot], kRawW + pr.M * kXRow);
+                tma_load_2d(S.raw[slot], &P.wmap[q.prob], q.stage * kRawRow, q.row0, &S.raw_full[slot]);
+            }
             __syncwarp();
-            const int64_t row_bytes = static_cast<int64_t>(pr.stages) * kRawRow;
-            for (int r = lane; r < rows; r += 32)
-                bulk_g2s(S.raw[slot] + r * kRawRow,
-                         pr.W + (static_cast<int64_t>(q.row0) + r) * row_bytes + static_cast<int64_t>(q.stage) * kRawRow,
-                         kRawRow, &S.raw_full[slot]);
             for (int m = lane; m < pr.M; m += 32)
                 bulk_g2s(S.raw[slot] + kRawW + m * kXRow,
                          pr.X + static_cast<int64_t>(m) * pr.K + static_cast<int64_t>(q.stage) * kStageK, kXRow,
@@ -409,42 +417,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
 
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 
-template <int MP>
-cudaError_t launch_mp(TParams &P, const q4::DeviceInfo &dev, cudaStream_t s) {
+template <int MP, int CAP>
+cudaError_t launch_mp(TParams<CAP> &P, const q4::DeviceInfo &dev, cudaStream_t s) {
     static int configured_device = -1;
     if (configured_device != dev.device) {
-        cudaError_t e = cudaFuncSetAttribute(decode_tmem_kernel<MP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(kSmemBytes));
+        cudaError_t e = cudaFuncSetAttribute(decode_tmem_kernel<MP, CAP>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
         if (e != cudaSuccess) return e;
         configured_device = dev.device;
     }
     const int grid = std::max(1, std::min(dev.sm_count, P.total_items));
-    decode_tmem_kernel<MP><<<grid, kThreads, kSmemBytes, s>>>(P);
+    decode_tmem_kernel<MP, CAP><<<grid, kThreads, kSmemBytes, s>>>(P);
     return cudaGetLastError();
 }
 
-}  // namespace
-
-namespace q4 {
-
-bool decode_tmem_supports(const Problem &p) {
-    return p.M >= 1 && p.M <= kMaxM && p.K >= kStageK && p.K % kStageK == 0 && p.N >= 1 && p.N < (1LL << 31) &&
-           p.K < (1LL << 31) && (reinterpret_cast<uintptr_t>(p.W) & 15) == 0 &&
-           (reinterpret_cast<uintptr_t>(p.X) & 15) == 0;
-}
-
-cudaError_t launch_decode_tmem(const Problem *probs, int count, const DeviceInfo &dev, cudaStream_t s) {
-    if (count <= 0) return cudaSuccess;
-    std::vector<int> order(count);
-    for (int i = 0; i < count; ++i) order[i] = i;
-    std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return probs[a].K > probs[b].K; });
-    static thread_local TParams P;
+// problems[0..count) sorted by K (largest first), count <= CAP
+template <int CAP>
+cudaError_t launch_cap(const q4::Problem *probs, const int *order, int count, const q4::DeviceInfo &dev,
+                       cudaStream_t s) {
+    static thread_local TParams<CAP> P;
     P.count = count;
     P.err = dev.err;
     int items = 0;
     int64_t maxM = 1;
     for (int i = 0; i < count; ++i) {
-        const Problem &q = probs[order[i]];
+        const q4::Problem &q = probs[order[i]];
         TProblem &t = P.p[i];
         t.W = q.W;
         t.X = q.X;
@@ -456,13 +453,42 @@ cudaError_t launch_decode_tmem(const Problem *probs, int count, const DeviceInfo
         t.item_begin = items;
         items += static_cast<int>((q.N + kRows - 1) / kRows);
         maxM = std::max(maxM, q.M);
+        if (!q4::get_tensor_map(&P.wmap[i], q.W, q.N, q.K / 32 * 18, q4::kMapWeights128))
+            return cudaErrorInvalidValue;
     }
     P.total_items = items;
-    if (maxM <= 1) return launch_mp<1>(P, dev, s);
-    if (maxM <= 2) return launch_mp<2>(P, dev, s);
-    if (maxM <= 4) return launch_mp<4>(P, dev, s);
-    if (maxM <= 8) return launch_mp<8>(P, dev, s);
-    return launch_mp<16>(P, dev, s);
+    if (maxM <= 1) return launch_mp<1, CAP>(P, dev, s);
+    if (maxM <= 2) return launch_mp<2, CAP>(P, dev, s);
+    if (maxM <= 4) return launch_mp<4, CAP>(P, dev, s);
+    if (maxM <= 8) return launch_mp<8, CAP>(P, dev, s);
+    return launch_mp<16, CAP>(P, dev, s);
+}
+
+constexpr int kSmallCap = 8, kLargeCap = 128;
+
+}  // namespace
+
+namespace q4 {
+
+bool decode_tmem_supports(const Problem &p) {
+    return p.M >= 1 && p.M <= kMaxM && p.K >= kStageK && p.K % kStageK == 0 && p.N >= 1 && p.N < (1LL << 31) &&
+           p.K < (1LL << 31) && (reinterpret_cast<uintptr_t>(p.W) & 15) == 0 &&
+           (reinterpret_cast<uintptr_t>(p.X) & 15) == 0 && tensor_maps_available();
+}
+
+cudaError_t launch_decode_tmem(const Problem *probs, int count, const DeviceInfo &dev, cudaStream_t s) {
+    if (count <= 0) return cudaSuccess;
+    std::vector<int> order(count);
+    for (int i = 0; i < count; ++i) order[i] = i;
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return probs[a].K > probs[b].K; });
+    for (int done = 0; done < count;) {
+        const int n = std::min(count - done, kLargeCap);
+        cudaError_t e = n <= kSmallCap ? launch_cap<kSmallCap>(probs, order.data() + done, n, dev, s)
+                                       : launch_cap<kLargeCap>(probs, order.data() + done, n, dev, s);
+        if (e != cudaSuccess) return e;
+        done += n;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace q4

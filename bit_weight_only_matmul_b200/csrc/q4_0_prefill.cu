@@ -36,6 +36,7 @@
 
 #include "q4_0_internal.cuh"
 #include "q4_0_tcgen05.cuh"
+#include "q4_0_tmap.cuh"
 
 namespace {
 
@@ -373,23 +374,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 
 // ---------------------------------------------------------------- host side
 
-using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                 const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled get_encoder() {
-    static EncodeTiled fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiled>(p);
-    });
-    return fn;
-}
-
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 
 }  // namespace
@@ -399,35 +383,15 @@ namespace q4 {
 bool prefill_supports(const Problem &p) {
     return p.M >= 1 && p.N >= 1 && p.K >= 256 && p.K % 256 == 0 && p.M < (1LL << 31) && p.N < (1LL << 31) &&
            p.K < (1LL << 31) && (reinterpret_cast<uintptr_t>(p.W) & 15) == 0 &&
-           (reinterpret_cast<uintptr_t>(p.X) & 15) == 0 && get_encoder() != nullptr;
+           (reinterpret_cast<uintptr_t>(p.X) & 15) == 0 && tensor_maps_available();
 }
 
 cudaError_t launch_prefill(const Problem &p, const DeviceInfo &dev, cudaStream_t s) {
-    EncodeTiled enc = get_encoder();
-    if (!enc) return cudaErrorNotSupported;
     PrefillParams local;
     std::memset(&local, 0, sizeof(local));
-    {
-        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.K), static_cast<cuuint64_t>(p.M)};
-        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.K) * 2};
-        const cuuint32_t box[2] = {static_cast<cuuint32_t>(kStageK), static_cast<cuuint32_t>(kTileM)};
-        const cuuint32_t estr[2] = {1, 1};
-        if (enc(&local.tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(p.X), dims, strides, box,
-                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
-    {
-        const int64_t row_bytes = p.K / 32 * 18;
-        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(p.N)};
-        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
-        const cuuint32_t box[2] = {static_cast<cuuint32_t>(kRawRowBytes), static_cast<cuuint32_t>(kTileN)};
-        const cuuint32_t estr[2] = {1, 1};
-        if (enc(&local.tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(p.W), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
+    if (!get_tensor_map(&local.tmap_x, p.X, p.M, p.K, kMapActivationsSw128) ||
+        !get_tensor_map(&local.tmap_w, p.W, p.N, p.K / 32 * 18, kMapWeights128Prefill))
+        return cudaErrorInvalidValue;
     local.Y = p.Y;
     local.err = dev.err;
     local.M = static_cast<int>(p.M);
