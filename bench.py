@@ -48,9 +48,9 @@ DEFAULT_WORKLOAD = "layer"
 
 # kernel that dominates each workload, and the source file it lives in
 DOMINANT = {
-    "gemv": ("decode_kernel", "q4_0_decode.cu"),
-    "layer": ("decode_kernel", "q4_0_decode.cu"),
-    "cfg_decode": ("decode_kernel", "q4_0_decode.cu"),
+    "gemv": ("decode_tmem_kernel", "q4_0_decode_tmem.cu"),
+    "layer": ("decode_tmem_kernel", "q4_0_decode_tmem.cu"),
+    "cfg_decode": ("decode_tmem_kernel", "q4_0_decode_tmem.cu"),
     "concurrent": ("decode_kernel", "q4_0_decode.cu"),
     "adapter": ("prefill_kernel", "q4_0_prefill.cu"),
     "qkv_prefill": ("prefill_kernel", "q4_0_prefill.cu"),
@@ -257,11 +257,7 @@ def run_ours(args, rank: int, world: int):
     barrier()
     e2e_ms = e0.elapsed_time(e1)
 
-    # max over ranks
-    t = torch.tensor([ms_total, e2e_ms, statistics.mean(launch_ms)], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total, e2e_ms, launch_avg_ms = (float(v) for v in t.tolist())
+    ms_total, e2e_ms, launch_avg_ms = max_over_ranks([ms_total, e2e_ms, statistics.mean(launch_ms)], world, "cuda")
     clock = clocks.summary()
 
     if rank != 0:
@@ -270,15 +266,15 @@ def run_ours(args, rank: int, world: int):
     kernel, src = DOMINANT[args.workload]
     if tensor:
         unit = "TFLOP/s"
-        value = world * args.steps * step_flops / (ms_total * 1e-3) / 1e12
-        e2e_value = world * args.steps * step_flops / (e2e_ms * 1e-3) / 1e12
+        value = whole_job_rate(step_flops, args.steps, world, ms_total) / 1e12
+        e2e_value = whole_job_rate(step_flops, args.steps, world, e2e_ms) / 1e12
         achieved = step_flops / (launch_avg_ms * 1e-3) / 1e12
         peak = peaks["bf16_tflops"]
         bound = "tensor"
     else:
         unit = "GB/s"
-        value = world * args.steps * step_bytes / (ms_total * 1e-3) / 1e9
-        e2e_value = world * args.steps * step_bytes / (e2e_ms * 1e-3) / 1e9
+        value = whole_job_rate(step_bytes, args.steps, world, ms_total) / 1e9
+        e2e_value = whole_job_rate(step_bytes, args.steps, world, e2e_ms) / 1e9
         achieved = step_bytes / (launch_avg_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         bound = "hbm"
@@ -323,6 +319,23 @@ def run_ours(args, rank: int, world: int):
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(wl, tensor, budget_s=args.cpu_seconds)
     return line
+
+
+def max_over_ranks(values, world: int, device: str):
+    """Element-wise max of per-rank timings (every rank gets the result)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_rate(units_per_rank_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Work of all ranks (weak scaling: every rank does the same work) over
+    the slowest rank's time, per second."""
+    return world * steps * units_per_rank_step / (max_ms * 1e-3)
 
 
 def launches_per_step(name, wl) -> int:

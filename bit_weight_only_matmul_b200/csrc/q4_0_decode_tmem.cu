@@ -62,8 +62,8 @@ constexpr int kXRow = kStageK * 2;          // 512 bytes of one X row per stage
 constexpr int kRawBytes = kRawW + kMaxM * kXRow;   // 26624
 constexpr int kRS = 4;                      // ring depth
 constexpr int kBBytes = kMaxM * kStageK * 2;       // 8192: 4 swizzle atoms of 16 rows x 128 bytes
-constexpr int kWarpProd = 0, kWarpMMA = 1, kWarp0 = 2, kWorkers = 8;
-constexpr int kThreads = 32 * (kWarp0 + kWorkers);  // 320
+constexpr int kWarpProd = 0, kWarpMMA = 1, kWarpX = 2, kWarp0 = 3, kWorkers = 8;
+constexpr int kThreads = 32 * (kWarp0 + kWorkers);  // 352
 constexpr uint32_t kTmemCols = 512;
 constexpr int kACol = 0;                    // A: 2 buffers x 128 columns (256 bf16 per row)
 constexpr int kDCol = 256;                  // D: 2 buffers x (8 blocks x 16 columns)
@@ -93,7 +93,7 @@ struct Smem {
     uint8_t b[2][kBBytes];                    // B operand, 1024-byte aligned
     float comb[2][4][kMaxM][32];              // partial sums handed between the two halves
     uint64_t raw_full[kRS], raw_empty[kRS];
-    uint64_t ab_full[2], d_full[2], d_empty[2];
+    uint64_t ab_full[2], b_full[2], b_empty[2], d_full[2], d_empty[2];
     uint64_t comb_full[2], comb_empty[2];
     uint64_t mma_done;
     uint32_t tmem_base;
@@ -137,17 +137,15 @@ struct Seq {
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, Smem &S, unsigned *err) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0) {
-            if (*reinterpret_cast<volatile int *>(&S.abort_flag)) return false;
-            if (global_ns() - t0 > kWaitLimitNs) {
-                atomicOr(err, (unsigned)Q4_DEVERR_WAIT_TIMEOUT);
-                *reinterpret_cast<volatile int *>(&S.abort_flag) = 1;
-                return false;
-            }
+    while (!mbar_try_wait_suspend(bar, parity)) {
+        if (*reinterpret_cast<volatile int *>(&S.abort_flag)) return false;
+        if (global_ns() - t0 > kWaitLimitNs) {
+            atomicOr(err, (unsigned)Q4_DEVERR_WAIT_TIMEOUT);
+            *reinterpret_cast<volatile int *>(&S.abort_flag) = 1;
+            return false;
         }
     }
+    return true;
 }
 
 // Exact bf16 pairs (q - 8) from one qs word v (bytes 4w..4w+3 of a block):
@@ -208,10 +206,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
     if (threadIdx.x == 0) {
         for (int s = 0; s < kRS; ++s) {
             mbar_init(&S.raw_full[s], 1);
-            mbar_init(&S.raw_empty[s], kWorkers);
+            mbar_init(&S.raw_empty[s], kWorkers + 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&S.ab_full[s], kWorkers);
+            mbar_init(&S.b_full[s], 1);
+            mbar_init(&S.b_empty[s], 1);
             mbar_init(&S.d_full[s], 1);
             mbar_init(&S.d_empty[s], kWorkers);
             mbar_init(&S.comb_full[s], kWorkers / 2);
@@ -235,8 +235,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
             const TProblem &pr = P.p[q.prob];
             const int slot = prod_issued % kRS;
             const uint32_t g = prod_issued;
-            const bool ok = wait_or_abort(&S.raw_empty[slot], ((g / kRS) & 1) ^ 1, S, P.err);
-            if (!__all_sync(0xffffffffu, ok)) break;
+            bool ok = true;
+            if (lane == 0) ok = wait_or_abort(&S.raw_empty[slot], ((g / kRS) & 1) ^ 1, S, P.err);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             // weights: one TMA box (rows past N are zero-filled and still counted)
             if (lane == 0) {
                 mbar_arrive_expect_tx(&S.raw_full[slot], kRawW + pr.M * kXRow);
@@ -259,6 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
             for (; q.item >= 0; q.next(P), ++g) {
                 const int buf = g & 1;
                 if (!wait_or_abort(&S.ab_full[buf], (g >> 1) & 1, S, P.err)) break;
+                if (!wait_or_abort(&S.b_full[buf], (g >> 1) & 1, S, P.err)) break;
                 if (!wait_or_abort(&S.d_empty[buf], ((g >> 1) & 1) ^ 1, S, P.err)) break;
                 tc_fence_after();
                 const uint64_t bdesc = sw128_kmajor_desc(smem_addr(S.b[buf]));
@@ -272,15 +274,49 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
                                   bdesc + (off >> 4), kIdesc, j);
                     }
                 tc_commit(&S.d_full[buf]);
+                tc_commit(&S.b_empty[buf]);
             }
             tc_commit(&S.mma_done);
             if (!wait_or_abort(&S.mma_done, 0, S, P.err)) mbar_wait(&S.mma_done, 0, P.err);
+        }
+    } else if (warp == kWarpX) {
+        // ---------------------------------------------------------------- X rows -> B operand
+        uint32_t g = 0;
+        Seq q;
+        q.start(P);
+        for (; q.item >= 0; q.next(P), ++g) {
+            const TProblem &pr = P.p[q.prob];
+            const int slot = g % kRS, buf = g & 1;
+            bool ok = true;
+            if (lane == 0) {
+                ok = wait_or_abort(&S.raw_full[slot], (g / kRS) & 1, S, P.err);
+                // B[buf] was last read by the MMAs of stage g-2
+                if (ok) ok = wait_or_abort(&S.b_empty[buf], ((g >> 1) & 1) ^ 1, S, P.err);
+            }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            // 128-byte swizzle; k permuted within 4-groups as in the A operand
+            for (int c = lane; c < pr.M * 32; c += 32) {
+                const int m = c >> 5, kc = c & 31;
+                const uint4 v = *reinterpret_cast<const uint4 *>(S.raw[slot] + kRawW + m * kXRow + kc * 16);
+                uint4 o;
+                o.x = prmt(v.x, v.y, 0x5410u);   // (x0, x2)
+                o.y = prmt(v.x, v.y, 0x7632u);   // (x1, x3)
+                o.z = prmt(v.z, v.w, 0x5410u);   // (x4, x6)
+                o.w = prmt(v.z, v.w, 0x7632u);   // (x5, x7)
+                *reinterpret_cast<uint4 *>(S.b[buf] + (kc >> 3) * 2048 + (m >> 3) * 1024 + (m & 7) * 128 +
+                                           (((kc & 7) ^ (m & 7)) * 16)) = o;
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&S.b_full[buf]);
+                mbar_arrive(&S.raw_empty[slot]);
+            }
         }
     } else {
         // ---------------------------------------------------------------- workers
         const int quad = warp & 3;            // tensor-memory lanes 32*quad ..
         const int half = (warp - kWarp0) >> 2;   // blocks 4*half .. 4*half+3 of each stage
-        const int wid = (warp - kWarp0) * 32 + lane;
         const uint32_t lane_base = uint32_t(32 * quad) << 16;
         float acc[MP];
         #pragma unroll
@@ -295,13 +331,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
             const int buf = gp & 1;
             if (!wait_or_abort(&S.d_full[buf], (gp >> 1) & 1, S, P.err)) return false;
             tc_fence_after();
-            #pragma unroll
-            for (int jb = 0; jb < 4; ++jb) {
-                float v[MP];
-                tc_ld_cols<MP>(tmem + lane_base + kDCol + 128 * buf + 16 * (4 * half + jb), v);
+            if constexpr (MP <= 4) {   // four loads in flight, one wait
+                float v[4][MP];
+                #pragma unroll
+                for (int jb = 0; jb < 4; ++jb)
+                    tc_ld_cols<MP>(tmem + lane_base + kDCol + 128 * buf + 16 * (4 * half + jb), v[jb]);
                 tc_wait_ld();
                 #pragma unroll
-                for (int m = 0; m < MP; ++m) acc[m] = fmaf(dprev[jb], v[m], acc[m]);
+                for (int jb = 0; jb < 4; ++jb)
+                    #pragma unroll
+                    for (int m = 0; m < MP; ++m) acc[m] = fmaf(dprev[jb], v[jb][m], acc[m]);
+            } else {
+                #pragma unroll
+                for (int jb = 0; jb < 4; ++jb) {
+                    float v[MP];
+                    tc_ld_cols<MP>(tmem + lane_base + kDCol + 128 * buf + 16 * (4 * half + jb), v);
+                    tc_wait_ld();
+                    #pragma unroll
+                    for (int m = 0; m < MP; ++m) acc[m] = fmaf(dprev[jb], v[m], acc[m]);
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -353,19 +401,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
                     w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
                 }
             }
-            // X rows of the stage -> B operand (128-byte swizzle), k permuted within 4-groups
-            for (int c = wid; c < pr.M * 32; c += kWorkers * 32) {
-                const int m = c >> 5, kc = c & 31;
-                const uint4 v = *reinterpret_cast<const uint4 *>(S.raw[slot] + kRawW + m * kXRow + kc * 16);
-                uint4 o;
-                o.x = prmt(v.x, v.y, 0x5410u);   // (x0, x2)
-                o.y = prmt(v.x, v.y, 0x7632u);   // (x1, x3)
-                o.z = prmt(v.z, v.w, 0x5410u);   // (x4, x6)
-                o.w = prmt(v.z, v.w, 0x7632u);   // (x5, x7)
-                *reinterpret_cast<uint4 *>(S.b[buf] + (kc >> 3) * 2048 + (m >> 3) * 1024 + (m & 7) * 128 +
-                                           (((kc & 7) ^ (m & 7)) * 16)) = o;
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.raw_empty[slot]);
 
@@ -382,12 +417,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
                 tc_st_32(ta, lo);
                 tc_st_32(ta + 32, hi);
             }
+            // while the stores drain: finish the previous stage
+            if (g > 0 && !(ok = scale(g - 1))) break;
             tc_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.ab_full[buf]);
 
-            if (g > 0 && !(ok = scale(g - 1))) break;
             #pragma unroll
             for (int jb = 0; jb < 4; ++jb) dprev[jb] = dcur[jb];
             prev_last = (q.stage == q.nstages - 1);

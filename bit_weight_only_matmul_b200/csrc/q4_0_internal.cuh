@@ -97,19 +97,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the thread for up to `hint_ns`
+// while the phase is incomplete (a waiting warp then issues nothing).
+constexpr uint32_t kSuspendHintNs = 1000000;   // 1 ms
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(kSuspendHintNs)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for phase `parity` of an mbarrier to complete, for at most
 // kWaitLimitNs.  Returns false (and ORs Q4_DEVERR_WAIT_TIMEOUT into *err) if
 // the wait ran out.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned *err) {
     if (mbar_try_wait(bar, parity)) return true;
-    unsigned long long t0 = global_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) {
+    const unsigned long long t0 = global_ns();
+    while (!mbar_try_wait_suspend(bar, parity)) {
+        if (global_ns() - t0 > kWaitLimitNs) {
             atomicOr(err, (unsigned)Q4_DEVERR_WAIT_TIMEOUT);
             return false;
         }
     }
+    return true;
 }
 
 // 1-D bulk copy global -> shared, completion counted on an mbarrier.

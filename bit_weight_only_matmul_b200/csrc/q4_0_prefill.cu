@@ -98,17 +98,15 @@ constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | (uint32_t(kTile
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, Smem &S, unsigned *err) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0) {
-            if (*reinterpret_cast<volatile int *>(&S.abort_flag)) return false;
-            if (global_ns() - t0 > kWaitLimitNs) {
-                atomicOr(err, (unsigned)Q4_DEVERR_WAIT_TIMEOUT);
-                *reinterpret_cast<volatile int *>(&S.abort_flag) = 1;
-                return false;
-            }
+    while (!mbar_try_wait_suspend(bar, parity)) {
+        if (*reinterpret_cast<volatile int *>(&S.abort_flag)) return false;
+        if (global_ns() - t0 > kWaitLimitNs) {
+            atomicOr(err, (unsigned)Q4_DEVERR_WAIT_TIMEOUT);
+            *reinterpret_cast<volatile int *>(&S.abort_flag) = 1;
+            return false;
         }
     }
+    return true;
 }
 
 // ---------------------------------------------------------------- dequantization

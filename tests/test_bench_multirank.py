@@ -1,0 +1,47 @@
+"""The N > 1 plumbing of bench.py on CPU: two gloo ranks (the path runs
+replicas, so the only cross-rank steps are the barrier and the max-over-ranks
+reduction of the timings)."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import bench
+        # rank r is slower by r ms; the reduction must return the slowest
+        local = [10.0 + rank, 20.0 + 2 * rank, 0.5 + rank]
+        dist.barrier()
+        got = bench.max_over_ranks(local, world, "cpu")
+        out[rank] = got
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    assert res[0] == res[1] == [11.0, 22.0, 1.5]
+
+
+def test_whole_job_rate_is_weak_scaling():
+    import bench
+    # 2 ranks x 10 steps x 1e9 bytes in 20 ms (slowest rank) = 1e12 B/s
+    assert bench.whole_job_rate(1e9, 10, 2, 20.0) == pytest.approx(1e12)
+    assert bench.max_over_ranks([1.0, 2.0], 1, "cpu") == [1.0, 2.0]
