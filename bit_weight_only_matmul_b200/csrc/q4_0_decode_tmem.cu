@@ -60,7 +60,7 @@ constexpr int kRawW = kRows * kRawRow;      // 18432
 constexpr int kMaxM = 16;                   // activation rows (the MMA's N)
 constexpr int kXRow = kStageK * 2;          // 512 bytes of one X row per stage
 constexpr int kRawBytes = kRawW + kMaxM * kXRow;   // 26624
-constexpr int kRS = 4;                      // ring depth
+constexpr int kRS = 6;                      // ring depth
 constexpr int kBBytes = kMaxM * kStageK * 2;       // 8192: 4 swizzle atoms of 16 rows x 128 bytes
 constexpr int kWarpProd = 0, kWarpMMA = 1, kWarpX = 2, kWarp0 = 3, kWorkers = 8;
 constexpr int kThreads = 32 * (kWarp0 + kWorkers);  // 352
@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
     uint32_t prod_issued = 0;   // stages whose copies the producer issued
 
     if (warp == kWarpProd) {
-        Seq q;
+        Seq q{};
         q.start(P);
         for (; q.item >= 0; q.next(P)) {
             const TProblem &pr = P.p[q.prob];
@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
     } else if (warp == kWarpMMA) {
         if (lane == 0) {
             uint32_t g = 0;
-            Seq q;
+            Seq q{};
             q.start(P);
             for (; q.item >= 0; q.next(P), ++g) {
                 const int buf = g & 1;
@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
     } else if (warp == kWarpX) {
         // ---------------------------------------------------------------- X rows -> B operand
         uint32_t g = 0;
-        Seq q;
+        Seq q{};
         q.start(P);
         for (; q.item >= 0; q.next(P), ++g) {
             const TProblem &pr = P.p[q.prob];
@@ -321,14 +321,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
         float acc[MP];
         #pragma unroll
         for (int m = 0; m < MP; ++m) acc[m] = 0.f;
-        float dprev[4] = {0.f, 0.f, 0.f, 0.f};
-        int prev_last = 0, prev_prob = 0, prev_row0 = 0;
+        // stages g-1 and g-2 still owe their scaling: a two-entry ring
+        struct Pending {
+            float d[4];
+            int last, prob, row0;
+        };
+        Pending pend[2];
         uint32_t items_done = 0;
         bool ok = true;
 
         // read back stage gp's per-block sums, scale by d, and finish the item if it was its last stage
         auto scale = [&](uint32_t gp) -> bool {
             const int buf = gp & 1;
+            const Pending &pd = pend[gp & 1];
             if (!wait_or_abort(&S.d_full[buf], (gp >> 1) & 1, S, P.err)) return false;
             tc_fence_after();
             if constexpr (MP <= 4) {   // four loads in flight, one wait
@@ -340,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
                 #pragma unroll
                 for (int jb = 0; jb < 4; ++jb)
                     #pragma unroll
-                    for (int m = 0; m < MP; ++m) acc[m] = fmaf(dprev[jb], v[jb][m], acc[m]);
+                    for (int m = 0; m < MP; ++m) acc[m] = fmaf(pd.d[jb], v[jb][m], acc[m]);
             } else {
                 #pragma unroll
                 for (int jb = 0; jb < 4; ++jb) {
@@ -348,14 +353,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
                     tc_ld_cols<MP>(tmem + lane_base + kDCol + 128 * buf + 16 * (4 * half + jb), v);
                     tc_wait_ld();
                     #pragma unroll
-                    for (int m = 0; m < MP; ++m) acc[m] = fmaf(dprev[jb], v[m], acc[m]);
+                    for (int m = 0; m < MP; ++m) acc[m] = fmaf(pd.d[jb], v[m], acc[m]);
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.d_empty[buf]);
-            if (prev_last) {
-                const TProblem &pr = P.p[prev_prob];
+            if (pd.last) {
+                const TProblem &pr = P.p[pd.prob];
                 const int cb = items_done & 1;
                 const uint32_t par = (items_done >> 1) & 1;
                 if (half == 1) {
@@ -370,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
                     for (int m = 0; m < MP; ++m) acc[m] += S.comb[cb][quad][m][lane];
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S.comb_empty[cb]);
-                    const int n = prev_row0 + 32 * quad + lane;
+                    const int n = pd.row0 + 32 * quad + lane;
                     if (n < pr.N) {
                         #pragma unroll
                         for (int m = 0; m < MP; ++m)
@@ -385,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
         };
 
         uint32_t g = 0;
-        Seq q;
+        Seq q{};
         q.start(P);
         for (; q.item >= 0; q.next(P), ++g) {
             const TProblem &pr = P.p[q.prob];
@@ -404,11 +409,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.raw_empty[slot]);
 
+            // Stage g-2: its MMAs were issued a whole iteration ago.  Reading
+            // its sums back also frees A[g&1] (the MMAs have finished reading
+            // it) and lets the MMAs of stage g reuse D[g&1].
+            if (g > 1 && !(ok = scale(g - 2))) break;
+
             // dequantize blocks 4*half .. 4*half+3 into 64 tensor-memory columns
             uint32_t cols[64];
-            float dcur[4];
-            if (half == 0) dequant_half<0>(w, cols, dcur);
-            else dequant_half<1>(w, cols, dcur);
+            Pending &pn = pend[g & 1];
+            if (half == 0) dequant_half<0>(w, cols, pn.d);
+            else dequant_half<1>(w, cols, pn.d);
+            pn.last = (q.stage == q.nstages - 1);
+            pn.prob = q.prob;
+            pn.row0 = q.row0;
             {
                 const uint32_t ta = tmem + lane_base + kACol + 128 * buf + 64 * half;
                 uint32_t lo[32], hi[32];
@@ -417,20 +430,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
                 tc_st_32(ta, lo);
                 tc_st_32(ta + 32, hi);
             }
-            // while the stores drain: finish the previous stage
-            if (g > 0 && !(ok = scale(g - 1))) break;
             tc_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.ab_full[buf]);
-
-            #pragma unroll
-            for (int jb = 0; jb < 4; ++jb) dprev[jb] = dcur[jb];
-            prev_last = (q.stage == q.nstages - 1);
-            prev_prob = q.prob;
-            prev_row0 = q.row0;
         }
-        if (ok && g > 0) scale(g - 1);
+        if (ok && g > 1) ok = scale(g - 2);
+        if (ok && g > 0) ok = scale(g - 1);
     }
 
     tc_fence_before();
