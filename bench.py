@@ -166,11 +166,23 @@ class GpuWorkload:
                 Y = torch.empty((lin.M, lin.N), dtype=torch.float32, device="cuda")
                 probs.append((W, X, Y, lin.M, lin.N, lin.K))
             self.sets.append((probs, q4.make_problems(probs)))
+        # the M > 32 GEMMs run through q4_0_gemm_ws with one shared workspace
+        # (X converted to fp16 once per GEMM); the M <= 32 ones in one grouped launch
+        self.small = [i for i, l in enumerate(wl.linears) if l.M <= 32]
+        self.large = [i for i, l in enumerate(wl.linears) if l.M > 32]
+        ws = max([q4.q4_0_gemm_workspace_size(l.M, l.N, l.K) for l in wl.linears] + [0])
+        self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device="cuda")
+        self.small_arrs = [q4.make_problems([probs[i] for i in self.small]) for probs, _ in self.sets]
         torch.cuda.synchronize()
 
     def launch(self, q4, step: int):
-        probs, arr = self.sets[step % len(self.sets)]
-        q4.q4_0_gemm_grouped(arr, len(probs))
+        k = step % len(self.sets)
+        probs, _ = self.sets[k]
+        if self.small:
+            q4.q4_0_gemm_grouped(self.small_arrs[k], len(self.small))
+        for i in self.large:
+            W, X, Y, M, N, K = probs[i]
+            q4.q4_0_gemm_ws(W, X, Y, M, N, K, self.ws)
 
 
 def run_ours(args, rank: int, world: int):
@@ -240,10 +252,10 @@ def run_ours(args, rank: int, world: int):
     e1 = torch.cuda.Event(enable_timing=True)
 
     def e2e_step(k):
-        probs, arr = G.sets[k % len(G.sets)]
+        probs, _ = G.sets[k % len(G.sets)]
         for (W, X, Y, *_), h in zip(probs, hx):
             X.copy_(h, non_blocking=True)
-        q4.q4_0_gemm_grouped(arr, len(probs))
+        G.launch(q4, k)
         for (W, X, Y, *_), h in zip(probs, hy):
             h.copy_(Y, non_blocking=True)
 
@@ -339,9 +351,10 @@ def whole_job_rate(units_per_rank_step: float, steps: int, world: int, max_ms: f
 
 
 def launches_per_step(name, wl) -> int:
-    # all M <= 32 problems of a step share one launch; each M > 32 problem is one launch
+    # all M <= 32 problems of a step share one launch; each M > 32 problem is
+    # two (the fp16 conversion of X, then the tensor-core GEMM)
     small = any(l.M <= 32 for l in wl.linears)
-    return int(small) + sum(1 for l in wl.linears if l.M > 32)
+    return int(small) + 2 * sum(1 for l in wl.linears if l.M > 32)
 
 
 # --------------------------------------------------------------------------- the oracle as a baseline

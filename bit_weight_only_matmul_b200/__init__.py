@@ -6,7 +6,7 @@ device addresses), passes their pointers, sizes and the current CUDA stream to
 the C entry point of the same name, and raises ``Q4Error`` on a non-zero
 status.  All arithmetic runs in the library's CUDA kernels; there is no CPU
 path.  Importing this package fails loudly if the library has not been built
-(``python -m bit_weight_only_matmul_b200.build``).
+(``python bit_weight_only_matmul_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -38,6 +38,8 @@ EXPORTS = (
     "q4_0_pack",
     "q4_0_dequant",
     "q4_0_gemm",
+    "q4_0_gemm_workspace_size",
+    "q4_0_gemm_ws",
     "q4_0_gemm_grouped",
     "q4_0_device_error",
     "q4_0_force_path",
@@ -60,7 +62,7 @@ class q4_0_problem(ctypes.Structure):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m bit_weight_only_matmul_b200.build`")
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python bit_weight_only_matmul_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     i64, vp, i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
     sig = {
@@ -70,6 +72,8 @@ def _load() -> ctypes.CDLL:
         "q4_0_pack": (i32, [vp, vp, vp, i64, i64, vp]),
         "q4_0_dequant": (i32, [vp, vp, i64, i64, vp]),
         "q4_0_gemm": (i32, [vp, vp, vp, i64, i64, i64, vp]),
+        "q4_0_gemm_workspace_size": (i64, [i64, i64, i64]),
+        "q4_0_gemm_ws": (i32, [vp, vp, vp, i64, i64, i64, vp, i64, vp]),
         "q4_0_gemm_grouped": (i32, [ctypes.POINTER(q4_0_problem), i32, vp]),
         "q4_0_device_error": (i32, [ctypes.POINTER(ctypes.c_uint32), i32]),
         "q4_0_force_path": (i32, [i32]),
@@ -127,6 +131,20 @@ def q4_0_dequant(W, out, N: int, K: int, stream=None) -> None:
 def q4_0_gemm(W, X, Y, M: int, N: int, K: int, stream=None) -> None:
     """Y[M,N] = X[M,K] * dequant(W)^T; X bf16 (or int16 bit patterns), Y fp32."""
     _check(_lib.q4_0_gemm(_ptr(W), _ptr(X), _ptr(Y), M, N, K, _stream(stream)), "q4_0_gemm")
+
+
+def q4_0_gemm_workspace_size(M: int, N: int, K: int) -> int:
+    return int(_lib.q4_0_gemm_workspace_size(M, N, K))
+
+
+def q4_0_gemm_ws(W, X, Y, M: int, N: int, K: int, workspace, workspace_bytes: Optional[int] = None,
+                 stream=None) -> None:
+    """q4_0_gemm with a device workspace (a CUDA tensor, its byte size taken
+    from the tensor unless given)."""
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.q4_0_gemm_ws(_ptr(W), _ptr(X), _ptr(Y), M, N, K, _ptr(workspace), workspace_bytes,
+                             _stream(stream)), "q4_0_gemm_ws")
 
 
 def make_problems(problems: Sequence) -> ctypes.Array:

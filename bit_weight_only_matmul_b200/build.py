@@ -1,6 +1,8 @@
 """Build libq4_0_b200.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m bit_weight_only_matmul_b200.build [--force] [--verbose]
+    python bit_weight_only_matmul_b200/build.py [--force] [--verbose] [--ptxas-info]
+
+(run it as a script: importing the package needs the library it builds).
 
 Each .cu under csrc/ is compiled to an object in _build/ (only when it or a
 header changed) and the objects are linked into

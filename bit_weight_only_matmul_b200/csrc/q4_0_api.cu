@@ -83,7 +83,7 @@ int check_problem(const q4_0_problem &p) {
 
 enum Path { kAuto = 0, kGeneric = 1, kDecode = 2, kTensor = 3, kDecodeMma = 4 };
 
-int run_problems(const q4_0_problem *probs, int count, cudaStream_t s) {
+int run_problems(const q4_0_problem *probs, int count, cudaStream_t s, void *ws = nullptr, int64_t ws_bytes = 0) {
     int st = Q4_OK;
     for (int i = 0; i < count; ++i) {
         st = check_problem(probs[i]);
@@ -124,7 +124,7 @@ int run_problems(const q4_0_problem *probs, int count, cudaStream_t s) {
     if (!dmma.empty()) e = q4::launch_decode(dmma.data(), static_cast<int>(dmma.size()), *dev, s);
     if (e != cudaSuccess) return cuda_fail(e);
     for (const q4::Problem &p : ten) {
-        e = q4::launch_prefill(p, *dev, s);
+        e = q4::launch_prefill(p, *dev, s, ws, ws_bytes);
         if (e != cudaSuccess) return cuda_fail(e);
     }
     if (!gen.empty()) e = q4::launch_generic(gen.data(), static_cast<int>(gen.size()), *dev, s);
@@ -187,6 +187,20 @@ int q4_0_gemm(const void *W, const uint16_t *X, float *Y, int64_t M, int64_t N, 
               q4_0_stream_t stream) {
     q4_0_problem p{W, X, Y, M, N, K};
     return run_problems(&p, 1, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int64_t q4_0_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
+    if (M < 0 || N < 0 || K < 0 || K % 32 != 0) return -1;
+    q4::Problem p{nullptr, nullptr, nullptr, M, N, K};
+    return q4::prefill_workspace_bytes(p);
+}
+
+int q4_0_gemm_ws(const void *W, const uint16_t *X, float *Y, int64_t M, int64_t N, int64_t K, void *workspace,
+                 int64_t workspace_bytes, q4_0_stream_t stream) {
+    if (workspace_bytes < 0 || (workspace_bytes > 0 && !workspace)) return Q4_ERR_INVALID_ARG;
+    if (workspace && !aligned16(workspace)) return Q4_ERR_MISALIGNED;
+    q4_0_problem p{W, X, Y, M, N, K};
+    return run_problems(&p, 1, reinterpret_cast<cudaStream_t>(stream), workspace, workspace_bytes);
 }
 
 int q4_0_gemm_grouped(const q4_0_problem *problems, int count, q4_0_stream_t stream) {

@@ -40,9 +40,13 @@ cudaError_t launch_decode(const Problem *probs, int count, const DeviceInfo &dev
 // problem must satisfy decode_tmem_supports().
 bool decode_tmem_supports(const Problem &p);
 cudaError_t launch_decode_tmem(const Problem *probs, int count, const DeviceInfo &dev, cudaStream_t s);
-// Tensor-core kernel: every problem must satisfy prefill_supports().
+// Tensor-core kernel: every problem must satisfy prefill_supports().  With a
+// workspace of at least prefill_workspace_bytes() X is converted to fp16 once
+// by a pre-pass; without one the kernel converts each X tile it loads.
 bool prefill_supports(const Problem &p);
-cudaError_t launch_prefill(const Problem &p, const DeviceInfo &dev, cudaStream_t s);
+int64_t prefill_workspace_bytes(const Problem &p);
+cudaError_t launch_prefill(const Problem &p, const DeviceInfo &dev, cudaStream_t s, void *workspace,
+                           int64_t workspace_bytes);
 
 }  // namespace q4
 

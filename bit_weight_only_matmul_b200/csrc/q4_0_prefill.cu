@@ -59,9 +59,12 @@ constexpr int kACol = 256;                     // A buffers: 32 columns each
 
 constexpr int kWarpTMA = 0, kWarpMMA = 1;
 constexpr int kWarpDeq0 = 2, kNumDeq = 4;      // warps 2..5
-constexpr int kWarpCvt0 = 6, kNumCvt = 8;      // warps 6..13
-constexpr int kWarpEpi0 = 14, kNumEpi = 4;     // warps 14..17
-constexpr int kThreads = 32 * (kWarpEpi0 + kNumEpi);   // 576
+constexpr int kWarpCvt0 = 6, kNumCvt = 8;      // warps 6..13 (X converted in the kernel)
+constexpr int kNumEpi = 4;                     // then 4 epilogue warps
+// XPRE: X arrives already in fp16 (converted once by the pre-pass into the
+// caller's workspace), so the eight conversion warps are not launched.
+template <bool XPRE> constexpr int epi_warp0() { return XPRE ? kWarpCvt0 : kWarpCvt0 + kNumCvt; }
+template <bool XPRE> constexpr int threads() { return 32 * (epi_warp0<XPRE>() + kNumEpi); }
 
 struct alignas(64) PrefillParams {
     CUtensorMap tmap_x;    // bf16 [M, K], box 64 x 256, 128-byte swizzle
@@ -153,7 +156,8 @@ __device__ __forceinline__ void block_words(const uint32_t (&raw)[36], int i, ui
 
 // ---------------------------------------------------------------- the kernel
 
-__global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ PrefillParams P) {
+template <bool XPRE>
+__global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __grid_constant__ PrefillParams P) {
     extern __shared__ uint8_t smem_raw[];
     Smem &S = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -232,7 +236,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 tc_fence_after();
                 for (int ks = 0; ks < ksteps; ++ks) {
                     const int sx = xc % kXStages, sa = ac % kAStages;
-                    if (!(ok = wait_or_abort(&S.x_conv[sx], (xc / kXStages) & 1, S, P.err))) break;
+                    if (!(ok = wait_or_abort(XPRE ? &S.x_full[sx] : &S.x_conv[sx], (xc / kXStages) & 1, S, P.err)))
+                        break;
                     if (!(ok = wait_or_abort(&S.a_full[sa], (ac / kAStages) & 1, S, P.err))) break;
                     tc_fence_after();
                     const uint64_t bdesc = sw128_desc(S.x[sx]);
@@ -300,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 }
             }
         }
-    } else if (warp >= kWarpCvt0 && warp < kWarpCvt0 + kNumCvt) {
+    } else if (!XPRE && warp >= kWarpCvt0 && warp < kWarpCvt0 + kNumCvt) {
         // each warp converts rows [32*cw, 32*cw + 32) of the stage; in one pass
         // 8 consecutive lanes take the 8 16-byte chunks of one row (the
         // conversion is chunk-local, so the swizzled order does not matter)
@@ -374,6 +379,27 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 
+// bf16 X -> fp16 X' in the permuted k order of the A operand (positions 1 and
+// 2 of every 4 swapped), 8 elements per thread.  Exact for |x| in the fp16
+// normal range.
+__global__ void x_to_fp16_kernel(const uint4 *__restrict__ X, uint4 *__restrict__ Xh, int64_t n8) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+        const uint4 v = __ldg(X + i);
+        const float f0 = __uint_as_float(v.x << 16), f1 = __uint_as_float(v.x & 0xFFFF0000u);
+        const float f2 = __uint_as_float(v.y << 16), f3 = __uint_as_float(v.y & 0xFFFF0000u);
+        const float f4 = __uint_as_float(v.z << 16), f5 = __uint_as_float(v.z & 0xFFFF0000u);
+        const float f6 = __uint_as_float(v.w << 16), f7 = __uint_as_float(v.w & 0xFFFF0000u);
+        __half2 h0 = __floats2half2_rn(f0, f2), h1 = __floats2half2_rn(f1, f3);
+        __half2 h2 = __floats2half2_rn(f4, f6), h3 = __floats2half2_rn(f5, f7);
+        uint4 o;
+        o.x = *reinterpret_cast<uint32_t *>(&h0);
+        o.y = *reinterpret_cast<uint32_t *>(&h1);
+        o.z = *reinterpret_cast<uint32_t *>(&h2);
+        o.w = *reinterpret_cast<uint32_t *>(&h3);
+        Xh[i] = o;
+    }
+}
+
 }  // namespace
 
 namespace q4 {
@@ -384,10 +410,27 @@ bool prefill_supports(const Problem &p) {
            (reinterpret_cast<uintptr_t>(p.X) & 15) == 0 && tensor_maps_available();
 }
 
-cudaError_t launch_prefill(const Problem &p, const DeviceInfo &dev, cudaStream_t s) {
+int64_t prefill_workspace_bytes(const Problem &p) {
+    return p.M > 32 ? ((p.M * p.K * 2 + 255) / 256) * 256 : 0;
+}
+
+cudaError_t launch_prefill(const Problem &p, const DeviceInfo &dev, cudaStream_t s, void *workspace,
+                           int64_t workspace_bytes) {
+    const bool xpre = workspace != nullptr && workspace_bytes >= prefill_workspace_bytes(p) &&
+                      (reinterpret_cast<uintptr_t>(workspace) & 15) == 0;
     PrefillParams local;
     std::memset(&local, 0, sizeof(local));
-    if (!get_tensor_map(&local.tmap_x, p.X, p.M, p.K, kMapActivationsSw128) ||
+    if (xpre) {
+        const int64_t n8 = p.M * p.K / 8;
+        const int64_t blocks = (n8 + 255) / 256;
+        const int grid = static_cast<int>(blocks < dev.sm_count * 8 ? blocks : dev.sm_count * 8);
+        x_to_fp16_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const uint4 *>(p.X), static_cast<uint4 *>(workspace),
+                                              n8);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (!get_tensor_map(&local.tmap_x, xpre ? workspace : p.X, p.M, p.K,
+                        xpre ? kMapActivationsF16Sw128 : kMapActivationsSw128) ||
         !get_tensor_map(&local.tmap_w, p.W, p.N, p.K / 32 * 18, kMapWeights128Prefill))
         return cudaErrorInvalidValue;
     local.Y = p.Y;
@@ -397,16 +440,27 @@ cudaError_t launch_prefill(const Problem &p, const DeviceInfo &dev, cudaStream_t
     local.K = static_cast<int>(p.K);
     local.tiles_n = static_cast<int>((p.N + kTileN - 1) / kTileN);
     local.tiles_m = static_cast<int>((p.M + kTileM - 1) / kTileM);
-    static int configured_device = -1;
-    if (configured_device != dev.device) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(kSmemBytes));
-        if (e != cudaSuccess) return e;
-        configured_device = dev.device;
-    }
     const int tiles = local.tiles_n * local.tiles_m;
     const int grid = tiles < dev.sm_count ? tiles : dev.sm_count;
-    prefill_kernel<<<grid, kThreads, kSmemBytes, s>>>(local);
+    if (xpre) {
+        static int configured_device = -1;
+        if (configured_device != dev.device) {
+            cudaError_t e = cudaFuncSetAttribute(prefill_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(kSmemBytes));
+            if (e != cudaSuccess) return e;
+            configured_device = dev.device;
+        }
+        prefill_kernel<true><<<grid, threads<true>(), kSmemBytes, s>>>(local);
+    } else {
+        static int configured_device = -1;
+        if (configured_device != dev.device) {
+            cudaError_t e = cudaFuncSetAttribute(prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(kSmemBytes));
+            if (e != cudaSuccess) return e;
+            configured_device = dev.device;
+        }
+        prefill_kernel<false><<<grid, threads<false>(), kSmemBytes, s>>>(local);
+    }
     return cudaGetLastError();
 }
 

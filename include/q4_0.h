@@ -123,6 +123,24 @@ Q4_0_API int q4_0_dequant(const void *W, float *out, int64_t N, int64_t K,
 Q4_0_API int q4_0_gemm(const void *W, const uint16_t *X, float *Y,
               int64_t M, int64_t N, int64_t K, q4_0_stream_t stream);
 
+/* Bytes of device workspace q4_0_gemm_ws can use for an (M, N, K) problem:
+ * M*K*2 rounded up to 256 when M > 32 (an fp16 copy of X for the
+ * tensor-core path), 0 when M <= 32.  -1 for invalid sizes. */
+Q4_0_API int64_t q4_0_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/* q4_0_gemm with a caller-provided device workspace (16-byte aligned, owned
+ * by the caller, contents overwritten).  With workspace_bytes >=
+ * q4_0_gemm_workspace_size(M, N, K), the tensor-core path (M > 32) first
+ * converts X to fp16 once in the workspace (one extra read and write of X)
+ * instead of converting every X tile in every CTA that loads it; with a
+ * smaller or NULL workspace it behaves exactly as q4_0_gemm.  Same results,
+ * bit for bit, either way.  Calls that share one workspace and overlap on
+ * the GPU race.  The pages have no counterpart: this is the B200 path's own
+ * trade of one pass over X against per-tile conversion work. */
+Q4_0_API int q4_0_gemm_ws(const void *W, const uint16_t *X, float *Y,
+                          int64_t M, int64_t N, int64_t K, void *workspace,
+                          int64_t workspace_bytes, q4_0_stream_t stream);
+
 /* One problem of a grouped launch: Y = X * dequant(W)^T, all device
  * pointers, same rules as q4_0_gemm. */
 typedef struct q4_0_problem {

@@ -99,3 +99,15 @@ def test_grouped_argument_checks(q4):
     assert gg(None, 0, None) == q4.Q4_OK
     empty = q4.make_problems([(None, None, None, 0, 8, 64)])
     assert gg(empty, 1, None) == q4.Q4_OK
+
+
+def test_workspace_size_and_checks(q4):
+    assert q4.q4_0_gemm_workspace_size(4096, 3072, 5120) == 4096 * 5120 * 2
+    assert q4.q4_0_gemm_workspace_size(33, 8, 32) == 2304   # 33*32*2 = 2112 -> 2304
+    assert q4.q4_0_gemm_workspace_size(32, 8, 64) == 0
+    assert q4.q4_0_gemm_workspace_size(4, 8, 33) == -1
+    ws = q4.lib.q4_0_gemm_ws
+    assert ws(A, A, A, 64, 8, 64, None, 16, None) == q4.Q4_ERR_INVALID_ARG    # bytes but no pointer
+    assert ws(A, A, A, 64, 8, 64, A + 4, 4096, None) == q4.Q4_ERR_MISALIGNED
+    assert ws(A, A, A, 64, 8, 64, A, -1, None) == q4.Q4_ERR_INVALID_ARG
+    assert ws(None, None, None, 0, 8, 64, None, 0, None) == q4.Q4_OK

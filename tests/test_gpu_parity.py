@@ -241,3 +241,37 @@ def test_decode_workloads_sampled(q4, name, layers):
     b = build_workload(q4, workloads.workload(name, layers=layers), samples=400)
     q4.q4_0_gemm_grouped(b.problems())
     check_built(b, name)
+
+
+@pytest.mark.parametrize("M,N,K", [(64, 128, 512), (300, 200, 1024), (4096, 256, 768)])
+def test_workspace_path_matches(q4, M, N, K):
+    """q4_0_gemm_ws (X converted to fp16 once, in the workspace) gives the
+    oracle's answer within tolerance and q4_0_gemm's answer bit for bit."""
+    rng = np.random.default_rng(M + N + K)
+    codes, scales, X = rand_inputs(rng, M, N, K, 0.5)
+    W = pack_on_gpu(q4, codes, scales)
+    Xd = dev(X)
+    ws_bytes = q4.q4_0_gemm_workspace_size(M, N, K)
+    assert ws_bytes == ((M * K * 2 + 255) // 256) * 256
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    Y1 = torch.full((M, N), float("nan"), device="cuda")
+    Y2 = torch.full((M, N), float("nan"), device="cuda")
+    q4.q4_0_gemm_ws(W, Xd, Y1, M, N, K, ws)
+    q4.q4_0_gemm(W, Xd, Y2, M, N, K)
+    torch.cuda.synchronize()
+    assert torch.equal(Y1, Y2)
+    Y_or, B_or = oracle.get().gemm(oracle.get().pack(codes, scales), X, M, N, K)
+    check_gemm(Y1.cpu().numpy(), Y_or, B_or, "workspace path")
+
+
+def test_workspace_too_small_falls_back(q4):
+    M, N, K = 64, 64, 512
+    rng = np.random.default_rng(4)
+    codes, scales, X = rand_inputs(rng, M, N, K, 0.5)
+    W = pack_on_gpu(q4, codes, scales)
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    Y = torch.empty((M, N), device="cuda")
+    q4.q4_0_gemm_ws(W, dev(X), Y, M, N, K, ws)
+    Y_or, B_or = oracle.get().gemm(oracle.get().pack(codes, scales), X, M, N, K)
+    check_gemm(Y.cpu().numpy(), Y_or, B_or, "small workspace")
+    assert q4.q4_0_gemm_workspace_size(8, 64, 512) == 0
