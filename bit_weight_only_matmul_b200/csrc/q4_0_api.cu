@@ -113,7 +113,7 @@ int run_problems(const q4_0_problem *probs, int count, cudaStream_t s, void *ws 
         else if (force == kDecode && (tmem_ok || mma_ok)) (tmem_ok ? dec : dmma).push_back(p);
         else if (force == kDecodeMma && mma_ok) dmma.push_back(p);
         else if (force == kTensor && ten_ok) ten.push_back(p);
-        else if (p.M <= 16 && tmem_ok) dec.push_back(p);
+        else if (p.M <= 32 && tmem_ok) dec.push_back(p);
         else if (p.M <= 32 && mma_ok) dmma.push_back(p);
         else if (p.M > 32 && ten_ok) ten.push_back(p);
         else gen.push_back(p);

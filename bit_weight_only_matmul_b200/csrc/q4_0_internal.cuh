@@ -36,7 +36,7 @@ cudaError_t launch_generic(const Problem *probs, int count, const DeviceInfo &de
 // decode_supports().
 bool decode_supports(const Problem &p);
 cudaError_t launch_decode(const Problem *probs, int count, const DeviceInfo &dev, cudaStream_t s);
-// Decode kernel on tcgen05 with weights in tensor memory (M <= 16): every
+// Decode kernel on tcgen05 with weights in tensor memory (M <= 32): every
 // problem must satisfy decode_tmem_supports().
 bool decode_tmem_supports(const Problem &p);
 cudaError_t launch_decode_tmem(const Problem *probs, int count, const DeviceInfo &dev, cudaStream_t s);
