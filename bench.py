@@ -48,10 +48,10 @@ DEFAULT_WORKLOAD = "layer"
 
 # kernel that dominates each workload, and the source file it lives in
 DOMINANT = {
-    "gemv": ("decode_tmem_kernel", "q4_0_decode_tmem.cu"),
-    "layer": ("decode_tmem_kernel", "q4_0_decode_tmem.cu"),
-    "cfg_decode": ("decode_tmem_kernel", "q4_0_decode_tmem.cu"),
-    "concurrent": ("decode_kernel", "q4_0_decode.cu"),
+    "gemv": ("decode_mma_kernel", "q4_0_decode_mma.cu"),
+    "layer": ("decode_mma_kernel", "q4_0_decode_mma.cu"),
+    "cfg_decode": ("decode_mma_kernel", "q4_0_decode_mma.cu"),
+    "concurrent": ("decode_mma_kernel", "q4_0_decode_mma.cu"),
     "adapter": ("prefill_kernel", "q4_0_prefill.cu"),
     "qkv_prefill": ("prefill_kernel", "q4_0_prefill.cu"),
 }

@@ -24,11 +24,10 @@ Q4_ERR_UNSUPPORTED_DEVICE = 3
 Q4_ERR_CUDA = 4
 
 Q4_DEVERR_WAIT_TIMEOUT = 1
-Q4_DEVERR_FP16_RANGE = 2
 
 Q4_0_MAX_GROUP = 256
 
-PATH_AUTO, PATH_GENERIC, PATH_DECODE, PATH_TENSOR, PATH_DECODE_MMA = 0, 1, 2, 3, 4
+PATH_AUTO, PATH_GENERIC, PATH_DECODE, PATH_TENSOR, PATH_DECODE_EXACT, PATH_DECODE_TMEM = 0, 1, 2, 3, 4, 5
 
 # every symbol include/q4_0.h declares
 EXPORTS = (

@@ -81,7 +81,7 @@ int check_problem(const q4_0_problem &p) {
     return Q4_OK;
 }
 
-enum Path { kAuto = 0, kGeneric = 1, kDecode = 2, kTensor = 3, kDecodeMma = 4 };
+enum Path { kAuto = 0, kGeneric = 1, kDecode = 2, kTensor = 3, kDecodeExact = 4, kDecodeTmem = 5 };
 
 int run_problems(const q4_0_problem *probs, int count, cudaStream_t s, void *ws = nullptr, int64_t ws_bytes = 0) {
     int st = Q4_OK;
@@ -96,7 +96,7 @@ int run_problems(const q4_0_problem *probs, int count, cudaStream_t s, void *ws 
     st = current_device(&dev);
     if (st != Q4_OK) return st;
     const int force = g_force_path.load(std::memory_order_relaxed);
-    std::vector<q4::Problem> dec, dmma, gen, ten;
+    std::vector<q4::Problem> dec, dexact, dtmem, gen, ten;
     for (int i = 0; i < count; ++i) {
         const q4_0_problem &a = probs[i];
         if (a.M == 0 || a.N == 0) continue;
@@ -106,22 +106,25 @@ int run_problems(const q4_0_problem *probs, int count, cudaStream_t s, void *ws 
             continue;
         }
         q4::Problem p{static_cast<const uint8_t *>(a.W), a.X, a.Y, a.M, a.N, a.K};
+        const bool dec_ok = q4::decode_mma_supports(p);
+        const bool exact_ok = q4::decode_supports(p);
         const bool tmem_ok = q4::decode_tmem_supports(p);
-        const bool mma_ok = q4::decode_supports(p);
         const bool ten_ok = q4::prefill_supports(p);
         if (force == kGeneric) gen.push_back(p);
-        else if (force == kDecode && (tmem_ok || mma_ok)) (tmem_ok ? dec : dmma).push_back(p);
-        else if (force == kDecodeMma && mma_ok) dmma.push_back(p);
+        else if (force == kDecode && dec_ok) dec.push_back(p);
+        else if (force == kDecodeExact && exact_ok) dexact.push_back(p);
+        else if (force == kDecodeTmem && tmem_ok) dtmem.push_back(p);
         else if (force == kTensor && ten_ok) ten.push_back(p);
-        else if (p.M <= 32 && tmem_ok) dec.push_back(p);
-        else if (p.M <= 32 && mma_ok) dmma.push_back(p);
+        else if (p.M <= 32 && dec_ok) dec.push_back(p);
         else if (p.M > 32 && ten_ok) ten.push_back(p);
         else gen.push_back(p);
     }
     cudaError_t e = cudaSuccess;
-    if (!dec.empty()) e = q4::launch_decode_tmem(dec.data(), static_cast<int>(dec.size()), *dev, s);
+    if (!dec.empty()) e = q4::launch_decode_mma(dec.data(), static_cast<int>(dec.size()), *dev, s);
     if (e != cudaSuccess) return cuda_fail(e);
-    if (!dmma.empty()) e = q4::launch_decode(dmma.data(), static_cast<int>(dmma.size()), *dev, s);
+    if (!dexact.empty()) e = q4::launch_decode(dexact.data(), static_cast<int>(dexact.size()), *dev, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (!dtmem.empty()) e = q4::launch_decode_tmem(dtmem.data(), static_cast<int>(dtmem.size()), *dev, s);
     if (e != cudaSuccess) return cuda_fail(e);
     for (const q4::Problem &p : ten) {
         e = q4::launch_prefill(p, *dev, s, ws, ws_bytes);
@@ -231,7 +234,7 @@ int q4_0_device_error(uint32_t *flags, int clear) {
 }
 
 int q4_0_force_path(int path) {
-    if (path < 0 || path > 4) return Q4_ERR_INVALID_ARG;
+    if (path < 0 || path > 5) return Q4_ERR_INVALID_ARG;
     g_force_path.store(path, std::memory_order_relaxed);
     return Q4_OK;
 }

@@ -1,0 +1,361 @@
+// q4_0_decode_mma.cu -- the memory-bound decode path (M <= 32): one
+// persistent launch streams the Q4_0 weights of one or many problems once
+// from HBM, dequantizes them in registers and multiplies them with the few
+// activation rows on the warp-level tensor cores (mma.sync).
+//
+// The pages' token loop runs a Q4 matmul for every decoder linear of each of
+// the 26 layers (voxtral-mini-realtime-rs (Shannon-Prime fork) README,
+// "Architecture Summary"; decode is most of the time: "Pipeline Overlap"),
+// with batch-2 CFG and fused QKV / gate-up projections ("TTS
+// (Text-to-Speech)", optimizations), and up to 32 concurrent sequences in the
+// Tenstorrent port (Voxtral-Mini-4B-Realtime-2602-tt-p300x2 README, serving).
+//
+// Why mma.sync and not tcgen05: a tcgen05.mma with M=128, K=16 takes ~112
+// cycles whatever N (measured), so with the weights as its A operand an SM
+// turns at most ~18 weights per cycle into products -- about 3 TB/s of Q4_0 on
+// B200, half of what HBM delivers.  The warp-level m16n8k16 has no such floor,
+// and its n=8 matches the few activation rows.
+//
+// Per CTA (one per SM): a producer warp, an X warp and 16 compute warps.
+//  * stage = 256 k of an item (128 weight rows x 144 bytes, one TMA box) plus
+//    the same 256 k of every row of X (1-D bulk copies), in a 4-6-deep ring;
+//    the TMA box pattern alone streams at ~6.9 TB/s (measured);
+//  * the X warp converts the stage's X rows to fp16 straight into mma.sync B
+//    fragments (three buffers), so a compute thread loads each fragment with
+//    one 8-byte shared load;
+//  * compute warp (tile, half) takes 16 weight rows and blocks 4*half ..
+//    4*half+3 of each stage; each thread turns one 4-byte code word of two
+//    rows into fp16 (q - 8) * d pairs -- the A fragments of two MMAs -- and
+//    accumulates across the whole item in fp32 mma.sync accumulators;
+//  * at the end of an item the two halves of a tile add their sums and store
+//    Y[m, n].
+// Numerics: each weight is rounded once to fp16 (relative error <= 2^-11,
+// inside the 1e-3 tolerance of the method); X is exact in fp16 within its
+// normal range; products are exact and accumulation is fp32.  Operands beyond
+// the fp16 range (|x| > 65504, |d| > 8188) overflow to +-inf.
+#include <cuda_fp16.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "q4_0_convert.cuh"
+#include "q4_0_internal.cuh"
+#include "q4_0_sched.cuh"
+#include "q4_0_tcgen05.cuh"
+#include "q4_0_tmap.cuh"
+
+namespace {
+
+using namespace q4dev;
+
+constexpr int kRawW = kItemRows * kStageRowBytes;   // 18432
+constexpr int kXRow = kStageK * 2;                  // 512 bytes of one bf16 X row per stage
+constexpr int kXBufs = 3;
+constexpr int kWarpProd = 0, kWarpX = 1, kWarp0 = 2, kCompute = 16;
+constexpr int kThreads = 32 * (kWarp0 + kCompute);  // 576
+
+// NT = n8 tiles of X rows (M <= 8*NT)
+template <int NT> constexpr int raw_bytes() { return kRawW + 8 * NT * kXRow; }
+template <int NT> constexpr int ring() { return NT == 4 ? 4 : 6; }
+
+template <int NT>
+struct Smem {
+    uint8_t raw[ring<NT>()][raw_bytes<NT>()];   // W rows (pitch 144) then X rows (pitch 512)
+    uint2 xf[kXBufs][8][2][NT][32];             // B fragments: [block][k16 slice][n tile][lane]
+    float comb[2][8][NT][4][32];                // half-1 sums handed to half 0 at an item's end
+    uint64_t raw_full[ring<NT>()], raw_empty[ring<NT>()];
+    uint64_t xf_full[kXBufs], xf_empty[kXBufs];
+    uint64_t comb_full[2], comb_empty[2];
+    int abort_flag;
+};
+
+__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint2 b) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b.x), "r"(b.y));
+}
+
+// Scale (d, d) and qs word t of block i (byte offset 18*i of a 144-byte stage
+// row starting 4-byte aligned at `row`): even blocks start 4-byte aligned,
+// odd ones at 2 mod 4.
+template <int I>
+__device__ __forceinline__ void block_word(const uint8_t *row, int t, uint32_t &d2, uint32_t &qw) {
+    constexpr int off = 18 * I;
+    if constexpr ((I & 1) == 0) {
+        const uint32_t w0 = *reinterpret_cast<const uint32_t *>(row + off + 4 * t);
+        const uint32_t w1 = *reinterpret_cast<const uint32_t *>(row + off + 4 * t + 4);
+        const uint32_t wd = *reinterpret_cast<const uint32_t *>(row + off);
+        d2 = prmt(wd, wd, 0x1010u);
+        qw = prmt(w0, w1, 0x5432u);
+    } else {
+        const uint32_t wd = *reinterpret_cast<const uint32_t *>(row + off - 2);
+        d2 = prmt(wd, wd, 0x3232u);
+        qw = *reinterpret_cast<const uint32_t *>(row + off + 2 + 4 * t);
+    }
+}
+
+template <int NT, int I>
+__device__ __forceinline__ void block_mma(const uint8_t *rowg, const uint8_t *rowg8, int t,
+                                          const uint2 (&xf)[8][2][NT][32], int lane, float (&acc)[NT][4]) {
+    uint32_t dg, dg8, qg, qg8;
+    block_word<I>(rowg, t, dg, qg);
+    block_word<I>(rowg8, t, dg8, qg8);
+    uint32_t cg[4], cg8[4];
+    q4_word_to_fp16(qg, dg, cg);
+    q4_word_to_fp16(qg8, dg8, cg8);
+    // slice 0: k cols (2t,2t+1) <- elements (4t,4t+2), (2t+8,2t+9) <- (4t+1,4t+3); slice 1: +16
+    #pragma unroll
+    for (int j = 0; j < NT; ++j) {
+        mma_f16(acc[j], cg[0], cg8[0], cg[1], cg8[1], xf[I][0][j][lane]);
+        mma_f16(acc[j], cg[2], cg8[2], cg[3], cg8[3], xf[I][1][j][lane]);
+    }
+}
+
+template <int NT, int CAP>
+__global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_constant__ GroupParams<CAP> P) {
+    constexpr int RS = ring<NT>();
+    extern __shared__ uint8_t smem_raw[];
+    using SM = Smem<NT>;
+    SM &S = *reinterpret_cast<SM *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < RS; ++s) {
+            mbar_init(&S.raw_full[s], 1);
+            mbar_init(&S.raw_empty[s], kCompute + 1);
+        }
+        for (int s = 0; s < kXBufs; ++s) {
+            mbar_init(&S.xf_full[s], 1);
+            mbar_init(&S.xf_empty[s], kCompute);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&S.comb_full[s], kCompute / 2);
+            mbar_init(&S.comb_empty[s], kCompute / 2);
+        }
+        S.abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    uint32_t prod_issued = 0;
+
+    if (warp == kWarpProd) {
+        // ---------------------------------------------------------------- loads
+        Seq q{};
+        q.start(P);
+        for (; q.item >= 0; q.next(P)) {
+            const GroupProblem &pr = P.p[q.prob];
+            const uint32_t g = prod_issued;
+            const int slot = g % RS;
+            bool ok = true;
+            if (lane == 0) ok = wait_or_abort(&S.raw_empty[slot], ((g / RS) & 1) ^ 1, &S.abort_flag, P.err);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            // weights: one TMA box (rows past N are zero-filled and still counted)
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&S.raw_full[slot], kRawW + pr.M * kXRow);
+                tma_load_2d(S.raw[slot], &P.wmap[q.prob], q.stage * kStageRowBytes, q.row0, &S.raw_full[slot]);
+            }
+            __syncwarp();
+            for (int m = lane; m < pr.M; m += 32)
+                bulk_g2s(S.raw[slot] + kRawW + m * kXRow,
+                         pr.X + static_cast<int64_t>(m) * pr.K + static_cast<int64_t>(q.stage) * kStageK, kXRow,
+                         &S.raw_full[slot]);
+            ++prod_issued;
+        }
+    } else if (warp == kWarpX) {
+        // ---------------------------------------------------------------- X rows -> fp16 B fragments
+        const int gx = lane >> 2, tx = lane & 3;   // this lane's fragment column (X row) and k group
+        uint32_t g = 0;
+        Seq q{};
+        q.start(P);
+        for (; q.item >= 0; q.next(P), ++g) {
+            const GroupProblem &pr = P.p[q.prob];
+            const int slot = g % RS, xb = g % kXBufs;
+            bool ok = true;
+            if (lane == 0) {
+                ok = wait_or_abort(&S.raw_full[slot], (g / RS) & 1, &S.abort_flag, P.err);
+                if (ok) ok = wait_or_abort(&S.xf_empty[xb], ((g / kXBufs) & 1) ^ 1, &S.abort_flag, P.err);
+            }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            const uint8_t *xr = S.raw[slot] + kRawW;
+            #pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                const int m = 8 * j + gx;
+                #pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    #pragma unroll
+                    for (int s = 0; s < 2; ++s) {
+                        uint2 o = make_uint2(0u, 0u);
+                        if (m < pr.M) {
+                            const uint2 v = *reinterpret_cast<const uint2 *>(xr + m * kXRow + 2 * (32 * i + 16 * s + 4 * tx));
+                            o = x4_to_fp16_permuted(v.x, v.y);
+                        }
+                        S.xf[xb][i][s][j][lane] = o;
+                    }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&S.xf_full[xb]);
+                mbar_arrive(&S.raw_empty[slot]);
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------- compute
+        const int cw = warp - kWarp0;
+        const int tile = cw >> 1, half = cw & 1;
+        const int gq = lane >> 2, t = lane & 3;
+        float acc[NT][4];
+        #pragma unroll
+        for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+        uint32_t g = 0, items_done = 0;
+        Seq q{};
+        q.start(P);
+        for (; q.item >= 0; q.next(P), ++g) {
+            const int slot = g % RS, xb = g % kXBufs;
+            if (!wait_or_abort(&S.raw_full[slot], (g / RS) & 1, &S.abort_flag, P.err)) break;
+            if (!wait_or_abort(&S.xf_full[xb], (g / kXBufs) & 1, &S.abort_flag, P.err)) break;
+            const uint8_t *rowg = S.raw[slot] + (16 * tile + gq) * kStageRowBytes;
+            const uint8_t *rowg8 = rowg + 8 * kStageRowBytes;
+            if (half == 0) {
+                block_mma<NT, 0>(rowg, rowg8, t, S.xf[xb], lane, acc);
+                block_mma<NT, 1>(rowg, rowg8, t, S.xf[xb], lane, acc);
+                block_mma<NT, 2>(rowg, rowg8, t, S.xf[xb], lane, acc);
+                block_mma<NT, 3>(rowg, rowg8, t, S.xf[xb], lane, acc);
+            } else {
+                block_mma<NT, 4>(rowg, rowg8, t, S.xf[xb], lane, acc);
+                block_mma<NT, 5>(rowg, rowg8, t, S.xf[xb], lane, acc);
+                block_mma<NT, 6>(rowg, rowg8, t, S.xf[xb], lane, acc);
+                block_mma<NT, 7>(rowg, rowg8, t, S.xf[xb], lane, acc);
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&S.raw_empty[slot]);
+                mbar_arrive(&S.xf_empty[xb]);
+            }
+            if (q.stage == q.nstages - 1) {
+                // end of the item: the two halves of the tile add their sums
+                const GroupProblem &pr = P.p[q.prob];
+                const int cb = items_done & 1;
+                const uint32_t par = (items_done >> 1) & 1;
+                if (half == 1) {
+                    if (!wait_or_abort(&S.comb_empty[cb], par ^ 1, &S.abort_flag, P.err)) break;
+                    #pragma unroll
+                    for (int j = 0; j < NT; ++j)
+                        #pragma unroll
+                        for (int e = 0; e < 4; ++e) S.comb[cb][tile][j][e][lane] = acc[j][e];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.comb_full[cb]);
+                } else {
+                    if (!wait_or_abort(&S.comb_full[cb], par, &S.abort_flag, P.err)) break;
+                    #pragma unroll
+                    for (int j = 0; j < NT; ++j)
+                        #pragma unroll
+                        for (int e = 0; e < 4; ++e) acc[j][e] += S.comb[cb][tile][j][e][lane];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.comb_empty[cb]);
+                    // thread holds rows gq / gq+8 of the tile x columns 8j+2t, 8j+2t+1
+                    #pragma unroll
+                    for (int j = 0; j < NT; ++j)
+                        #pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int m = 8 * j + 2 * t + (e & 1);
+                            const int n = q.row0 + 16 * tile + gq + ((e & 2) ? 8 : 0);
+                            if (m < pr.M && n < pr.N) pr.Y[static_cast<int64_t>(m) * pr.N + n] = acc[j][e];
+                        }
+                }
+                #pragma unroll
+                for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+                ++items_done;
+            }
+        }
+    }
+
+    __syncthreads();
+    // Abort path: copies issued but never consumed may still be in flight;
+    // let them land (bounded) before the CTA exits.
+    if (*reinterpret_cast<volatile int *>(&S.abort_flag) && warp == kWarpProd && lane == 0) {
+        for (uint32_t i = 0; i < RS && i < prod_issued; ++i) {
+            const uint32_t gg = prod_issued - 1 - i;
+            mbar_wait(&S.raw_full[gg % RS], (gg / RS) & 1, P.err);
+        }
+    }
+}
+
+template <int NT>
+constexpr size_t smem_bytes() { return sizeof(Smem<NT>) + 128; }
+static_assert(smem_bytes<4>() <= 232448, "shared memory budget");
+
+template <int NT, int CAP>
+cudaError_t launch_nt(GroupParams<CAP> &P, const q4::DeviceInfo &dev, cudaStream_t s) {
+    static int configured_device = -1;
+    if (configured_device != dev.device) {
+        cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<NT, CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem_bytes<NT>()));
+        if (e != cudaSuccess) return e;
+        configured_device = dev.device;
+    }
+    const int grid = std::max(1, std::min(dev.sm_count, P.total_items));
+    decode_mma_kernel<NT, CAP><<<grid, kThreads, smem_bytes<NT>(), s>>>(P);
+    return cudaGetLastError();
+}
+
+// problems[order[0..count)] sorted by K (largest first), count <= CAP
+template <int CAP>
+cudaError_t launch_cap(const q4::Problem *probs, const int *order, int count, const q4::DeviceInfo &dev,
+                       cudaStream_t s) {
+    static thread_local GroupParams<CAP> P;
+    P.count = count;
+    P.err = dev.err;
+    int items = 0;
+    int64_t maxM = 1;
+    for (int i = 0; i < count; ++i) {
+        const q4::Problem &q = probs[order[i]];
+        GroupProblem &t = P.p[i];
+        t.W = q.W;
+        t.X = q.X;
+        t.Y = q.Y;
+        t.M = static_cast<int>(q.M);
+        t.N = static_cast<int>(q.N);
+        t.K = static_cast<int>(q.K);
+        t.stages = static_cast<int>(q.K / kStageK);
+        t.item_begin = items;
+        items += static_cast<int>((q.N + kItemRows - 1) / kItemRows);
+        maxM = std::max(maxM, q.M);
+        if (!q4::get_tensor_map(&P.wmap[i], q.W, q.N, q.K / 32 * 18, q4::kMapWeights128))
+            return cudaErrorInvalidValue;
+    }
+    P.total_items = items;
+    if (maxM <= 8) return launch_nt<1, CAP>(P, dev, s);
+    if (maxM <= 16) return launch_nt<2, CAP>(P, dev, s);
+    return launch_nt<4, CAP>(P, dev, s);
+}
+
+constexpr int kSmallCap = 8, kLargeCap = 128;
+
+}  // namespace
+
+namespace q4 {
+
+bool decode_mma_supports(const Problem &p) {
+    return p.M >= 1 && p.M <= 32 && p.K >= kStageK && p.K % kStageK == 0 && p.N >= 1 && p.N < (1LL << 31) &&
+           p.K < (1LL << 31) && (reinterpret_cast<uintptr_t>(p.W) & 15) == 0 &&
+           (reinterpret_cast<uintptr_t>(p.X) & 15) == 0 && tensor_maps_available();
+}
+
+cudaError_t launch_decode_mma(const Problem *probs, int count, const DeviceInfo &dev, cudaStream_t s) {
+    if (count <= 0) return cudaSuccess;
+    std::vector<int> order(count);
+    for (int i = 0; i < count; ++i) order[i] = i;
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return probs[a].K > probs[b].K; });
+    for (int done = 0; done < count;) {
+        const int n = std::min(count - done, kLargeCap);
+        cudaError_t e = n <= kSmallCap ? launch_cap<kSmallCap>(probs, order.data() + done, n, dev, s)
+                                       : launch_cap<kLargeCap>(probs, order.data() + done, n, dev, s);
+        if (e != cudaSuccess) return e;
+        done += n;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace q4

@@ -49,6 +49,7 @@
 #include <vector>
 
 #include "q4_0_internal.cuh"
+#include "q4_0_convert.cuh"
 #include "q4_0_tcgen05.cuh"
 #include "q4_0_tmap.cuh"
 
@@ -155,30 +156,6 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, S 
     return true;
 }
 
-// fp16 pairs of (q - 8) * d for one qs word v (bytes 4w .. 4w+3 of a block):
-//   c[0] = elements (4w, 4w+2), c[1] = (4w+1, 4w+3)        (low nibbles)
-//   c[2] = elements (4w+16, 4w+18), c[3] = (4w+17, 4w+19)  (high nibbles)
-// 0x6400 is fp16 1024 (10 fraction bits): 1024 + q and 1024 + 16q are exact,
-// and so are (1024 + q) - 1032 and (1024 + 16q) / 16 - 72 = q - 8; the only
-// rounding is the product with d.
-__device__ __forceinline__ void dequant_word(uint32_t v, uint32_t d2, uint32_t (&c)[4]) {
-    const uint32_t v8 = v >> 8;
-    const __half2 k1032 = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
-    const __half2 k16th = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
-    const __half2 km72 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));
-    const __half2 d = *reinterpret_cast<const __half2 *>(&d2);
-    uint32_t t[4] = {and_or(v, 0x000F000Fu, 0x64006400u), and_or(v8, 0x000F000Fu, 0x64006400u),
-                     and_or(v, 0x00F000F0u, 0x64006400u), and_or(v8, 0x00F000F0u, 0x64006400u)};
-    __half2 r0 = __hmul2(__hsub2(*reinterpret_cast<__half2 *>(&t[0]), k1032), d);
-    __half2 r1 = __hmul2(__hsub2(*reinterpret_cast<__half2 *>(&t[1]), k1032), d);
-    __half2 r2 = __hmul2(__hfma2(*reinterpret_cast<__half2 *>(&t[2]), k16th, km72), d);
-    __half2 r3 = __hmul2(__hfma2(*reinterpret_cast<__half2 *>(&t[3]), k16th, km72), d);
-    c[0] = *reinterpret_cast<uint32_t *>(&r0);
-    c[1] = *reinterpret_cast<uint32_t *>(&r1);
-    c[2] = *reinterpret_cast<uint32_t *>(&r2);
-    c[3] = *reinterpret_cast<uint32_t *>(&r3);
-}
-
 // Blocks 4*HALF .. 4*HALF+3 of a stage row, held in w[] = bytes
 // [64*HALF, 64*HALF + 80) of the 144-byte row: 64 tensor-memory columns (16
 // per block, fp16 pairs in the permuted k order above).  Blocks at an even
@@ -202,29 +179,13 @@ __device__ __forceinline__ void dequant_half(const uint32_t (&w)[20], uint32_t (
         #pragma unroll
         for (int k = 0; k < 4; ++k) {
             uint32_t c[4];
-            dequant_word(qw[k], d2, c);
+            q4_word_to_fp16(qw[k], d2, c);
             cols[16 * jb + 2 * k] = c[0];
             cols[16 * jb + 2 * k + 1] = c[1];
             cols[16 * jb + 8 + 2 * k] = c[2];
             cols[16 * jb + 8 + 2 * k + 1] = c[3];
         }
     }
-}
-
-// bf16 (x0..x7) -> fp16 pairs (x0,x2) (x1,x3) (x4,x6) (x5,x7).
-__device__ __forceinline__ uint4 x8_to_fp16_permuted(uint4 v) {
-    const float f0 = __uint_as_float(v.x << 16), f1 = __uint_as_float(v.x & 0xFFFF0000u);
-    const float f2 = __uint_as_float(v.y << 16), f3 = __uint_as_float(v.y & 0xFFFF0000u);
-    const float f4 = __uint_as_float(v.z << 16), f5 = __uint_as_float(v.z & 0xFFFF0000u);
-    const float f6 = __uint_as_float(v.w << 16), f7 = __uint_as_float(v.w & 0xFFFF0000u);
-    __half2 h0 = __floats2half2_rn(f0, f2), h1 = __floats2half2_rn(f1, f3);
-    __half2 h2 = __floats2half2_rn(f4, f6), h3 = __floats2half2_rn(f5, f7);
-    uint4 o;
-    o.x = *reinterpret_cast<uint32_t *>(&h0);
-    o.y = *reinterpret_cast<uint32_t *>(&h1);
-    o.z = *reinterpret_cast<uint32_t *>(&h2);
-    o.w = *reinterpret_cast<uint32_t *>(&h3);
-    return o;
 }
 
 template <int NN, int CAP>

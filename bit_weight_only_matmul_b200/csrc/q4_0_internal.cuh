@@ -32,8 +32,12 @@ cudaError_t launch_pack(const uint8_t *codes, const uint16_t *scales, uint8_t *W
 cudaError_t launch_dequant(const uint8_t *W, float *out, int64_t N, int64_t K, cudaStream_t s);
 cudaError_t launch_zero(float *Y, int64_t count, cudaStream_t s);
 cudaError_t launch_generic(const Problem *probs, int count, const DeviceInfo &dev, cudaStream_t s);
-// Decode kernel on warp-level mma.sync (M <= 32): every problem must satisfy
-// decode_supports().
+// Decode kernel on warp-level mma.sync with fp16 weights (M <= 32), the
+// default decode path: every problem must satisfy decode_mma_supports().
+bool decode_mma_supports(const Problem &p);
+cudaError_t launch_decode_mma(const Problem *probs, int count, const DeviceInfo &dev, cudaStream_t s);
+// Exact-arithmetic decode kernel on warp-level mma.sync (bf16 (q - 8), fp32
+// scale per block; M <= 32): every problem must satisfy decode_supports().
 bool decode_supports(const Problem &p);
 cudaError_t launch_decode(const Problem *probs, int count, const DeviceInfo &dev, cudaStream_t s);
 // Decode kernel on tcgen05 with weights in tensor memory (M <= 32): every

@@ -35,6 +35,7 @@
 #include <mutex>
 
 #include "q4_0_internal.cuh"
+#include "q4_0_convert.cuh"
 #include "q4_0_tcgen05.cuh"
 #include "q4_0_tmap.cuh"
 
@@ -113,30 +114,6 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, Sm
 }
 
 // ---------------------------------------------------------------- dequantization
-
-// fp16 pairs of (q - 8) * d for one qs word v (bytes 4w .. 4w+3 of a block):
-//   c[0] = elements (4w, 4w+2), c[1] = (4w+1, 4w+3)        (low nibbles)
-//   c[2] = elements (4w+16, 4w+18), c[3] = (4w+17, 4w+19)  (high nibbles)
-// 0x6400 is fp16 1024 (10 fraction bits): 1024 + q and 1024 + 16q are exact,
-// and so are (1024 + q) - 1032 and (1024 + 16q) / 16 - 72 = q - 8; the only
-// rounding is the final product with d.
-__device__ __forceinline__ void dequant_word(uint32_t v, uint32_t d2, uint32_t (&c)[4]) {
-    const uint32_t v8 = v >> 8;
-    const __half2 k1032 = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
-    const __half2 k16th = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
-    const __half2 km72 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));
-    const __half2 d = *reinterpret_cast<const __half2 *>(&d2);
-    uint32_t t[4] = {and_or(v, 0x000F000Fu, 0x64006400u), and_or(v8, 0x000F000Fu, 0x64006400u),
-                     and_or(v, 0x00F000F0u, 0x64006400u), and_or(v8, 0x00F000F0u, 0x64006400u)};
-    __half2 r0 = __hmul2(__hsub2(*reinterpret_cast<__half2 *>(&t[0]), k1032), d);
-    __half2 r1 = __hmul2(__hsub2(*reinterpret_cast<__half2 *>(&t[1]), k1032), d);
-    __half2 r2 = __hmul2(__hfma2(*reinterpret_cast<__half2 *>(&t[2]), k16th, km72), d);
-    __half2 r3 = __hmul2(__hfma2(*reinterpret_cast<__half2 *>(&t[3]), k16th, km72), d);
-    c[0] = *reinterpret_cast<uint32_t *>(&r0);
-    c[1] = *reinterpret_cast<uint32_t *>(&r1);
-    c[2] = *reinterpret_cast<uint32_t *>(&r2);
-    c[3] = *reinterpret_cast<uint32_t *>(&r3);
-}
 
 // Block i (0..7) of a 144-byte raw row held in 36 registers: the fp16 scale
 // bits and the four qs words.
@@ -289,7 +266,7 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
                         #pragma unroll
                         for (int w = 0; w < 4; ++w) {
                             uint32_t c[4];
-                            dequant_word(q[w], d2, c);
+                            q4_word_to_fp16(q[w], d2, c);
                             cols[16 * h + 2 * w] = c[0];
                             cols[16 * h + 2 * w + 1] = c[1];
                             cols[16 * h + 8 + 2 * w] = c[2];
@@ -320,19 +297,7 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
                 for (int it = 0; it < 8; ++it) {
                     const int row = 32 * cw + 4 * it + (lane >> 3);
                     uint4 *p = reinterpret_cast<uint4 *>(S.x[s] + row * 128 + 16 * (lane & 7));
-                    const uint4 v = *p;
-                    // bf16 (x0..x7) -> fp16 pairs (x0,x2) (x1,x3) (x4,x6) (x5,x7)
-                    const float f0 = __uint_as_float(v.x << 16), f1 = __uint_as_float(v.x & 0xFFFF0000u);
-                    const float f2 = __uint_as_float(v.y << 16), f3 = __uint_as_float(v.y & 0xFFFF0000u);
-                    const float f4 = __uint_as_float(v.z << 16), f5 = __uint_as_float(v.z & 0xFFFF0000u);
-                    const float f6 = __uint_as_float(v.w << 16), f7 = __uint_as_float(v.w & 0xFFFF0000u);
-                    __half2 h0 = __floats2half2_rn(f0, f2), h1 = __floats2half2_rn(f1, f3);
-                    __half2 h2 = __floats2half2_rn(f4, f6), h3 = __floats2half2_rn(f5, f7);
-                    uint4 o;
-                    o.x = *reinterpret_cast<uint32_t *>(&h0);
-                    o.y = *reinterpret_cast<uint32_t *>(&h1);
-                    o.z = *reinterpret_cast<uint32_t *>(&h2);
-                    o.w = *reinterpret_cast<uint32_t *>(&h3);
+                    const uint4 o = x8_to_fp16_permuted(*p);
                     *p = o;
                 }
                 // make the generic-proxy writes visible to the tensor core (async proxy)
@@ -384,18 +349,7 @@ constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 // normal range.
 __global__ void x_to_fp16_kernel(const uint4 *__restrict__ X, uint4 *__restrict__ Xh, int64_t n8) {
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
-        const uint4 v = __ldg(X + i);
-        const float f0 = __uint_as_float(v.x << 16), f1 = __uint_as_float(v.x & 0xFFFF0000u);
-        const float f2 = __uint_as_float(v.y << 16), f3 = __uint_as_float(v.y & 0xFFFF0000u);
-        const float f4 = __uint_as_float(v.z << 16), f5 = __uint_as_float(v.z & 0xFFFF0000u);
-        const float f6 = __uint_as_float(v.w << 16), f7 = __uint_as_float(v.w & 0xFFFF0000u);
-        __half2 h0 = __floats2half2_rn(f0, f2), h1 = __floats2half2_rn(f1, f3);
-        __half2 h2 = __floats2half2_rn(f4, f6), h3 = __floats2half2_rn(f5, f7);
-        uint4 o;
-        o.x = *reinterpret_cast<uint32_t *>(&h0);
-        o.y = *reinterpret_cast<uint32_t *>(&h1);
-        o.z = *reinterpret_cast<uint32_t *>(&h2);
-        o.w = *reinterpret_cast<uint32_t *>(&h3);
+        const uint4 o = x8_to_fp16_permuted(__ldg(X + i));
         Xh[i] = o;
     }
 }

@@ -68,8 +68,7 @@ enum {
 
 /* Device error bits reported by q4_0_device_error. */
 enum {
-    Q4_DEVERR_WAIT_TIMEOUT = 1u,   /* a bounded on-chip wait gave up; the output is incomplete */
-    Q4_DEVERR_FP16_RANGE = 2u      /* tensor-core path: an operand was beyond the fp16 range */
+    Q4_DEVERR_WAIT_TIMEOUT = 1u    /* a bounded on-chip wait gave up; the output is incomplete */
 };
 
 /* Largest N, K and M accepted (each dimension below 2^31). */
@@ -114,12 +113,15 @@ Q4_0_API int q4_0_dequant(const void *W, float *out, int64_t N, int64_t K,
  *   W, X, Y must be 16-byte aligned; K % 32 == 0; X and Y must not overlap W
  *   or each other.
  *   M == 0 or N == 0: nothing is done.  K == 0: Y is filled with zeros.
- * Path: M <= 32 runs the memory-bound decode kernel (dequantization in
- * registers); M > 32 runs the tcgen05 tensor-core kernel (tiles dequantized
- * to fp16 in shared memory, fp32 accumulators in tensor memory), whose
- * operands must lie in the fp16 range (|x| <= 65504, |d| <= 8188); outside
- * it the result is not within the tolerance and Q4_DEVERR_FP16_RANGE is set
- * in the device error word. */
+ * Path: M <= 32 runs the memory-bound decode kernel (weights dequantized in
+ * registers, products on the warp-level tensor cores); M > 32 runs the
+ * tcgen05 tensor-core kernel (weight tiles dequantized into tensor memory,
+ * fp32 accumulators in tensor memory).  Both feed the tensor cores fp16
+ * operands: each weight (q - 8) * d is rounded once to fp16 (relative error
+ * <= 2^-11) and X is exact in fp16 within its normal range, so operands must
+ * lie in the fp16 range (|x| <= 65504, |d| <= 8188); beyond it products
+ * overflow to +-inf.  q4_0_force_path(4) selects an exact-arithmetic decode
+ * kernel without that restriction. */
 Q4_0_API int q4_0_gemm(const void *W, const uint16_t *X, float *Y,
               int64_t M, int64_t N, int64_t K, q4_0_stream_t stream);
 
@@ -173,10 +175,11 @@ Q4_0_API int q4_0_device_error(uint32_t *flags, int clear);
 
 /* Testing knob, process-wide: force the kernel family used by q4_0_gemm and
  * q4_0_gemm_grouped.  0 = automatic (default), 1 = portable kernel (any
- * shape), 2 = decode kernels (M <= 32 only), 3 = tensor-core kernel, 4 =
- * the warp-level mma.sync decode kernel (M <= 32).  A forced family that
- * cannot run a given shape falls back to automatic.  The pages have no
- * counterpart. */
+ * shape), 2 = decode kernel (M <= 32 only), 3 = tensor-core kernel, 4 = the
+ * exact-arithmetic decode kernel ((q - 8) exact in bf16, d applied in fp32;
+ * M <= 32), 5 = the tcgen05 decode kernel (weights in tensor memory; M <= 32).
+ * A forced family that cannot run a given shape falls back to automatic.  The
+ * pages have no counterpart. */
 Q4_0_API int q4_0_force_path(int path);
 
 #ifdef __cplusplus

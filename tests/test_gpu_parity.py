@@ -233,7 +233,7 @@ def test_prefill_workload_sampled(q4, name):
 
 @pytest.mark.parametrize("M,N,K", [(1, 100, 1024), (2, 129, 3072), (8, 64, 512), (16, 33, 2048)])
 def test_forced_warp_mma_decode(q4, M, N, K):
-    run_gemm(q4, M, N, K, path=q4.PATH_DECODE_MMA)
+    run_gemm(q4, M, N, K, path=q4.PATH_DECODE_EXACT)
 
 
 @pytest.mark.parametrize("name,layers", [("cfg_decode", [0, 13, 25]), ("concurrent", [0, 25])])
@@ -275,3 +275,8 @@ def test_workspace_too_small_falls_back(q4):
     Y_or, B_or = oracle.get().gemm(oracle.get().pack(codes, scales), X, M, N, K)
     check_gemm(Y.cpu().numpy(), Y_or, B_or, "small workspace")
     assert q4.q4_0_gemm_workspace_size(8, 64, 512) == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 100, 1024), (2, 129, 3072), (16, 33, 2048), (32, 70, 512)])
+def test_forced_tmem_decode(q4, M, N, K):
+    run_gemm(q4, M, N, K, path=q4.PATH_DECODE_TMEM)
