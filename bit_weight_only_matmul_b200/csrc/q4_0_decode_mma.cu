@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
     constexpr int RS = ring<NT>();
     extern __shared__ uint8_t smem_raw[];
     using SM = Smem<NT>;
-    SM &S = *reinterpret_cast<SM *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    SM &S = *reinterpret_cast<SM *>(align_smem<128>(smem_raw));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {

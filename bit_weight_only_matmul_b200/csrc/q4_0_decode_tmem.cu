@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
     constexpr uint32_t kIdesc = f16_idesc(128, NN, false);
     extern __shared__ uint8_t smem_raw[];
     using SM = Smem<NN>;
-    SM &S = *reinterpret_cast<SM *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    SM &S = *reinterpret_cast<SM *>(align_smem<1024>(smem_raw));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {

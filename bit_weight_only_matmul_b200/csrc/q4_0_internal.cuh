@@ -73,6 +73,16 @@ __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first ALIGN-aligned byte of a dynamic shared-memory array, reached by
+// offsetting the array itself so that the compiler keeps knowing the pointer
+// is in shared memory (a round trip through an integer would make every
+// access through it a generic one).
+template <int ALIGN>
+__device__ __forceinline__ uint8_t *align_smem(uint8_t *base) {
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(base));
+    return base + ((ALIGN - (a & (ALIGN - 1))) & (ALIGN - 1));
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
 }

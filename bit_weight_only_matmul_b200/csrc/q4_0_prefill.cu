@@ -136,7 +136,7 @@ __device__ __forceinline__ void block_words(const uint32_t (&raw)[36], int i, ui
 template <bool XPRE>
 __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __grid_constant__ PrefillParams P) {
     extern __shared__ uint8_t smem_raw[];
-    Smem &S = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Smem &S = *reinterpret_cast<Smem *>(align_smem<1024>(smem_raw));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tiles = P.tiles_n * P.tiles_m;
     const int ksteps = P.K / kStageK;
