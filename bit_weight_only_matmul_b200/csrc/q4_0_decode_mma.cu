@@ -16,19 +16,21 @@
 // B200, half of what HBM delivers.  The warp-level m16n8k16 has no such floor,
 // and its n=8 matches the few activation rows.
 //
-// Per CTA (one per SM): a producer warp, an X warp and 16 compute warps.
+// Per CTA (one per SM): a producer warp, two X warps and 8 compute warps.
 //  * stage = 256 k of an item (128 weight rows x 144 bytes, one TMA box) plus
 //    the same 256 k of every row of X (1-D bulk copies), in a 4-6-deep ring;
 //    the TMA box pattern alone streams at ~6.9 TB/s (measured);
-//  * the X warp converts the stage's X rows to fp16 straight into mma.sync B
-//    fragments (three buffers), so a compute thread loads each fragment with
-//    one 8-byte shared load;
-//  * compute warp (tile, half) takes 16 weight rows and blocks 4*half ..
-//    4*half+3 of each stage; each thread turns one 4-byte code word of two
-//    rows into fp16 (q - 8) * d pairs -- the A fragments of two MMAs -- and
-//    accumulates across the whole item in fp32 mma.sync accumulators;
-//  * at the end of an item the two halves of a tile add their sums and store
-//    Y[m, n].
+//  * compute warp w owns rows 16w .. 16w+15 of the item; thread (g, t) reads
+//    the 36 contiguous bytes of blocks 2t and 2t+1 of rows g and g+8 (nine
+//    conflict-free 4-byte loads per row), turns them into fp16 (q - 8) * d
+//    pairs and feeds them as A fragments of 16 mma.sync per stage: with the
+//    scale folded into each weight, one MMA may mix blocks, so every byte a
+//    thread loads is its own;
+//  * the X warps convert the stage's X rows to fp16 straight into the
+//    matching mma.sync B fragments (three buffers), one 8-byte shared load per
+//    fragment for the compute threads;
+//  * the accumulators (two chains per n-tile) live across the whole item and
+//    the warp stores Y[m, n] for its 16 rows at the item's end.
 // Numerics: each weight is rounded once to fp16 (relative error <= 2^-11,
 // inside the 1e-3 tolerance of the method); X is exact in fp16 within its
 // normal range; products are exact and accumulation is fp32.  Operands beyond
@@ -50,22 +52,21 @@ using namespace q4dev;
 
 constexpr int kRawW = kItemRows * kStageRowBytes;   // 18432
 constexpr int kXRow = kStageK * 2;                  // 512 bytes of one bf16 X row per stage
+constexpr int kXPitch = kXRow + 16;                 // skews consecutive X rows by four banks
 constexpr int kXBufs = 3;
-constexpr int kWarpProd = 0, kWarpX = 1, kWarp0 = 2, kCompute = 16;
-constexpr int kThreads = 32 * (kWarp0 + kCompute);  // 576
+constexpr int kWarpProd = 0, kWarpX0 = 1, kNumX = 2, kWarp0 = 3, kCompute = 8;
+constexpr int kThreads = 32 * (kWarp0 + kCompute);  // 352
 
 // NT = n8 tiles of X rows (M <= 8*NT)
-template <int NT> constexpr int raw_bytes() { return kRawW + 8 * NT * kXRow; }
+template <int NT> constexpr int raw_bytes() { return kRawW + 8 * NT * kXPitch; }
 template <int NT> constexpr int ring() { return NT == 4 ? 4 : 6; }
 
 template <int NT>
 struct Smem {
-    uint8_t raw[ring<NT>()][raw_bytes<NT>()];   // W rows (pitch 144) then X rows (pitch 512)
-    uint2 xf[kXBufs][8][2][NT][32];             // B fragments: [block][k16 slice][n tile][lane]
-    float comb[2][8][NT][4][32];                // half-1 sums handed to half 0 at an item's end
+    uint8_t raw[ring<NT>()][raw_bytes<NT>()];   // W rows (pitch 144) then X rows (pitch 528)
+    uint2 xf[kXBufs][16][NT][32];               // B fragments: [mma u][n tile][lane]
     uint64_t raw_full[ring<NT>()], raw_empty[ring<NT>()];
     uint64_t xf_full[kXBufs], xf_empty[kXBufs];
-    uint64_t comb_full[2], comb_empty[2];
     int abort_flag;
 };
 
@@ -77,39 +78,44 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1,
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b.x), "r"(b.y));
 }
 
-// Scale (d, d) and qs word t of block i (byte offset 18*i of a 144-byte stage
-// row starting 4-byte aligned at `row`): even blocks start 4-byte aligned,
-// odd ones at 2 mod 4.
-template <int I>
-__device__ __forceinline__ void block_word(const uint8_t *row, int t, uint32_t &d2, uint32_t &qw) {
-    constexpr int off = 18 * I;
-    if constexpr ((I & 1) == 0) {
-        const uint32_t w0 = *reinterpret_cast<const uint32_t *>(row + off + 4 * t);
-        const uint32_t w1 = *reinterpret_cast<const uint32_t *>(row + off + 4 * t + 4);
-        const uint32_t wd = *reinterpret_cast<const uint32_t *>(row + off);
-        d2 = prmt(wd, wd, 0x1010u);
-        qw = prmt(w0, w1, 0x5432u);
+// One row's blocks 2t and 2t+1 of a stage: the 36 bytes at 36t of the
+// 144-byte row, as nine 4-byte words r[0..8].  Block 2t starts 4-byte
+// aligned (scale = low half of r[0], codes straddle words), block 2t+1 at
+// 2 mod 4 (scale = high half of r[4], codes in r[5..8]).
+__device__ __forceinline__ void load_blocks(const uint8_t *row, int t, uint32_t (&r)[9]) {
+    const uint32_t *p = reinterpret_cast<const uint32_t *>(row + 36 * t);
+    #pragma unroll
+    for (int i = 0; i < 9; ++i) r[i] = p[i];
+}
+
+// (d, d) and code word w of block b (0: block 2t, 1: block 2t+1).
+template <int B>
+__device__ __forceinline__ void block_word(const uint32_t (&r)[9], int w, uint32_t &d2, uint32_t &qw) {
+    if constexpr (B == 0) {
+        d2 = prmt(r[0], r[0], 0x1010u);
+        qw = prmt(r[w], r[w + 1], 0x5432u);
     } else {
-        const uint32_t wd = *reinterpret_cast<const uint32_t *>(row + off - 2);
-        d2 = prmt(wd, wd, 0x3232u);
-        qw = *reinterpret_cast<const uint32_t *>(row + off + 2 + 4 * t);
+        d2 = prmt(r[4], r[4], 0x3232u);
+        qw = r[5 + w];
     }
 }
 
-template <int NT, int I>
-__device__ __forceinline__ void block_mma(const uint8_t *rowg, const uint8_t *rowg8, int t,
-                                          const uint2 (&xf)[8][2][NT][32], int lane, float (&acc)[NT][4]) {
+// MMAs u = 8B + 2w (low nibbles) and u + 1 (high nibbles) of the stage.
+template <int NT, int B, int W>
+__device__ __forceinline__ void word_mma(const uint32_t (&rg)[9], const uint32_t (&rg8)[9],
+                                         const uint2 (&xf)[16][NT][32], int lane, float (&acc)[2][NT][4]) {
     uint32_t dg, dg8, qg, qg8;
-    block_word<I>(rowg, t, dg, qg);
-    block_word<I>(rowg8, t, dg8, qg8);
+    block_word<B>(rg, W, dg, qg);
+    block_word<B>(rg8, W, dg8, qg8);
     uint32_t cg[4], cg8[4];
     q4_word_to_fp16(qg, dg, cg);
     q4_word_to_fp16(qg8, dg8, cg8);
-    // slice 0: k cols (2t,2t+1) <- elements (4t,4t+2), (2t+8,2t+9) <- (4t+1,4t+3); slice 1: +16
+    constexpr int u = 8 * B + 2 * W;
     #pragma unroll
     for (int j = 0; j < NT; ++j) {
-        mma_f16(acc[j], cg[0], cg8[0], cg[1], cg8[1], xf[I][0][j][lane]);
-        mma_f16(acc[j], cg[2], cg8[2], cg[3], cg8[3], xf[I][1][j][lane]);
+        // a0/a1: k cols (2t, 2t+1) of rows g / g+8; a2/a3: k cols (2t+8, 2t+9)
+        mma_f16(acc[0][j], cg[0], cg8[0], cg[1], cg8[1], xf[u][j][lane]);
+        mma_f16(acc[1][j], cg[2], cg8[2], cg[3], cg8[3], xf[u + 1][j][lane]);
     }
 }
 
@@ -124,15 +130,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
     if (threadIdx.x == 0) {
         for (int s = 0; s < RS; ++s) {
             mbar_init(&S.raw_full[s], 1);
-            mbar_init(&S.raw_empty[s], kCompute + 1);
+            mbar_init(&S.raw_empty[s], kCompute + kNumX);
         }
         for (int s = 0; s < kXBufs; ++s) {
-            mbar_init(&S.xf_full[s], 1);
+            mbar_init(&S.xf_full[s], kNumX);
             mbar_init(&S.xf_empty[s], kCompute);
-        }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&S.comb_full[s], kCompute / 2);
-            mbar_init(&S.comb_empty[s], kCompute / 2);
         }
         S.abort_flag = 0;
         fence_mbar_init();
@@ -158,14 +160,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
             }
             __syncwarp();
             for (int m = lane; m < pr.M; m += 32)
-                bulk_g2s(S.raw[slot] + kRawW + m * kXRow,
+                bulk_g2s(S.raw[slot] + kRawW + m * kXPitch,
                          pr.X + static_cast<int64_t>(m) * pr.K + static_cast<int64_t>(q.stage) * kStageK, kXRow,
                          &S.raw_full[slot]);
             ++prod_issued;
         }
-    } else if (warp == kWarpX) {
+    } else if (warp < kWarpX0 + kNumX) {
         // ---------------------------------------------------------------- X rows -> fp16 B fragments
-        const int gx = lane >> 2, tx = lane & 3;   // this lane's fragment column (X row) and k group
+        // X warp xw fills MMAs u = 8*xw .. 8*xw+7: lane (gx, tx) -> X row 8j+gx, block 2*tx+xw.
+        // With the 528-byte pitch the 16-byte loads of a warp fall in eight
+        // distinct bank groups and the 8-byte stores in sixteen bank pairs.
+        const int xw = warp - kWarpX0;
+        const int gx = lane >> 2, tx = lane & 3;
         uint32_t g = 0;
         Seq q{};
         q.start(P);
@@ -183,15 +189,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
             for (int j = 0; j < NT; ++j) {
                 const int m = 8 * j + gx;
                 #pragma unroll
-                for (int i = 0; i < 8; ++i)
+                for (int h = 0; h < 2; ++h)
                     #pragma unroll
-                    for (int s = 0; s < 2; ++s) {
-                        uint2 o = make_uint2(0u, 0u);
+                    for (int wp = 0; wp < 2; ++wp) {
+                        uint4 o = make_uint4(0u, 0u, 0u, 0u);
                         if (m < pr.M) {
-                            const uint2 v = *reinterpret_cast<const uint2 *>(xr + m * kXRow + 2 * (32 * i + 16 * s + 4 * tx));
-                            o = x4_to_fp16_permuted(v.x, v.y);
+                            const int k = 32 * (2 * tx + xw) + 16 * h + 8 * wp;
+                            o = x8_to_fp16_permuted(*reinterpret_cast<const uint4 *>(xr + m * kXPitch + 2 * k));
                         }
-                        S.xf[xb][i][s][j][lane] = o;
+                        S.xf[xb][8 * xw + 4 * wp + h][j][lane] = make_uint2(o.x, o.y);
+                        S.xf[xb][8 * xw + 4 * wp + 2 + h][j][lane] = make_uint2(o.z, o.w);
                     }
             }
             __syncwarp();
@@ -202,71 +209,49 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
         }
     } else {
         // ---------------------------------------------------------------- compute
-        const int cw = warp - kWarp0;
-        const int tile = cw >> 1, half = cw & 1;
+        const int tile = warp - kWarp0;   // rows 16*tile .. 16*tile+15 of the item
         const int gq = lane >> 2, t = lane & 3;
-        float acc[NT][4];
+        float acc[2][NT][4];
         #pragma unroll
-        for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-        uint32_t g = 0, items_done = 0;
+        for (int c = 0; c < 2; ++c)
+            #pragma unroll
+            for (int j = 0; j < NT; ++j) acc[c][j][0] = acc[c][j][1] = acc[c][j][2] = acc[c][j][3] = 0.f;
+        uint32_t g = 0;
         Seq q{};
         q.start(P);
         for (; q.item >= 0; q.next(P), ++g) {
             const int slot = g % RS, xb = g % kXBufs;
             if (!wait_or_abort(&S.raw_full[slot], (g / RS) & 1, &S.abort_flag, P.err)) break;
-            if (!wait_or_abort(&S.xf_full[xb], (g / kXBufs) & 1, &S.abort_flag, P.err)) break;
             const uint8_t *rowg = S.raw[slot] + (16 * tile + gq) * kStageRowBytes;
-            const uint8_t *rowg8 = rowg + 8 * kStageRowBytes;
-            if (half == 0) {
-                block_mma<NT, 0>(rowg, rowg8, t, S.xf[xb], lane, acc);
-                block_mma<NT, 1>(rowg, rowg8, t, S.xf[xb], lane, acc);
-                block_mma<NT, 2>(rowg, rowg8, t, S.xf[xb], lane, acc);
-                block_mma<NT, 3>(rowg, rowg8, t, S.xf[xb], lane, acc);
-            } else {
-                block_mma<NT, 4>(rowg, rowg8, t, S.xf[xb], lane, acc);
-                block_mma<NT, 5>(rowg, rowg8, t, S.xf[xb], lane, acc);
-                block_mma<NT, 6>(rowg, rowg8, t, S.xf[xb], lane, acc);
-                block_mma<NT, 7>(rowg, rowg8, t, S.xf[xb], lane, acc);
-            }
+            uint32_t rg[9], rg8[9];
+            load_blocks(rowg, t, rg);
+            load_blocks(rowg + 8 * kStageRowBytes, t, rg8);
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&S.raw_empty[slot]);
-                mbar_arrive(&S.xf_empty[xb]);
-            }
+            if (lane == 0) mbar_arrive(&S.raw_empty[slot]);
+            if (!wait_or_abort(&S.xf_full[xb], (g / kXBufs) & 1, &S.abort_flag, P.err)) break;
+            word_mma<NT, 0, 0>(rg, rg8, S.xf[xb], lane, acc);
+            word_mma<NT, 0, 1>(rg, rg8, S.xf[xb], lane, acc);
+            word_mma<NT, 0, 2>(rg, rg8, S.xf[xb], lane, acc);
+            word_mma<NT, 0, 3>(rg, rg8, S.xf[xb], lane, acc);
+            word_mma<NT, 1, 0>(rg, rg8, S.xf[xb], lane, acc);
+            word_mma<NT, 1, 1>(rg, rg8, S.xf[xb], lane, acc);
+            word_mma<NT, 1, 2>(rg, rg8, S.xf[xb], lane, acc);
+            word_mma<NT, 1, 3>(rg, rg8, S.xf[xb], lane, acc);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.xf_empty[xb]);
             if (q.stage == q.nstages - 1) {
-                // end of the item: the two halves of the tile add their sums
+                // end of the item: thread holds rows gq / gq+8 x columns 8j+2t, 8j+2t+1
                 const GroupProblem &pr = P.p[q.prob];
-                const int cb = items_done & 1;
-                const uint32_t par = (items_done >> 1) & 1;
-                if (half == 1) {
-                    if (!wait_or_abort(&S.comb_empty[cb], par ^ 1, &S.abort_flag, P.err)) break;
-                    #pragma unroll
-                    for (int j = 0; j < NT; ++j)
-                        #pragma unroll
-                        for (int e = 0; e < 4; ++e) S.comb[cb][tile][j][e][lane] = acc[j][e];
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&S.comb_full[cb]);
-                } else {
-                    if (!wait_or_abort(&S.comb_full[cb], par, &S.abort_flag, P.err)) break;
-                    #pragma unroll
-                    for (int j = 0; j < NT; ++j)
-                        #pragma unroll
-                        for (int e = 0; e < 4; ++e) acc[j][e] += S.comb[cb][tile][j][e][lane];
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&S.comb_empty[cb]);
-                    // thread holds rows gq / gq+8 of the tile x columns 8j+2t, 8j+2t+1
-                    #pragma unroll
-                    for (int j = 0; j < NT; ++j)
-                        #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int m = 8 * j + 2 * t + (e & 1);
-                            const int n = q.row0 + 16 * tile + gq + ((e & 2) ? 8 : 0);
-                            if (m < pr.M && n < pr.N) pr.Y[static_cast<int64_t>(m) * pr.N + n] = acc[j][e];
-                        }
-                }
                 #pragma unroll
-                for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-                ++items_done;
+                for (int j = 0; j < NT; ++j)
+                    #pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int m = 8 * j + 2 * t + (e & 1);
+                        const int n = q.row0 + 16 * tile + gq + ((e & 2) ? 8 : 0);
+                        if (m < pr.M && n < pr.N)
+                            pr.Y[static_cast<int64_t>(m) * pr.N + n] = acc[0][j][e] + acc[1][j][e];
+                        acc[0][j][e] = acc[1][j][e] = 0.f;
+                    }
             }
         }
     }
