@@ -16,21 +16,24 @@
 // B200, half of what HBM delivers.  The warp-level m16n8k16 has no such floor,
 // and its n=8 matches the few activation rows.
 //
-// Per CTA (one per SM): a producer warp, two X warps and 8 compute warps.
+// Per CTA (one per SM): a producer warp, two X warps and two groups of 8
+// compute warps; X warp G and compute group G take the stages g with
+// g mod 2 == G, so that two stages are worked on at once.
 //  * stage = 256 k of an item (128 weight rows x 144 bytes, one TMA box) plus
 //    the same 256 k of every row of X (1-D bulk copies), in a 4-6-deep ring;
 //    the TMA box pattern alone streams at ~6.9 TB/s (measured);
-//  * compute warp w owns rows 16w .. 16w+15 of the item; thread (g, t) reads
+//  * compute warp w of a group owns rows 16w .. 16w+15; thread (g, t) reads
 //    the 36 contiguous bytes of blocks 2t and 2t+1 of rows g and g+8 (nine
 //    conflict-free 4-byte loads per row), turns them into fp16 (q - 8) * d
 //    pairs and feeds them as A fragments of 16 mma.sync per stage: with the
 //    scale folded into each weight, one MMA may mix blocks, so every byte a
 //    thread loads is its own;
 //  * the X warps convert the stage's X rows to fp16 straight into the
-//    matching mma.sync B fragments (three buffers), one 8-byte shared load per
-//    fragment for the compute threads;
-//  * the accumulators (two chains per n-tile) live across the whole item and
-//    the warp stores Y[m, n] for its 16 rows at the item's end.
+//    matching mma.sync B fragments (two buffers per group), one 8-byte shared
+//    load per fragment for the compute threads;
+//  * the accumulators (two chains per n-tile) live across the whole item; at
+//    its end the group-1 warp hands its sums through shared memory to the
+//    group-0 warp of the same rows, which stores Y[m, n].
 // Numerics: each weight is rounded once to fp16 (relative error <= 2^-11,
 // inside the 1e-3 tolerance of the method); X is exact in fp16 within its
 // normal range; products are exact and accumulation is fp32.  Operands beyond
@@ -53,9 +56,9 @@ using namespace q4dev;
 constexpr int kRawW = kItemRows * kStageRowBytes;   // 18432
 constexpr int kXRow = kStageK * 2;                  // 512 bytes of one bf16 X row per stage
 constexpr int kXPitch = kXRow + 16;                 // skews consecutive X rows by four banks
-constexpr int kXBufs = 3;
-constexpr int kWarpProd = 0, kWarpX0 = 1, kNumX = 2, kWarp0 = 3, kCompute = 8;
-constexpr int kThreads = 32 * (kWarp0 + kCompute);  // 352
+constexpr int kXBufs = 4;                           // buffer g mod 4 belongs to group g mod 2
+constexpr int kWarpProd = 0, kWarpX0 = 1, kWarp0 = 3, kGroupWarps = 8;
+constexpr int kThreads = 32 * (kWarp0 + 2 * kGroupWarps);  // 608
 
 // NT = n8 tiles of X rows (M <= 8*NT)
 template <int NT> constexpr int raw_bytes() { return kRawW + 8 * NT * kXPitch; }
@@ -65,8 +68,10 @@ template <int NT>
 struct Smem {
     uint8_t raw[ring<NT>()][raw_bytes<NT>()];   // W rows (pitch 144) then X rows (pitch 528)
     uint2 xf[kXBufs][16][NT][32];               // B fragments: [mma u][n tile][lane]
+    float comb[8][NT][4][32];                   // group-1 sums handed to group 0 at an item's end
     uint64_t raw_full[ring<NT>()], raw_empty[ring<NT>()];
     uint64_t xf_full[kXBufs], xf_empty[kXBufs];
+    uint64_t comb_full, comb_empty;
     int abort_flag;
 };
 
@@ -130,12 +135,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
     if (threadIdx.x == 0) {
         for (int s = 0; s < RS; ++s) {
             mbar_init(&S.raw_full[s], 1);
-            mbar_init(&S.raw_empty[s], kCompute + kNumX);
+            mbar_init(&S.raw_empty[s], kGroupWarps + 1);
         }
         for (int s = 0; s < kXBufs; ++s) {
-            mbar_init(&S.xf_full[s], kNumX);
-            mbar_init(&S.xf_empty[s], kCompute);
+            mbar_init(&S.xf_full[s], 1);
+            mbar_init(&S.xf_empty[s], kGroupWarps);
         }
+        mbar_init(&S.comb_full, kGroupWarps);
+        mbar_init(&S.comb_empty, kGroupWarps);
         S.abort_flag = 0;
         fence_mbar_init();
     }
@@ -165,17 +172,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
                          &S.raw_full[slot]);
             ++prod_issued;
         }
-    } else if (warp < kWarpX0 + kNumX) {
+    } else if (warp < kWarp0) {
         // ---------------------------------------------------------------- X rows -> fp16 B fragments
-        // X warp xw fills MMAs u = 8*xw .. 8*xw+7: lane (gx, tx) -> X row 8j+gx, block 2*tx+xw.
-        // With the 528-byte pitch the 16-byte loads of a warp fall in eight
-        // distinct bank groups and the 8-byte stores in sixteen bank pairs.
-        const int xw = warp - kWarpX0;
+        // X warp G fills all 16 MMAs of the stages of its parity: lane (gx, tx)
+        // -> X row 8j+gx, blocks 2tx and 2tx+1.  With the 528-byte pitch the
+        // 16-byte loads of a warp fall in eight distinct bank groups and the
+        // 8-byte stores in sixteen bank pairs.
+        const int G = warp - kWarpX0;
         const int gx = lane >> 2, tx = lane & 3;
         uint32_t g = 0;
         Seq q{};
         q.start(P);
         for (; q.item >= 0; q.next(P), ++g) {
+            if ((g & 1) != static_cast<uint32_t>(G)) continue;
             const GroupProblem &pr = P.p[q.prob];
             const int slot = g % RS, xb = g % kXBufs;
             bool ok = true;
@@ -189,17 +198,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
             for (int j = 0; j < NT; ++j) {
                 const int m = 8 * j + gx;
                 #pragma unroll
-                for (int h = 0; h < 2; ++h)
+                for (int xw = 0; xw < 2; ++xw)
                     #pragma unroll
-                    for (int wp = 0; wp < 2; ++wp) {
-                        uint4 o = make_uint4(0u, 0u, 0u, 0u);
-                        if (m < pr.M) {
-                            const int k = 32 * (2 * tx + xw) + 16 * h + 8 * wp;
-                            o = x8_to_fp16_permuted(*reinterpret_cast<const uint4 *>(xr + m * kXPitch + 2 * k));
+                    for (int h = 0; h < 2; ++h)
+                        #pragma unroll
+                        for (int wp = 0; wp < 2; ++wp) {
+                            uint4 o = make_uint4(0u, 0u, 0u, 0u);
+                            if (m < pr.M) {
+                                const int k = 32 * (2 * tx + xw) + 16 * h + 8 * wp;
+                                o = x8_to_fp16_permuted(*reinterpret_cast<const uint4 *>(xr + m * kXPitch + 2 * k));
+                            }
+                            S.xf[xb][8 * xw + 4 * wp + h][j][lane] = make_uint2(o.x, o.y);
+                            S.xf[xb][8 * xw + 4 * wp + 2 + h][j][lane] = make_uint2(o.z, o.w);
                         }
-                        S.xf[xb][8 * xw + 4 * wp + h][j][lane] = make_uint2(o.x, o.y);
-                        S.xf[xb][8 * xw + 4 * wp + 2 + h][j][lane] = make_uint2(o.z, o.w);
-                    }
             }
             __syncwarp();
             if (lane == 0) {
@@ -209,49 +220,76 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
         }
     } else {
         // ---------------------------------------------------------------- compute
-        const int tile = warp - kWarp0;   // rows 16*tile .. 16*tile+15 of the item
+        const int cw = warp - kWarp0;
+        const int G = cw >> 3, tile = cw & 7;   // stage parity, rows 16*tile .. 16*tile+15
         const int gq = lane >> 2, t = lane & 3;
         float acc[2][NT][4];
         #pragma unroll
         for (int c = 0; c < 2; ++c)
             #pragma unroll
             for (int j = 0; j < NT; ++j) acc[c][j][0] = acc[c][j][1] = acc[c][j][2] = acc[c][j][3] = 0.f;
-        uint32_t g = 0;
+        uint32_t g = 0, items_done = 0;
         Seq q{};
         q.start(P);
         for (; q.item >= 0; q.next(P), ++g) {
-            const int slot = g % RS, xb = g % kXBufs;
-            if (!wait_or_abort(&S.raw_full[slot], (g / RS) & 1, &S.abort_flag, P.err)) break;
-            const uint8_t *rowg = S.raw[slot] + (16 * tile + gq) * kStageRowBytes;
-            uint32_t rg[9], rg8[9];
-            load_blocks(rowg, t, rg);
-            load_blocks(rowg + 8 * kStageRowBytes, t, rg8);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.raw_empty[slot]);
-            if (!wait_or_abort(&S.xf_full[xb], (g / kXBufs) & 1, &S.abort_flag, P.err)) break;
-            word_mma<NT, 0, 0>(rg, rg8, S.xf[xb], lane, acc);
-            word_mma<NT, 0, 1>(rg, rg8, S.xf[xb], lane, acc);
-            word_mma<NT, 0, 2>(rg, rg8, S.xf[xb], lane, acc);
-            word_mma<NT, 0, 3>(rg, rg8, S.xf[xb], lane, acc);
-            word_mma<NT, 1, 0>(rg, rg8, S.xf[xb], lane, acc);
-            word_mma<NT, 1, 1>(rg, rg8, S.xf[xb], lane, acc);
-            word_mma<NT, 1, 2>(rg, rg8, S.xf[xb], lane, acc);
-            word_mma<NT, 1, 3>(rg, rg8, S.xf[xb], lane, acc);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.xf_empty[xb]);
+            if ((g & 1) == static_cast<uint32_t>(G)) {
+                const int slot = g % RS, xb = g % kXBufs;
+                if (!wait_or_abort(&S.raw_full[slot], (g / RS) & 1, &S.abort_flag, P.err)) break;
+                const uint8_t *rowg = S.raw[slot] + (16 * tile + gq) * kStageRowBytes;
+                uint32_t rg[9], rg8[9];
+                load_blocks(rowg, t, rg);
+                load_blocks(rowg + 8 * kStageRowBytes, t, rg8);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.raw_empty[slot]);
+                if (!wait_or_abort(&S.xf_full[xb], (g / kXBufs) & 1, &S.abort_flag, P.err)) break;
+                word_mma<NT, 0, 0>(rg, rg8, S.xf[xb], lane, acc);
+                word_mma<NT, 0, 1>(rg, rg8, S.xf[xb], lane, acc);
+                word_mma<NT, 0, 2>(rg, rg8, S.xf[xb], lane, acc);
+                word_mma<NT, 0, 3>(rg, rg8, S.xf[xb], lane, acc);
+                word_mma<NT, 1, 0>(rg, rg8, S.xf[xb], lane, acc);
+                word_mma<NT, 1, 1>(rg, rg8, S.xf[xb], lane, acc);
+                word_mma<NT, 1, 2>(rg, rg8, S.xf[xb], lane, acc);
+                word_mma<NT, 1, 3>(rg, rg8, S.xf[xb], lane, acc);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.xf_empty[xb]);
+            }
             if (q.stage == q.nstages - 1) {
-                // end of the item: thread holds rows gq / gq+8 x columns 8j+2t, 8j+2t+1
+                // end of the item: the two groups add their sums
                 const GroupProblem &pr = P.p[q.prob];
-                #pragma unroll
-                for (int j = 0; j < NT; ++j)
+                const uint32_t par = items_done & 1;
+                if (G == 1) {
+                    if (!wait_or_abort(&S.comb_empty, par ^ 1, &S.abort_flag, P.err)) break;
                     #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int m = 8 * j + 2 * t + (e & 1);
-                        const int n = q.row0 + 16 * tile + gq + ((e & 2) ? 8 : 0);
-                        if (m < pr.M && n < pr.N)
-                            pr.Y[static_cast<int64_t>(m) * pr.N + n] = acc[0][j][e] + acc[1][j][e];
-                        acc[0][j][e] = acc[1][j][e] = 0.f;
-                    }
+                    for (int j = 0; j < NT; ++j)
+                        #pragma unroll
+                        for (int e = 0; e < 4; ++e) S.comb[tile][j][e][lane] = acc[0][j][e] + acc[1][j][e];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.comb_full);
+                } else {
+                    if (!wait_or_abort(&S.comb_full, par, &S.abort_flag, P.err)) break;
+                    float sum[NT][4];
+                    #pragma unroll
+                    for (int j = 0; j < NT; ++j)
+                        #pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            sum[j][e] = acc[0][j][e] + acc[1][j][e] + S.comb[tile][j][e][lane];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.comb_empty);
+                    // thread holds rows gq / gq+8 of the tile x columns 8j+2t, 8j+2t+1
+                    #pragma unroll
+                    for (int j = 0; j < NT; ++j)
+                        #pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int m = 8 * j + 2 * t + (e & 1);
+                            const int n = q.row0 + 16 * tile + gq + ((e & 2) ? 8 : 0);
+                            if (m < pr.M && n < pr.N) pr.Y[static_cast<int64_t>(m) * pr.N + n] = sum[j][e];
+                        }
+                }
+                #pragma unroll
+                for (int c = 0; c < 2; ++c)
+                    #pragma unroll
+                    for (int j = 0; j < NT; ++j) acc[c][j][0] = acc[c][j][1] = acc[c][j][2] = acc[c][j][3] = 0.f;
+                ++items_done;
             }
         }
     }
