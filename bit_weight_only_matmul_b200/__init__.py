@@ -22,10 +22,12 @@ Q4_ERR_INVALID_ARG = 1
 Q4_ERR_MISALIGNED = 2
 Q4_ERR_UNSUPPORTED_DEVICE = 3
 Q4_ERR_CUDA = 4
+Q4_ERR_TOO_LARGE = 5
 
 Q4_DEVERR_WAIT_TIMEOUT = 1
 
 Q4_0_MAX_GROUP = 256
+Q4_0_STATIC_WS_BYTES = 64 << 20
 
 PATH_AUTO, PATH_GENERIC, PATH_DECODE, PATH_TENSOR, PATH_DECODE_EXACT, PATH_DECODE_TMEM = 0, 1, 2, 3, 4, 5
 
@@ -39,6 +41,7 @@ EXPORTS = (
     "q4_0_gemm",
     "q4_0_gemm_workspace_size",
     "q4_0_gemm_ws",
+    "q4_0_gemm_static_ws",
     "q4_0_gemm_grouped",
     "q4_0_device_error",
     "q4_0_force_path",
@@ -73,6 +76,7 @@ def _load() -> ctypes.CDLL:
         "q4_0_gemm": (i32, [vp, vp, vp, i64, i64, i64, vp]),
         "q4_0_gemm_workspace_size": (i64, [i64, i64, i64]),
         "q4_0_gemm_ws": (i32, [vp, vp, vp, i64, i64, i64, vp, i64, vp]),
+        "q4_0_gemm_static_ws": (i32, [vp, vp, vp, i64, i64, i64, vp]),
         "q4_0_gemm_grouped": (i32, [ctypes.POINTER(q4_0_problem), i32, vp]),
         "q4_0_device_error": (i32, [ctypes.POINTER(ctypes.c_uint32), i32]),
         "q4_0_force_path": (i32, [i32]),
@@ -144,6 +148,13 @@ def q4_0_gemm_ws(W, X, Y, M: int, N: int, K: int, workspace, workspace_bytes: Op
         workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_lib.q4_0_gemm_ws(_ptr(W), _ptr(X), _ptr(Y), M, N, K, _ptr(workspace), workspace_bytes,
                              _stream(stream)), "q4_0_gemm_ws")
+
+
+def q4_0_gemm_static_ws(W, X, Y, M: int, N: int, K: int, stream=None) -> None:
+    """q4_0_gemm_ws on the library's fixed device scratch array: the call
+    allocates nothing (Q4Error Q4_ERR_TOO_LARGE when M*K*2 exceeds
+    Q4_0_STATIC_WS_BYTES for M > 32)."""
+    _check(_lib.q4_0_gemm_static_ws(_ptr(W), _ptr(X), _ptr(Y), M, N, K, _stream(stream)), "q4_0_gemm_static_ws")
 
 
 def make_problems(problems: Sequence) -> ctypes.Array:

@@ -146,6 +146,9 @@ const char *q4_0_status_string(int status) {
         case Q4_ERR_MISALIGNED: return "Q4_ERR_MISALIGNED: a pointer is not 16-byte aligned";
         case Q4_ERR_UNSUPPORTED_DEVICE: return "Q4_ERR_UNSUPPORTED_DEVICE: current device is not sm_100 (CC 10.0)";
         case Q4_ERR_CUDA: return "Q4_ERR_CUDA: a CUDA runtime call failed";
+        case Q4_ERR_TOO_LARGE:
+            return "Q4_ERR_TOO_LARGE: the problem needs more scratch than the library's fixed buffer "
+                   "(Q4_0_STATIC_WS_BYTES) holds";
         default: return "unknown q4_0 status";
     }
 }
@@ -204,6 +207,20 @@ int q4_0_gemm_ws(const void *W, const uint16_t *X, float *Y, int64_t M, int64_t 
     if (workspace && !aligned16(workspace)) return Q4_ERR_MISALIGNED;
     q4_0_problem p{W, X, Y, M, N, K};
     return run_problems(&p, 1, reinterpret_cast<cudaStream_t>(stream), workspace, workspace_bytes);
+}
+
+int q4_0_gemm_static_ws(const void *W, const uint16_t *X, float *Y, int64_t M, int64_t N, int64_t K,
+                        q4_0_stream_t stream) {
+    const int64_t need = q4_0_gemm_workspace_size(M, N, K);
+    if (need < 0 || M > Q4_0_MAX_DIM || N > Q4_0_MAX_DIM || K > Q4_0_MAX_DIM) return Q4_ERR_INVALID_ARG;
+    if (need > Q4_0_STATIC_WS_BYTES) return Q4_ERR_TOO_LARGE;
+    const q4::DeviceInfo *dev = nullptr;
+    int st = current_device(&dev);
+    if (st != Q4_OK) return st;
+    void *ws = nullptr;
+    const cudaError_t e = q4::static_workspace(dev->device, &ws);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return q4_0_gemm_ws(W, X, Y, M, N, K, ws, Q4_0_STATIC_WS_BYTES, stream);
 }
 
 int q4_0_gemm_grouped(const q4_0_problem *problems, int count, q4_0_stream_t stream) {

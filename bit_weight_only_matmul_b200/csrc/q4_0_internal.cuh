@@ -49,6 +49,10 @@ cudaError_t launch_decode_tmem(const Problem *probs, int count, const DeviceInfo
 // by a pre-pass; without one the kernel converts each X tile it loads.
 bool prefill_supports(const Problem &p);
 int64_t prefill_workspace_bytes(const Problem &p);
+// Device address of this device's copy of the library's fixed scratch array
+// (Q4_0_STATIC_WS_BYTES, 256-byte aligned); looked up once per device, with
+// `dev` current.
+cudaError_t static_workspace(int dev, void **out);
 cudaError_t launch_prefill(const Problem &p, const DeviceInfo &dev, cudaStream_t s, void *workspace,
                            int64_t workspace_bytes);
 

@@ -63,7 +63,8 @@ enum {
     Q4_ERR_INVALID_ARG = 1,        /* null pointer, negative size, K % 32 != 0, too large */
     Q4_ERR_MISALIGNED = 2,         /* a pointer is not 16-byte aligned */
     Q4_ERR_UNSUPPORTED_DEVICE = 3, /* current device is not compute capability 10.0 */
-    Q4_ERR_CUDA = 4                /* a CUDA runtime call failed; see q4_0_last_cuda_error */
+    Q4_ERR_CUDA = 4,               /* a CUDA runtime call failed; see q4_0_last_cuda_error */
+    Q4_ERR_TOO_LARGE = 5           /* the problem needs more scratch than Q4_0_STATIC_WS_BYTES */
 };
 
 /* Device error bits reported by q4_0_device_error. */
@@ -142,6 +143,36 @@ Q4_0_API int64_t q4_0_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 Q4_0_API int q4_0_gemm_ws(const void *W, const uint16_t *X, float *Y,
                           int64_t M, int64_t N, int64_t K, void *workspace,
                           int64_t workspace_bytes, q4_0_stream_t stream);
+
+/* Size of the library's fixed device scratch array used by
+ * q4_0_gemm_static_ws: 64 MiB on each device (an fp16 copy of X up to
+ * M*K = 32 Mi elements, e.g. M = 4096 rows at K = 8192). */
+#define Q4_0_STATIC_WS_BYTES (64LL << 20)
+
+/* q4_0_gemm_ws with the library's own fixed scratch array as the workspace:
+ * it allocates nothing, neither device nor host memory, on any call.  For
+ * callers that may not allocate when they multiply: a real-time audio thread
+ * that must not block in an allocator, a process that budgets device memory
+ * once at start-up, code that runs where no allocator is reachable.
+ *   * The array (Q4_0_STATIC_WS_BYTES, 256-byte aligned) is a __device__
+ *     variable of the library, one copy per device.  A problem whose
+ *     workspace size (q4_0_gemm_workspace_size) exceeds it is rejected with
+ *     Q4_ERR_TOO_LARGE and nothing is launched; M <= 32 needs none.
+ *   * Nothing in the array has to start at zero: each call writes every byte
+ *     it reads before reading it, on `stream`.
+ *   * Calls whose kernels can overlap on one device (different streams or
+ *     host threads without ordering between them) share the array and race;
+ *     calls on one stream, or otherwise ordered, are safe.
+ *   * The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current, which may load the
+ *     library module holding it); make that first call before any stream
+ *     capture begins.  Every call needs a current sm_100 device, even one
+ *     with nothing to compute.
+ * Results are those of q4_0_gemm_ws with a large enough workspace (the same
+ * as q4_0_gemm, bit for bit).  The pages have no counterpart: this is a
+ * deployment convenience of this library. */
+Q4_0_API int q4_0_gemm_static_ws(const void *W, const uint16_t *X, float *Y,
+                                 int64_t M, int64_t N, int64_t K, q4_0_stream_t stream);
 
 /* One problem of a grouped launch: Y = X * dequant(W)^T, all device
  * pointers, same rules as q4_0_gemm. */
