@@ -96,7 +96,13 @@ int run_problems(const q4_0_problem *probs, int count, cudaStream_t s, void *ws 
     st = current_device(&dev);
     if (st != Q4_OK) return st;
     const int force = g_force_path.load(std::memory_order_relaxed);
-    std::vector<q4::Problem> dec, dexact, dtmem, gen, ten;
+    // per-thread lists, reused from call to call (no allocation once grown)
+    static thread_local std::vector<q4::Problem> dec, dexact, dtmem, gen, ten;
+    dec.clear();
+    dexact.clear();
+    dtmem.clear();
+    gen.clear();
+    ten.clear();
     for (int i = 0; i < count; ++i) {
         const q4_0_problem &a = probs[i];
         if (a.M == 0 || a.N == 0) continue;

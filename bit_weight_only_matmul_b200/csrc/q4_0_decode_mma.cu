@@ -34,6 +34,16 @@
 //  * the accumulators (two chains per n-tile) live across the whole item; at
 //    its end the group-1 warp hands its sums through shared memory to the
 //    group-0 warp of the same rows, which stores Y[m, n].
+// Split mode (M <= 8, between one item per SM and kMaxItems items): when a
+// launch has few items, whole items leave a tail -- one decoder layer at M=1
+// has 24 items of 32 stages next to 192 of 12, so the busiest CTA works 32
+// stages against a mean of 21.  The CTAs then run in clusters of two.  An
+// item longer than the mean load of a CTA is split: the two CTAs of a
+// cluster take its two halves, both first thing, and the second CTA's sums
+// reach the first through distributed shared memory before the first stores
+// Y.  The other items stay whole, each on one CTA.  The host deals the split
+// items to the clusters and then the whole items to the CTAs, longest first
+// onto the least loaded.
 // Numerics: each weight is rounded once to fp16 (relative error <= 2^-11,
 // inside the 1e-3 tolerance of the method); X is exact in fp16 within its
 // normal range; products are exact and accumulation is fp32.  Operands beyond
@@ -41,6 +51,8 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <queue>
+#include <utility>
 #include <vector>
 
 #include "q4_0_convert.cuh"
@@ -59,12 +71,26 @@ constexpr int kXPitch = kXRow + 16;                 // skews consecutive X rows 
 constexpr int kXBufs = 4;                           // buffer g mod 4 belongs to group g mod 2
 constexpr int kWarpProd = 0, kWarpX0 = 1, kWarp0 = 3, kGroupWarps = 8;
 constexpr int kThreads = 32 * (kWarp0 + 2 * kGroupWarps);  // 608
+constexpr int kMaxItems = 1024;                     // items per launch in split mode
+constexpr int kMaxSplitCtas = 256;
+constexpr int kMaxSched = 2 * kMaxItems;            // schedule entries (a split item has two)
+constexpr uint16_t kSplitFlag = 0x8000;
 
 // NT = n8 tiles of X rows (M <= 8*NT)
 template <int NT> constexpr int raw_bytes() { return kRawW + 8 * NT * kXPitch; }
 template <int NT> constexpr int ring() { return NT == 4 ? 4 : 6; }
 
+// Partner sums in split mode: written remotely by CTA 1 of a cluster into
+// CTA 0's copy (two buffers, by item parity).
+template <int NT, bool SPLIT>
+struct XComb {
+    float v[2][8][NT][4][32];
+    uint64_t full[2], empty[2];
+};
 template <int NT>
+struct XComb<NT, false> {};
+
+template <int NT, bool SPLIT>
 struct Smem {
     uint8_t raw[ring<NT>()][raw_bytes<NT>()];   // W rows (pitch 144) then X rows (pitch 528)
     uint2 xf[kXBufs][16][NT][32];               // B fragments: [mma u][n tile][lane]
@@ -72,6 +98,7 @@ struct Smem {
     uint64_t raw_full[ring<NT>()], raw_empty[ring<NT>()];
     uint64_t xf_full[kXBufs], xf_empty[kXBufs];
     uint64_t comb_full, comb_empty;
+    XComb<NT, SPLIT> x;
     int abort_flag;
 };
 
@@ -124,11 +151,121 @@ __device__ __forceinline__ void word_mma(const uint32_t (&rg)[9], const uint32_t
     }
 }
 
-template <int NT, int CAP>
-__global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_constant__ GroupParams<CAP> P) {
+template <int CAP>
+struct DecodeParams {
+    GroupParams<CAP> g;
+    // split mode: CTA b runs sched[sched_begin[b] .. sched_begin[b+1]), each
+    // entry an item index, with kSplitFlag set for a half of a split item
+    uint16_t sched_begin[kMaxSplitCtas + 1];
+    uint16_t sched[kMaxSched];
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t remote_addr(const void *local, uint32_t rank) {
+    uint32_t ra;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_addr(local)), "r"(rank));
+    return ra;
+}
+
+__device__ __forceinline__ void st_remote(float *local, uint32_t rank, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote_addr(local, rank)), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint64_t *local, uint32_t rank) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_addr(local, rank))
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(kSuspendHintNs)
+        : "memory");
+    return ok != 0;
+}
+
+// wait_or_abort for a barrier that the partner CTA arrives on.
+__device__ __forceinline__ bool wait_cluster_or_abort(uint64_t *bar, uint32_t parity, int *abort_flag,
+                                                      unsigned *err) {
+    const unsigned long long t0 = global_ns();
+    while (!mbar_try_wait_cluster(bar, parity)) {
+        if (*reinterpret_cast<volatile int *>(abort_flag)) return false;
+        if (global_ns() - t0 > kWaitLimitNs) {
+            atomicOr(err, (unsigned)Q4_DEVERR_WAIT_TIMEOUT);
+            *reinterpret_cast<volatile int *>(abort_flag) = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+// One CTA's walk over its (item, stage) sequence.  Plain mode: the items dealt
+// to the CTAs in boustrophedon order.  Split mode: the CTA's list from the
+// host; of a split n-stage item rank 0 takes the first ceil(n/2) stages and
+// rank 1 the rest.
+template <bool SPLIT>
+struct Walk {
+    int round, idx, item, prob, row0, stage, end;
+    bool split;
+    template <int CAP>
+    __device__ __forceinline__ void load(const DecodeParams<CAP> &D, uint32_t rank) {
+        const GroupParams<CAP> &P = D.g;
+        if constexpr (!SPLIT) {
+            const int G = gridDim.x;
+            const int pos = (round & 1) ? (G - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
+            item = round * G + pos;
+            if (item >= P.total_items) { item = -1; return; }
+            prob = find_problem(P, item);
+            stage = 0;
+            end = P.p[prob].stages;
+            split = false;
+        } else {
+            if (idx >= D.sched_begin[blockIdx.x + 1]) { item = -1; return; }
+            const uint16_t e = D.sched[idx];
+            item = e & (kSplitFlag - 1);
+            split = (e & kSplitFlag) != 0;
+            prob = find_problem(P, item);
+            const int n = P.p[prob].stages;
+            const int n0 = (n + 1) / 2;
+            stage = split && rank == 1 ? n0 : 0;
+            end = split && rank == 0 ? n0 : n;
+        }
+        row0 = (item - P.p[prob].item_begin) * kItemRows;
+    }
+    template <int CAP>
+    __device__ __forceinline__ void start(const DecodeParams<CAP> &D, uint32_t rank) {
+        round = 0;
+        idx = 0;
+        if constexpr (SPLIT) idx = D.sched_begin[blockIdx.x];
+        load(D, rank);
+    }
+    template <int CAP>
+    __device__ __forceinline__ void next(const DecodeParams<CAP> &D, uint32_t rank) {
+        if (++stage < end) return;
+        ++round;
+        ++idx;
+        load(D, rank);
+    }
+};
+
+template <int NT, int CAP, bool SPLIT>
+__global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_constant__ DecodeParams<CAP> D) {
     constexpr int RS = ring<NT>();
+    const GroupParams<CAP> &P = D.g;
     extern __shared__ uint8_t smem_raw[];
-    using SM = Smem<NT>;
+    using SM = Smem<NT, SPLIT>;
     SM &S = *reinterpret_cast<SM *>(align_smem<128>(smem_raw));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -143,17 +280,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
         }
         mbar_init(&S.comb_full, kGroupWarps);
         mbar_init(&S.comb_empty, kGroupWarps);
+        if constexpr (SPLIT) {
+            for (int s = 0; s < 2; ++s) {
+                mbar_init(&S.x.full[s], 32 * kGroupWarps);    // every thread of the partner's group 0
+                mbar_init(&S.x.empty[s], 32 * kGroupWarps);
+            }
+        }
         S.abort_flag = 0;
         fence_mbar_init();
     }
-    __syncthreads();
+    uint32_t rank = 0;
+    if constexpr (SPLIT) {
+        rank = cluster_rank();
+        cluster_sync_all();   // the partner's barriers exist before anyone arrives on them
+    } else {
+        __syncthreads();
+    }
     uint32_t prod_issued = 0;
 
     if (warp == kWarpProd) {
         // ---------------------------------------------------------------- loads
-        Seq q{};
-        q.start(P);
-        for (; q.item >= 0; q.next(P)) {
+        Walk<SPLIT> q{};
+        q.start(D, rank);
+        for (; q.item >= 0; q.next(D, rank)) {
             const GroupProblem &pr = P.p[q.prob];
             const uint32_t g = prod_issued;
             const int slot = g % RS;
@@ -181,9 +330,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
         const int G = warp - kWarpX0;
         const int gx = lane >> 2, tx = lane & 3;
         uint32_t g = 0;
-        Seq q{};
-        q.start(P);
-        for (; q.item >= 0; q.next(P), ++g) {
+        Walk<SPLIT> q{};
+        q.start(D, rank);
+        for (; q.item >= 0; q.next(D, rank), ++g) {
             if ((g & 1) != static_cast<uint32_t>(G)) continue;
             const GroupProblem &pr = P.p[q.prob];
             const int slot = g % RS, xb = g % kXBufs;
@@ -228,10 +377,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
         for (int c = 0; c < 2; ++c)
             #pragma unroll
             for (int j = 0; j < NT; ++j) acc[c][j][0] = acc[c][j][1] = acc[c][j][2] = acc[c][j][3] = 0.f;
-        uint32_t g = 0, items_done = 0;
-        Seq q{};
-        q.start(P);
-        for (; q.item >= 0; q.next(P), ++g) {
+        uint32_t g = 0, items_done = 0, split_done = 0;
+        Walk<SPLIT> q{};
+        q.start(D, rank);
+        for (; q.item >= 0; q.next(D, rank), ++g) {
             if ((g & 1) == static_cast<uint32_t>(G)) {
                 const int slot = g % RS, xb = g % kXBufs;
                 if (!wait_or_abort(&S.raw_full[slot], (g / RS) & 1, &S.abort_flag, P.err)) break;
@@ -253,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.xf_empty[xb]);
             }
-            if (q.stage == q.nstages - 1) {
+            if (q.stage == q.end - 1) {
                 // end of the item: the two groups add their sums
                 const GroupProblem &pr = P.p[q.prob];
                 const uint32_t par = items_done & 1;
@@ -275,15 +424,40 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
                             sum[j][e] = acc[0][j][e] + acc[1][j][e] + S.comb[tile][j][e][lane];
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S.comb_empty);
-                    // thread holds rows gq / gq+8 of the tile x columns 8j+2t, 8j+2t+1
-                    #pragma unroll
-                    for (int j = 0; j < NT; ++j)
-                        #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int m = 8 * j + 2 * t + (e & 1);
-                            const int n = q.row0 + 16 * tile + gq + ((e & 2) ? 8 : 0);
-                            if (m < pr.M && n < pr.N) pr.Y[static_cast<int64_t>(m) * pr.N + n] = sum[j][e];
+                    if constexpr (SPLIT) {
+                        if (q.split) {
+                            // rank 1 hands its sums to rank 0 of the cluster
+                            const int xb2 = split_done & 1;
+                            const uint32_t xpar = (split_done >> 1) & 1;
+                            ++split_done;
+                            if (rank == 1) {
+                                if (!wait_cluster_or_abort(&S.x.empty[xb2], xpar ^ 1, &S.abort_flag, P.err)) break;
+                                #pragma unroll
+                                for (int j = 0; j < NT; ++j)
+                                    #pragma unroll
+                                    for (int e = 0; e < 4; ++e) st_remote(&S.x.v[xb2][tile][j][e][lane], 0, sum[j][e]);
+                                mbar_arrive_remote(&S.x.full[xb2], 0);
+                            } else {
+                                if (!wait_cluster_or_abort(&S.x.full[xb2], xpar, &S.abort_flag, P.err)) break;
+                                #pragma unroll
+                                for (int j = 0; j < NT; ++j)
+                                    #pragma unroll
+                                    for (int e = 0; e < 4; ++e) sum[j][e] += S.x.v[xb2][tile][j][e][lane];
+                                mbar_arrive_remote(&S.x.empty[xb2], 1);
+                            }
                         }
+                    }
+                    // thread holds rows gq / gq+8 of the tile x columns 8j+2t, 8j+2t+1
+                    if (!q.split || rank == 0) {
+                        #pragma unroll
+                        for (int j = 0; j < NT; ++j)
+                            #pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int m = 8 * j + 2 * t + (e & 1);
+                                const int n = q.row0 + 16 * tile + gq + ((e & 2) ? 8 : 0);
+                                if (m < pr.M && n < pr.N) pr.Y[static_cast<int64_t>(m) * pr.N + n] = sum[j][e];
+                            }
+                    }
                 }
                 #pragma unroll
                 for (int c = 0; c < 2; ++c)
@@ -303,31 +477,154 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
             mbar_wait(&S.raw_full[gg % RS], (gg / RS) & 1, P.err);
         }
     }
+    if constexpr (SPLIT) {
+        __syncthreads();
+        cluster_sync_all();   // no CTA leaves while its partner may still reach its shared memory
+    }
 }
 
-template <int NT>
-constexpr size_t smem_bytes() { return sizeof(Smem<NT>) + 128; }
-static_assert(smem_bytes<4>() <= 232448, "shared memory budget");
+template <int NT, bool SPLIT>
+constexpr size_t smem_bytes() { return sizeof(Smem<NT, SPLIT>) + 128; }
+static_assert(smem_bytes<4, false>() <= 232448, "shared memory budget");
+static_assert(smem_bytes<1, true>() <= 232448, "shared memory budget");
+
+template <int NT, int CAP, bool SPLIT>
+cudaError_t configure(const q4::DeviceInfo &dev) {
+    static int configured_device = -1;
+    if (configured_device == dev.device) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<NT, CAP, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem_bytes<NT, SPLIT>()));
+    if (e != cudaSuccess) return e;
+    configured_device = dev.device;
+    return cudaSuccess;
+}
 
 template <int NT, int CAP>
-cudaError_t launch_nt(GroupParams<CAP> &P, const q4::DeviceInfo &dev, cudaStream_t s) {
-    static int configured_device = -1;
-    if (configured_device != dev.device) {
-        cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<NT, CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem_bytes<NT>()));
-        if (e != cudaSuccess) return e;
-        configured_device = dev.device;
-    }
-    const int grid = std::max(1, std::min(dev.sm_count, P.total_items));
-    decode_mma_kernel<NT, CAP><<<grid, kThreads, smem_bytes<NT>(), s>>>(P);
+cudaError_t launch_plain(DecodeParams<CAP> &D, const q4::DeviceInfo &dev, cudaStream_t s) {
+    cudaError_t e = configure<NT, CAP, false>(dev);
+    if (e != cudaSuccess) return e;
+    const int grid = std::max(1, std::min(dev.sm_count, D.g.total_items));
+    decode_mma_kernel<NT, CAP, false><<<grid, kThreads, smem_bytes<NT, false>(), s>>>(D);
     return cudaGetLastError();
+}
+
+cudaLaunchConfig_t cluster_config(int clusters, cudaStream_t s, cudaLaunchAttribute *attr) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * clusters, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem_bytes<1, true>();
+    cfg.stream = s;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cfg;
+}
+
+// Clusters of two that can be resident at once on this device (0 if none).
+template <int CAP>
+int split_clusters(const q4::DeviceInfo &dev) {
+    static int cached_device = -1, cached = 0;
+    if (cached_device == dev.device) return cached;
+    int n = 0;
+    if (configure<1, CAP, true>(dev) == cudaSuccess) {
+        cudaLaunchAttribute attr[1];
+        cudaLaunchConfig_t cfg = cluster_config(std::max(1, dev.sm_count / 2), nullptr, attr);
+        if (cudaOccupancyMaxActiveClusters(&n, decode_mma_kernel<1, CAP, true>, &cfg) != cudaSuccess) n = 0;
+    }
+    (void)cudaGetLastError();
+    cached = std::min(n, kMaxSplitCtas / 2);
+    cached_device = dev.device;
+    return cached;
+}
+
+// The split-mode schedule.  Items longer than the mean load of a CTA are
+// split and dealt to the clusters (cost ceil(n/2) on each CTA of the pair);
+// each CTA's list starts with its cluster's split items, in the same order on
+// both CTAs.  The whole items follow, dealt to single CTAs; every deal puts
+// the next-longest item onto the least loaded cluster or CTA.
+template <int CAP>
+void build_schedule(DecodeParams<CAP> &D, int clusters) {
+    const GroupParams<CAP> &P = D.g;
+    const int ctas = 2 * clusters;
+    long total = 0;
+    for (int i = 0; i < P.count; ++i) {
+        const int nitems = (i + 1 < P.count ? P.p[i + 1].item_begin : P.total_items) - P.p[i].item_begin;
+        total += static_cast<long>(nitems) * P.p[i].stages;
+    }
+    const long mean = (total + ctas - 1) / ctas;
+    using Load = std::pair<long, int>;
+    std::vector<std::vector<uint16_t>> split_of(clusters), whole_of(ctas);
+    std::vector<long> load(ctas, 0);
+    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> cl;
+    for (int c = 0; c < clusters; ++c) cl.push({0, c});
+    for (int i = 0; i < P.count; ++i) {   // problems come sorted by K, largest first
+        const int n = P.p[i].stages;
+        if (n < 2 || n <= mean) continue;
+        const int nitems = (i + 1 < P.count ? P.p[i + 1].item_begin : P.total_items) - P.p[i].item_begin;
+        for (int k = 0; k < nitems; ++k) {
+            Load l = cl.top();
+            cl.pop();
+            split_of[l.second].push_back(static_cast<uint16_t>(P.p[i].item_begin + k));
+            l.first += (n + 1) / 2;
+            load[2 * l.second] = load[2 * l.second + 1] = l.first;
+            cl.push(l);
+        }
+    }
+    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> ct;
+    for (int b = 0; b < ctas; ++b) ct.push({load[b], b});
+    for (int i = 0; i < P.count; ++i) {
+        const int n = P.p[i].stages;
+        if (!(n < 2 || n <= mean)) continue;
+        const int nitems = (i + 1 < P.count ? P.p[i + 1].item_begin : P.total_items) - P.p[i].item_begin;
+        for (int k = 0; k < nitems; ++k) {
+            Load l = ct.top();
+            ct.pop();
+            whole_of[l.second].push_back(static_cast<uint16_t>(P.p[i].item_begin + k));
+            l.first += n;
+            ct.push(l);
+        }
+    }
+    int pos = 0;
+    for (int b = 0; b < ctas; ++b) {
+        D.sched_begin[b] = static_cast<uint16_t>(pos);
+        for (uint16_t it : split_of[b >> 1]) D.sched[pos++] = static_cast<uint16_t>(it | kSplitFlag);
+        for (uint16_t it : whole_of[b]) D.sched[pos++] = it;
+    }
+    D.sched_begin[ctas] = static_cast<uint16_t>(pos);
+}
+
+// The schedule depends only on the clusters and on each problem's stages and
+// item count; a call with the same shapes as the previous one on this thread
+// (the usual case: the same layer every token) keeps the schedule that `D`
+// still holds.
+template <int CAP>
+cudaError_t launch_split(DecodeParams<CAP> &D, int clusters, cudaStream_t s) {
+    static thread_local std::vector<int> last;
+    thread_local std::vector<int> sig;
+    const GroupParams<CAP> &P = D.g;
+    sig.assign({clusters, P.count, P.total_items});
+    for (int i = 0; i < P.count; ++i) {
+        sig.push_back(P.p[i].stages);
+        sig.push_back(P.p[i].item_begin);
+    }
+    if (sig != last) {
+        build_schedule(D, clusters);
+        last = sig;
+    }
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = cluster_config(clusters, s, attr);
+    return cudaLaunchKernelEx(&cfg, decode_mma_kernel<1, CAP, true>, D);
 }
 
 // problems[order[0..count)] sorted by K (largest first), count <= CAP
 template <int CAP>
 cudaError_t launch_cap(const q4::Problem *probs, const int *order, int count, const q4::DeviceInfo &dev,
                        cudaStream_t s) {
-    static thread_local GroupParams<CAP> P;
+    static thread_local DecodeParams<CAP> D;
+    GroupParams<CAP> &P = D.g;
     P.count = count;
     P.err = dev.err;
     int items = 0;
@@ -349,9 +646,18 @@ cudaError_t launch_cap(const q4::Problem *probs, const int *order, int count, co
             return cudaErrorInvalidValue;
     }
     P.total_items = items;
-    if (maxM <= 8) return launch_nt<1, CAP>(P, dev, s);
-    if (maxM <= 16) return launch_nt<2, CAP>(P, dev, s);
-    return launch_nt<4, CAP>(P, dev, s);
+    if (maxM <= 8) {
+        // fewer items than SMs: each CTA has at most one item and the launch is
+        // latency-bound, where the hand-over between a pair costs more than it
+        // saves (measured on a single 3072 x 3072 GEMV)
+        if (items >= dev.sm_count && items <= kMaxItems) {
+            const int clusters = std::min(split_clusters<CAP>(dev), items);
+            if (clusters >= 1) return launch_split<CAP>(D, clusters, s);
+        }
+        return launch_plain<1, CAP>(D, dev, s);
+    }
+    if (maxM <= 16) return launch_plain<2, CAP>(D, dev, s);
+    return launch_plain<4, CAP>(D, dev, s);
 }
 
 constexpr int kSmallCap = 8, kLargeCap = 128;
@@ -368,7 +674,8 @@ bool decode_mma_supports(const Problem &p) {
 
 cudaError_t launch_decode_mma(const Problem *probs, int count, const DeviceInfo &dev, cudaStream_t s) {
     if (count <= 0) return cudaSuccess;
-    std::vector<int> order(count);
+    static thread_local std::vector<int> order;
+    order.resize(count);
     for (int i = 0; i < count; ++i) order[i] = i;
     std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return probs[a].K > probs[b].K; });
     for (int done = 0; done < count;) {

@@ -243,6 +243,67 @@ def test_decode_workloads_sampled(q4, name, layers):
     check_built(b, name)
 
 
+def test_split_mode_mixed_stage_counts(q4):
+    """M <= 8 with between 148 and 1024 items runs in clusters of two CTAs:
+    items longer than the mean load (K = 8192 here, 32 stages; and the odd
+    7424, 29 stages, whose first half gets the extra stage) are halved
+    between the pair, the rest (8-, 3- and 1-stage items) stay whole."""
+    o = oracle.get()
+    rng = np.random.default_rng(31)
+    shapes = [(3, 12800, 2048), (3, 2900, 8192), (2, 300, 7424), (1, 3000, 256), (8, 1000, 768)]
+    probs, refs, Ys = [], [], []
+    for (M, N, K) in shapes:
+        codes, scales, X = rand_inputs(rng, M, N, K)
+        Y = torch.full((M, N), float("nan"), device="cuda")
+        probs.append((pack_on_gpu(q4, codes, scales), dev(X), Y, M, N, K))
+        refs.append(o.gemm(o.pack(codes, scales), X, M, N, K))
+        Ys.append(Y)
+    for rep in range(2):
+        for Y in Ys:
+            Y.fill_(float("nan"))
+        q4.q4_0_gemm_grouped(probs)
+        for (M, N, K), Y, (Y_or, B_or) in zip(shapes, Ys, refs):
+            check_gemm(Y.cpu().numpy(), Y_or, B_or, f"split mode M={M} N={N} K={K} rep {rep}")
+    no_device_error(q4)
+
+
+def test_grouped_call_replays_from_cuda_graph(q4):
+    """A grouped decode call captured in a CUDA graph (after one eager call,
+    which does the per-device set-up) replays to the eager call's bits."""
+    rng = np.random.default_rng(41)
+    shapes = [(1, 5120, 3072), (1, 3072, 3072), (1, 16384, 3072), (1, 3072, 8192)]   # one decoder layer
+    probs, Ys = [], []
+    for (M, N, K) in shapes:
+        codes, scales, X = rand_inputs(rng, M, N, K)
+        Y = torch.full((M, N), float("nan"), device="cuda")
+        probs.append((pack_on_gpu(q4, codes, scales), dev(X), Y, M, N, K))
+        Ys.append(Y)
+    arr = q4.make_problems(probs)
+    q4.q4_0_gemm_grouped(arr, len(probs))
+    torch.cuda.synchronize()
+    eager = [Y.clone() for Y in Ys]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        q4.q4_0_gemm_grouped(arr, len(probs))
+    for rep in range(2):
+        for Y in Ys:
+            Y.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        for Y, E in zip(Ys, eager):
+            assert torch.equal(Y, E)
+    no_device_error(q4)
+
+
+def test_plain_mode_many_items(q4):
+    """More than 1024 items at M <= 8: one CTA per item, boustrophedon deal."""
+    b = build_workload(q4, workloads.workload("cfg_decode", layers=[0, 1, 2, 3, 4]), samples=200)
+    assert sum((N + 127) // 128 for (_, N, _) in b.shapes) > 1024
+    q4.q4_0_gemm_grouped(b.problems())
+    check_built(b, "cfg_decode 5 layers")
+    no_device_error(q4)
+
+
 @pytest.mark.parametrize("M,N,K", [(64, 128, 512), (300, 200, 1024), (4096, 256, 768)])
 def test_workspace_path_matches(q4, M, N, K):
     """q4_0_gemm_ws (X converted to fp16 once, in the workspace) gives the
