@@ -37,7 +37,7 @@ def build(mutant: int = 0, force: bool = False) -> str:
         return out
     os.makedirs(_BUILD, exist_ok=True)
     tmp = out + f".tmp{os.getpid()}"
-    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math", "-ffp-contract=off",
            f"-DORACLE_MUTANT={mutant}", _SRC, "-o", tmp, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, out)
@@ -67,6 +67,12 @@ class Oracle:
         L.oracle_q4_0_gemm.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64]
         L.oracle_q4_0_gemm_sampled.restype = None
         L.oracle_q4_0_gemm_sampled.argtypes = [_p, _p, _i64, _i64, _i64, _p, _p, _i64, _p, _p]
+        L.oracle_q4_0_gather_f32.restype = _i64
+        L.oracle_q4_0_gather_f32.argtypes = [_p, _p, _p, _i64, _i64, _i64]
+        L.oracle_float_to_half.restype = ctypes.c_uint16
+        L.oracle_float_to_half.argtypes = [ctypes.c_float]
+        L.oracle_q4_0_quantize.restype = None
+        L.oracle_q4_0_quantize.argtypes = [_p, _p, _i64, _i64]
 
     # -- scalar decoders -------------------------------------------------
     def half_to_double(self, h: int) -> float:
@@ -142,6 +148,28 @@ class Oracle:
                                            ms.ctypes.data, ns.ctypes.data, len(ms),
                                            Y.ctypes.data, B.ctypes.data)
         return Y, B
+
+
+    def gather_f32(self, W: np.ndarray, ids: np.ndarray, V: int, D: int):
+        """Rows ids of W[V, D] (Q4_0) as float32 [T, D]; returns (out, count of ids outside [0, V))."""
+        W = self._c(W, np.uint8)
+        ids = self._c(ids, np.int32)
+        out = np.empty((len(ids), D), np.float32)
+        bad = self._lib.oracle_q4_0_gather_f32(W.ctypes.data, ids.ctypes.data, out.ctypes.data, len(ids), V, D)
+        return out, int(bad)
+
+    def float_to_half(self, f: float) -> int:
+        return int(self._lib.oracle_float_to_half(float(f)))
+
+    def quantize(self, X: np.ndarray) -> np.ndarray:
+        """float32 [N, K] -> Q4_0 bytes [N, K/32*18] by the GGUF Q4_0 rule."""
+        X = self._c(X, np.float32)
+        N, K = X.shape
+        if K % 32:
+            raise ValueError("K must be a multiple of 32")
+        W = np.empty((N, K // 32 * 18), np.uint8)
+        self._lib.oracle_q4_0_quantize(X.ctypes.data, W.ctypes.data, N, K)
+        return W
 
 
 _default = None

@@ -29,6 +29,23 @@
  *
  * Every product (q-8)*d*x is exact in float64 (4 + 11 + 8 significant bits).
  *
+ * Two more operations around the product (the next steps the survey ranks,
+ * not the hot path itself):
+ *   gather   -- rows ids[t] of a Q4_0 matrix W[V, D] dequantized to float32:
+ *               the Q4 embedding lookup the pages run on the CPU instead of
+ *               keeping a 1.5 GiB fp32 table (hakusoku.com story 5135, linear
+ *               ops and embeddings; voxtral-mini-realtime-rs README, "WASM
+ *               Constraints Solved", item 3).  An id outside [0, V) gives a
+ *               row of zeros (the pages do not say; reading of this library).
+ *   quantize -- float32 weights to Q4_0 blocks by the GGUF Q4_0 rule, which
+ *               the pages use offline (their quantize_tts_gguf.py, named in
+ *               the voxtral-mini-realtime-rs README, TTS section) but do not
+ *               print: per block of 32, m = the value of largest magnitude
+ *               (the first one on ties), d = m / -8, id = 1/d (0 if d == 0),
+ *               q = min(15, trunc(x * id + 8.5)), all in float32 with no
+ *               fused multiply-add; the block stores fp16(d), rounded to
+ *               nearest even.  Inputs must be finite.
+ *
  * ORACLE_MUTANT: when compiled with -DORACLE_MUTANT=<n> (n >= 1) one
  * deliberate mistake is planted so that the pin tests can show they catch it.
  * The default build (no macro) is the oracle.
@@ -37,6 +54,7 @@
 #include <stddef.h>
 #include <stdlib.h>
 #include <math.h>
+#include <string.h>
 
 #ifndef ORACLE_MUTANT
 #define ORACLE_MUTANT 0
@@ -215,4 +233,108 @@ void oracle_q4_0_gemm_sampled(const uint8_t *W, const uint16_t *X, int64_t M,
     (void)N;
     for (int64_t i = 0; i < count; i++)
         q4_0_dot(W, X, K, ms[i], ns[i], &Y[i], &B[i]);
+}
+
+/* Rows ids[0..T) of W[V, D] (Q4_0) dequantized to float32 (exact); an id
+ * outside [0, V) gives a row of zeros.  Returns the number of such ids. */
+int64_t oracle_q4_0_gather_f32(const uint8_t *W, const int32_t *ids, float *out,
+                               int64_t T, int64_t V, int64_t D)
+{
+    int64_t bad = 0;
+    for (int64_t t = 0; t < T; t++) {
+#if ORACLE_MUTANT == 7
+        int64_t v = (int64_t)ids[t] + 1; /* planted: off-by-one row */
+#else
+        int64_t v = (int64_t)ids[t];
+#endif
+        for (int64_t k = 0; k < D; k++) {
+            if (v < 0 || v >= V)
+                out[t * D + k] = 0.0f;
+            else
+                out[t * D + k] = (float)q4_0_weight(W, D, v, k);
+        }
+        if (v < 0 || v >= V)
+            bad++;
+    }
+    return bad;
+}
+
+/* IEEE binary32 -> binary16 bits, rounding to nearest, ties to even, by bit
+ * arithmetic: overflow gives +-inf, NaN stays NaN (quiet), values below half
+ * the smallest subnormal give +-0. */
+uint16_t oracle_float_to_half(float f)
+{
+    uint32_t x;
+    memcpy(&x, &f, 4);
+    uint32_t sign = (x >> 16) & 0x8000u;
+    int32_t exp = (int32_t)((x >> 23) & 0xffu);
+    uint32_t man = x & 0x7fffffu;
+    if (exp == 0xff)
+        return (uint16_t)(sign | 0x7c00u | (man ? 0x200u : 0u));
+    int32_t e = exp - 127 + 15;              /* biased binary16 exponent */
+    if (e >= 31)
+        return (uint16_t)(sign | 0x7c00u);
+    if (e <= 0) {                            /* binary16 subnormal or zero */
+        if (e < -10)
+            return (uint16_t)sign;
+        uint32_t full = man | 0x800000u;     /* 24-bit significand */
+        int shift = 14 - e;                  /* 14 .. 24 */
+        uint32_t hm = full >> shift;
+        uint32_t rem = full & ((1u << shift) - 1u);
+        uint32_t half = 1u << (shift - 1);
+        if (rem > half || (rem == half && (hm & 1u)))
+            hm++;                            /* may carry into the smallest normal */
+        return (uint16_t)(sign | hm);
+    }
+    uint32_t h = sign | ((uint32_t)e << 10) | (man >> 13);
+    uint32_t rem = man & 0x1fffu;
+    if (rem > 0x1000u || (rem == 0x1000u && (h & 1u)))
+        h++;                                 /* a carry moves into the exponent, up to inf */
+    return (uint16_t)h;
+}
+
+/* X[N, K] float32 -> W (Q4_0), K a multiple of 32, by the rule in the header. */
+void oracle_q4_0_quantize(const float *X, uint8_t *W, int64_t N, int64_t K)
+{
+    int64_t nb = K / 32;
+    for (int64_t n = 0; n < N; n++) {
+        for (int64_t b = 0; b < nb; b++) {
+            const float *x = X + n * K + b * 32;
+            float amax = 0.0f, m = 0.0f;
+            for (int j = 0; j < 32; j++) {
+                float a = fabsf(x[j]);
+#if ORACLE_MUTANT == 9
+                if (amax <= a) { /* planted: the last of equal magnitudes wins */
+#else
+                if (amax < a) {
+#endif
+                    amax = a;
+                    m = x[j];
+                }
+            }
+#if ORACLE_MUTANT == 8
+            float d = m / 8.0f; /* planted: scale sign flipped */
+#else
+            float d = m / -8.0f;
+#endif
+            float id = (d != 0.0f) ? 1.0f / d : 0.0f;
+            uint8_t q[32];
+            for (int j = 0; j < 32; j++) {
+                volatile float p = x[j] * id;   /* separate rounding of the product */
+#if ORACLE_MUTANT == 10
+                float v = p + 8.0f;             /* planted: truncation, not rounding */
+#else
+                float v = p + 8.5f;
+#endif
+                int c = (int)v;                 /* v >= 0 for finite inputs: truncation */
+                q[j] = (uint8_t)(c > 15 ? 15 : c);
+            }
+            uint16_t dh = oracle_float_to_half(d);
+            uint8_t *blk = W + (n * nb + b) * 18;
+            blk[0] = (uint8_t)(dh & 0xff);
+            blk[1] = (uint8_t)(dh >> 8);
+            for (int j = 0; j < 16; j++)
+                blk[2 + j] = (uint8_t)((q[j] & 0x0f) | ((q[j + 16] & 0x0f) << 4));
+        }
+    }
 }

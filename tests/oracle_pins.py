@@ -15,6 +15,14 @@ What each pin is tied to:
     nibble gives exactly (c-8)*d*x; constant codes with constant X give
     x*(c-8)*32*sum(d)), linearity in X, and brute force on tiny shapes via
     numpy's matmul on weights built straight from the unpacked codes;
+  * fp32 -> fp16 rounding: numpy's float16 conversion (round to nearest
+    even) on special values and random bit patterns;
+  * quantization: hand-derived blocks in tests/golden/q4_0_quantize.txt, and
+    properties of the rule computed independently with numpy (the extreme
+    element maps to code 0, every other element is within half a step of
+    its reconstruction, symmetry under negation and power-of-two scaling);
+  * gather: equals the pinned dequantization row by row, zero rows for ids
+    out of range;
   * sizes: 4.5 bits per weight, cross-checked with the pages' 1.5 GiB fp32
     embedding table that becomes 216 MB in Q4 (hakusoku.com story 5135,
     linear ops and embeddings; voxtral-mini-realtime-rs README, "WASM
@@ -29,6 +37,7 @@ from fractions import Fraction
 import numpy as np
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "q4_0_blocks.txt")
+QGOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "q4_0_quantize.txt")
 
 
 def load_golden():
@@ -245,6 +254,112 @@ def pin_sizes(o):
     assert o.row_bytes(3072) * 8 * 2 == 3072 * 9
 
 
+def load_quantize_golden():
+    cases, cur = [], None
+    for raw in open(QGOLDEN):
+        line = raw.strip()
+        if not line or line.startswith("#"):
+            continue
+        key, _, rest = line.partition(" ")
+        if key == "case":
+            cur = {"name": rest}
+        elif key == "x":
+            vals = [Fraction(v) for v in rest.split()]
+            x = np.array([float(v) for v in vals], np.float32)
+            assert [Fraction(float(v)) for v in x] == vals, "fixture values must be exact in float32"
+            cur["x"] = x
+        elif key == "bytes":
+            cur["bytes"] = np.array([int(b, 16) for b in rest.split()], np.uint8)
+        elif key == "end":
+            assert len(cur["x"]) == 32 and len(cur["bytes"]) == 18
+            cases.append(cur)
+            cur = None
+    return cases
+
+
+def pin_float_to_half(o):
+    special = np.array([0.0, -0.0, 1.0, -1.0, 65504.0, 65519.99, 65520.0, 1e9, -1e9, np.inf, -np.inf,
+                        2.0**-14, 2.0**-24, 2.0**-25, 2.0**-25 * 1.0000001, 2.0**-26, 3 * 2.0**-25,
+                        2.0**-14 - 2.0**-25, 1.0 + 2.0**-11, 1.0 + 3 * 2.0**-11, 0.1, 1 / 3], np.float32)
+    rng = np.random.default_rng(5)
+    bits = rng.integers(0, 2**32, size=200000, dtype=np.uint64).astype(np.uint32)
+    vals = np.concatenate([special, bits.view(np.float32)])
+    with np.errstate(over="ignore"):
+        ref = vals.astype(np.float16)
+    for v, r in zip(vals, ref):
+        h = o.float_to_half(float(v))
+        if np.isnan(v):
+            assert (h & 0x7c00) == 0x7c00 and (h & 0x3ff) != 0
+        else:
+            assert h == int(r.view(np.uint16)), (float(v), hex(h), hex(int(r.view(np.uint16))))
+
+
+def pin_quantize_golden(o):
+    for c in load_quantize_golden():
+        W = o.quantize(c["x"].reshape(1, 32))
+        assert np.array_equal(W.reshape(-1), c["bytes"]), (c["name"], W.reshape(-1).tobytes().hex(" "))
+
+
+def _blocks(rng, n):
+    """Blocks of 32 float32 values at scales over many binades, some with
+    repeated extreme magnitudes."""
+    x = rng.standard_normal((n, 32)).astype(np.float32)
+    x *= np.exp2(rng.integers(-12, 12, size=(n, 1))).astype(np.float32)
+    x[::7, 9] = -x[::7, 3]            # the same magnitude twice, opposite signs
+    return x
+
+
+def pin_quantize_rounding_bound(o):
+    rng = np.random.default_rng(6)
+    X = _blocks(rng, 400)
+    W = o.quantize(X.reshape(-1, 64))   # 200 rows of two blocks
+    codes, scales = o.unpack(W, 200, 64)
+    codes = codes.reshape(-1, 32).astype(np.float64)
+    scales = scales.reshape(-1)
+    for x, q, dh in zip(X, codes, scales):
+        i = int(np.argmax(np.abs(x)))          # first of the largest magnitudes
+        d = np.float32(x[i]) / np.float32(-8.0)
+        assert int(np.float16(d).view(np.uint16)) == int(dh)
+        assert q[i] == 0
+        err = np.abs((q - 8) * np.float64(d) - x.astype(np.float64))
+        step = abs(float(d))
+        # x/d lies in [-8, 8]; codes above 15 are clamped, so values with
+        # x/d >= 7.5 (the far side from the extreme) may be off by one step
+        clamped = x.astype(np.float64) / np.float64(d) >= 7.5 - 2.0**-18
+        assert np.all(err[~clamped] <= 0.5 * step * (1 + 2.0**-20)), float(err[~clamped].max() / step)
+        assert np.all(err[clamped] <= step * (1 + 2.0**-20))
+        assert np.all(q[clamped] == 15)
+
+
+def pin_quantize_sign_and_scale(o):
+    rng = np.random.default_rng(7)
+    X = _blocks(rng, 64).reshape(-1, 64)
+    c0, s0 = o.unpack(o.quantize(X), 32, 64)
+    c1, s1 = o.unpack(o.quantize(-X), 32, 64)
+    assert np.array_equal(c0, c1) and np.array_equal(s0 ^ 0x8000, s1)
+    for k in (-3, 5):
+        c2, s2 = o.unpack(o.quantize(X * np.float32(2.0**k)), 32, 64)
+        assert np.array_equal(c0, c2)
+        d = s0.view(np.float16).astype(np.float64) * 2.0**k
+        ok = np.abs(d) >= 2.0**-14           # scales that stay normal in fp16
+        assert np.array_equal(s2.view(np.float16).astype(np.float64)[ok], d[ok])
+
+
+def pin_gather_matches_dequant(o):
+    rng = np.random.default_rng(8)
+    V, D = 37, 96
+    codes = rng.integers(0, 16, size=(V, D), dtype=np.uint8)
+    scales = (rng.standard_normal((V, D // 32)) * 0.01).astype(np.float16).view(np.uint16)
+    W = o.pack(codes, scales)
+    full = o.dequant_f32(W, V, D)
+    ids = np.concatenate([rng.permutation(V), rng.integers(0, V, 20), [0, V - 1, V - 1]]).astype(np.int32)
+    out, bad = o.gather_f32(W, ids, V, D)
+    assert bad == 0 and np.array_equal(out, full[ids])
+    out, bad = o.gather_f32(W, np.array([-1, 3, V, 2**31 - 1], np.int32), V, D)
+    assert bad == 3 and np.array_equal(out[1], full[3])
+    assert not out[[0, 2, 3]].any()
+
+
 ALL_PINS = [
     pin_half_decoder,
     pin_bf16_decoder,
@@ -258,4 +373,9 @@ ALL_PINS = [
     pin_linearity,
     pin_sampled_matches_full,
     pin_sizes,
+    pin_float_to_half,
+    pin_quantize_golden,
+    pin_quantize_rounding_bound,
+    pin_quantize_sign_and_scale,
+    pin_gather_matches_dequant,
 ]

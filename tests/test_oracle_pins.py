@@ -24,6 +24,10 @@ MUTANTS = {
     4: "last block of each row dropped from the sum",
     5: "fp16 exponent bias off by one",
     6: "output written transposed",
+    7: "gather reads the next row",
+    8: "quantization scale with the wrong sign",
+    9: "quantization takes the last of equal extreme magnitudes",
+    10: "quantization truncates instead of rounding",
 }
 
 
