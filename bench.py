@@ -56,6 +56,7 @@ DOMINANT = {
     "qkv_prefill": ("prefill_kernel", "q4_0_prefill.cu"),
 }
 TENSOR_WORKLOADS = ("adapter", "qkv_prefill")
+UTIL_KERNELS = {"embed": ("gather_kernel", "q4_0_embed.cu"), "quantize": ("quantize_kernel", "q4_0_embed.cu")}
 
 
 def log(*a):
@@ -83,7 +84,7 @@ def source_sha(fname: str) -> str:
 def recorded_traffic(workload: str):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
     summary, or None when absent or when the kernel source changed since."""
-    kernel, src = DOMINANT[workload]
+    kernel, src = DOMINANT[workload] if workload in DOMINANT else UTIL_KERNELS[workload]
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.traffic.json")
     if not os.path.exists(path):
         return None
@@ -357,6 +358,180 @@ def run_ours(args, rank: int, world: int):
     return line
 
 
+# --------------------------------------------------------------------------- the utilities
+
+def util_setup(q4, name: str, seed: int):
+    """Device buffers of one utility workload and a launch per step.  Returns
+    (launch(k), bytes per step, e2e step(k), h2d bytes, d2h bytes)."""
+    import torch
+    if name == "embed":
+        V, D, T = workloads.EMBED_VOCAB, workloads.EMBED_DIM, workloads.EMBED_TOKENS
+        W = torch.empty(q4.q4_0_bytes(V, D), dtype=torch.uint8, device="cuda")
+        rows = 8192
+        for r0 in range(0, V, rows):   # the table, packed on the GPU from seeded codes and scales, in slices
+            codes = torch.from_numpy(workloads.gen_codes(rows, D, seed, layer=r0 // rows)).cuda()
+            scales = torch.from_numpy(workloads.gen_scales(rows, D, seed, layer=r0 // rows).view(np.int16)).cuda()
+            q4.q4_0_pack(codes, scales, W[r0 * (D // 32) * 18:(r0 + rows) * (D // 32) * 18], rows, D)
+        ids = [torch.from_numpy(workloads.gen_ids(T, V, seed, stream=i)).cuda() for i in range(4)]
+        outs = [torch.empty((T, D), device="cuda") for _ in range(2)]
+        hid = torch.empty(T, dtype=torch.int32, pin_memory=True).copy_(ids[0].cpu())
+        hout = torch.empty((T, D), dtype=torch.float32, pin_memory=True)
+
+        def launch(k):
+            q4.q4_0_gather(W, ids[k % 4], outs[k % 2], T, V, D)
+
+        def e2e(k):
+            ids[k % 4].copy_(hid, non_blocking=True)
+            launch(k)
+            hout.copy_(outs[k % 2], non_blocking=True)
+
+        return launch, T * (D // 32 * 18 + 4 + 4 * D), e2e, T * 4, T * D * 4
+    N, K = workloads.QUANT_N, workloads.QUANT_K
+    Xs = [torch.from_numpy(workloads.gen_weights(N, K, seed, stream=i)).cuda() for i in range(2)]
+    Ws = [torch.empty(q4.q4_0_bytes(N, K), dtype=torch.uint8, device="cuda") for _ in range(2)]
+    hx = torch.empty((N, K), dtype=torch.float32, pin_memory=True).copy_(Xs[0].cpu())
+    hw = torch.empty(q4.q4_0_bytes(N, K), dtype=torch.uint8, pin_memory=True)
+
+    def launch(k):
+        q4.q4_0_quantize(Xs[k % 2], Ws[k % 2], N, K)
+
+    def e2e(k):
+        Xs[k % 2].copy_(hx, non_blocking=True)
+        launch(k)
+        hw.copy_(Ws[k % 2], non_blocking=True)
+
+    return launch, N * K * 4 + q4.q4_0_bytes(N, K), e2e, N * K * 4, q4.q4_0_bytes(N, K)
+
+
+def util_cpu_sample(name: str, budget_s: float):
+    """The oracle on a host-generated sample of the same workload; returns
+    (GB/s, sample description)."""
+    import oracle
+    o = oracle.get()
+    if name == "embed":
+        V, D = 2048, workloads.EMBED_DIM
+        W = o.pack(workloads.gen_codes(V, D), workloads.gen_scales(V, D))
+        ids = workloads.gen_ids(256, V)
+        per = len(ids) * (D // 32 * 18 + 4 + 4 * D)
+        fn = lambda: o.gather_f32(W, ids, V, D)   # noqa: E731
+        what = f"gather of 256 random rows of a {V} x {D} table per pass"
+    else:
+        X = workloads.gen_weights(64, workloads.QUANT_K)
+        per = X.size * 4 + X.size // 32 * 18
+        fn = lambda: o.quantize(X)   # noqa: E731
+        what = f"quantize of a 64 x {workloads.QUANT_K} slice per pass"
+    t0, reps = time.perf_counter(), 0
+    while True:
+        fn()
+        reps += 1
+        if time.perf_counter() - t0 > budget_s or reps >= 2000:
+            break
+    dt = time.perf_counter() - t0
+    return per * reps / dt / 1e9, f"{reps} passes: {what}, {dt:.1f} s, scaled by bytes"
+
+
+def run_util(args, rank: int, world: int):
+    import torch
+    import bit_weight_only_matmul_b200 as q4
+    launch, step_bytes, e2e, h2d, d2h = util_setup(q4, args.workload, workloads.SEED + 1000 * rank)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    q4.q4_0_device_error(clear=True)
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        for k in range(args.warmup):
+            launch(k)
+        barrier()
+        t_end, k = time.time() + args.soak, 0
+        while time.time() < t_end:
+            for _ in range(8):
+                launch(k)
+                k += 1
+            torch.cuda.synchronize()
+        barrier()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for k in range(args.steps):
+            launch(k)
+        t1.record(stream)
+        barrier()
+    ms_total = t0.elapsed_time(t1)
+    if q4.q4_0_device_error(clear=True):
+        raise RuntimeError("device error word set after the timed region")
+    for k in range(args.warmup):
+        e2e(k)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for k in range(args.steps):
+        e2e(k)
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    ms_total, e2e_ms = max_over_ranks([ms_total, e2e_ms], world, "cuda")
+    if rank != 0:
+        return None
+    peaks = measured_peaks()
+    kernel, _ = UTIL_KERNELS[args.workload]
+    value = whole_job_rate(step_bytes, args.steps, world, ms_total) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_total / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "q4_0 -> fp32" if args.workload == "embed" else "fp32 -> q4_0",
+        "data": "synthetic (seeded Philox)",
+        "config": {"workload": f"{args.workload}: {workloads.UTIL_WORKLOADS[args.workload]}",
+                   "bytes_per_step": step_bytes,
+                   "l2": "inputs larger than L2 (the 216 MiB table / 201 MB of fp32 weights), rotating buffers",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU", "launch": "eager"},
+        "roofline": {"bound": "hbm", "kernel": kernel, "achieved": round(value / world, 2),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(value / world / peaks["hbm_gbs"], 4),
+                     "peak_source": peaks["source"] + " (STREAM-style copy)",
+                     "traffic": recorded_traffic(args.workload), "algorithmic_per_launch": step_bytes},
+        "e2e": {"value": round(whole_job_rate(step_bytes, args.steps, world, e2e_ms) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+    }
+    if not args.no_cpu_baseline and world == 1:
+        v, what = util_cpu_sample(args.workload, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": what}
+    return line
+
+
+def run_util_reference(args, rank: int):
+    if rank != 0:
+        return None
+    for _ in range(args.warmup):
+        util_cpu_sample(args.workload, 0.0)
+    t0 = time.perf_counter()
+    vals = [util_cpu_sample(args.workload, 0.0) for _ in range(args.steps)]
+    dt = time.perf_counter() - t0
+    value = statistics.mean(v for v, _ in vals)
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded Philox)",
+            "config": {"workload": f"{args.workload}: {workloads.UTIL_WORKLOADS[args.workload]}",
+                       "parallelism": "one host core"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": vals[0][1]},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
 def max_over_ranks(values, world: int, device: str):
     """Element-wise max of per-rank timings (every rank gets the result)."""
     if world <= 1:
@@ -475,7 +650,7 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=workloads.WORKLOADS)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=workloads.WORKLOADS + list(UTIL_KERNELS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline budget (rank 0, N=1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -495,7 +670,10 @@ def main(argv=None):
         log(f"note: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE")
 
     if args.impl == "reference":
-        line = run_reference(args, rank, world)
+        if args.workload in UTIL_KERNELS:
+            line = run_util_reference(args, rank)
+        else:
+            line = run_reference(args, rank, world)
         if line is not None:
             print(json.dumps(line), flush=True)
         return 0
@@ -507,7 +685,7 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
     try:
-        line = run_ours(args, rank, world)
+        line = run_util(args, rank, world) if args.workload in UTIL_KERNELS else run_ours(args, rank, world)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -25,6 +25,7 @@ Q4_ERR_CUDA = 4
 Q4_ERR_TOO_LARGE = 5
 
 Q4_DEVERR_WAIT_TIMEOUT = 1
+Q4_DEVERR_BAD_INDEX = 2
 
 Q4_0_MAX_GROUP = 256
 Q4_0_STATIC_WS_BYTES = 64 << 20
@@ -43,6 +44,8 @@ EXPORTS = (
     "q4_0_gemm_ws",
     "q4_0_gemm_static_ws",
     "q4_0_gemm_grouped",
+    "q4_0_gather",
+    "q4_0_quantize",
     "q4_0_device_error",
     "q4_0_force_path",
 )
@@ -78,6 +81,8 @@ def _load() -> ctypes.CDLL:
         "q4_0_gemm_ws": (i32, [vp, vp, vp, i64, i64, i64, vp, i64, vp]),
         "q4_0_gemm_static_ws": (i32, [vp, vp, vp, i64, i64, i64, vp]),
         "q4_0_gemm_grouped": (i32, [ctypes.POINTER(q4_0_problem), i32, vp]),
+        "q4_0_gather": (i32, [vp, vp, vp, i64, i64, i64, vp]),
+        "q4_0_quantize": (i32, [vp, vp, i64, i64, vp]),
         "q4_0_device_error": (i32, [ctypes.POINTER(ctypes.c_uint32), i32]),
         "q4_0_force_path": (i32, [i32]),
     }
@@ -174,6 +179,16 @@ def q4_0_gemm_grouped(problems, count: Optional[int] = None, stream=None) -> Non
     elif count is None:
         count = len(problems)
     _check(_lib.q4_0_gemm_grouped(problems, count, _stream(stream)), "q4_0_gemm_grouped")
+
+
+def q4_0_gather(W, ids, out, T: int, V: int, D: int, stream=None) -> None:
+    """out[t] = dequant(W)[ids[t]] (float32 [T, D]); ids int32 on the device."""
+    _check(_lib.q4_0_gather(_ptr(W), _ptr(ids), _ptr(out), T, V, D, _stream(stream)), "q4_0_gather")
+
+
+def q4_0_quantize(X, W, N: int, K: int, stream=None) -> None:
+    """float32 X [N, K] -> Q4_0 bytes W (GGUF Q4_0 rule, bit-exact)."""
+    _check(_lib.q4_0_quantize(_ptr(X), _ptr(W), N, K, _stream(stream)), "q4_0_quantize")
 
 
 def q4_0_device_error(clear: bool = True) -> int:

@@ -229,6 +229,35 @@ int q4_0_gemm_static_ws(const void *W, const uint16_t *X, float *Y, int64_t M, i
     return q4_0_gemm_ws(W, X, Y, M, N, K, ws, Q4_0_STATIC_WS_BYTES, stream);
 }
 
+int q4_0_gather(const void *W, const int32_t *ids, float *out, int64_t T, int64_t V, int64_t D,
+                q4_0_stream_t stream) {
+    if (T < 0 || T > Q4_0_MAX_DIM || V < 0 || V > Q4_0_MAX_DIM) return Q4_ERR_INVALID_ARG;
+    int st = check_dims(V, D);
+    if (st != Q4_OK) return st;
+    if (T == 0 || D == 0) return Q4_OK;
+    if (V == 0 || !W || !ids || !out) return Q4_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(out) || (reinterpret_cast<uintptr_t>(ids) & 3u) != 0) return Q4_ERR_MISALIGNED;
+    const q4::DeviceInfo *dev = nullptr;
+    st = current_device(&dev);
+    if (st != Q4_OK) return st;
+    cudaError_t e = q4::launch_gather(static_cast<const uint8_t *>(W), ids, out, T, V, D, *dev,
+                                      reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? Q4_OK : cuda_fail(e);
+}
+
+int q4_0_quantize(const float *X, void *W, int64_t N, int64_t K, q4_0_stream_t stream) {
+    int st = check_dims(N, K);
+    if (st != Q4_OK) return st;
+    if (N == 0 || K == 0) return Q4_OK;
+    if (!X || !W) return Q4_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(W)) return Q4_ERR_MISALIGNED;
+    const q4::DeviceInfo *dev = nullptr;
+    st = current_device(&dev);
+    if (st != Q4_OK) return st;
+    cudaError_t e = q4::launch_quantize(X, static_cast<uint8_t *>(W), N, K, *dev, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? Q4_OK : cuda_fail(e);
+}
+
 int q4_0_gemm_grouped(const q4_0_problem *problems, int count, q4_0_stream_t stream) {
     if (count < 0 || count > Q4_0_MAX_GROUP) return Q4_ERR_INVALID_ARG;
     if (count == 0) return Q4_OK;

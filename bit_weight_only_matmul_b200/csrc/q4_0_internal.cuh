@@ -31,6 +31,10 @@ cudaError_t launch_pack(const uint8_t *codes, const uint16_t *scales, uint8_t *W
                         int64_t N, int64_t K, cudaStream_t s);
 cudaError_t launch_dequant(const uint8_t *W, float *out, int64_t N, int64_t K, cudaStream_t s);
 cudaError_t launch_zero(float *Y, int64_t count, cudaStream_t s);
+cudaError_t launch_gather(const uint8_t *W, const int32_t *ids, float *out, int64_t T, int64_t V, int64_t D,
+                          const DeviceInfo &dev, cudaStream_t s);
+cudaError_t launch_quantize(const float *X, uint8_t *W, int64_t N, int64_t K, const DeviceInfo &dev,
+                            cudaStream_t s);
 cudaError_t launch_generic(const Problem *probs, int count, const DeviceInfo &dev, cudaStream_t s);
 // Decode kernel on warp-level mma.sync with fp16 weights (M <= 32), the
 // default decode path: every problem must satisfy decode_mma_supports().

@@ -69,7 +69,8 @@ enum {
 
 /* Device error bits reported by q4_0_device_error. */
 enum {
-    Q4_DEVERR_WAIT_TIMEOUT = 1u    /* a bounded on-chip wait gave up; the output is incomplete */
+    Q4_DEVERR_WAIT_TIMEOUT = 1u,   /* a bounded on-chip wait gave up; the output is incomplete */
+    Q4_DEVERR_BAD_INDEX = 2u       /* q4_0_gather met an id outside [0, V) (its row was zeroed) */
 };
 
 /* Largest N, K and M accepted (each dimension below 2^31). */
@@ -173,6 +174,31 @@ Q4_0_API int q4_0_gemm_ws(const void *W, const uint16_t *X, float *Y,
  * deployment convenience of this library. */
 Q4_0_API int q4_0_gemm_static_ws(const void *W, const uint16_t *X, float *Y,
                                  int64_t M, int64_t N, int64_t K, q4_0_stream_t stream);
+
+/* Row gather (a Q4 embedding lookup): out[t, :] = dequant(W)[ids[t], :] for
+ * t < T, W a Q4_0 matrix of V rows by D weights, out float32 [T, D] row-major
+ * (exact: each (q - 8) * d is representable in float32).  The pages keep the
+ * 131072 x 3072 token embeddings of the Voxtral models in Q4 and dequantize
+ * the looked-up rows on the host (hakusoku.com story 5135, linear ops and
+ * embeddings; voxtral-mini-realtime-rs README, "WASM Constraints Solved",
+ * item 3); this is that step on the GPU.  ids: int32 device array of T
+ * entries (4-byte aligned); W and out 16-byte aligned; D % 32 == 0.  An id
+ * outside [0, V) -- which the host cannot see without a synchronisation --
+ * gives a row of zeros and sets Q4_DEVERR_BAD_INDEX in q4_0_device_error.
+ * T == 0 or D == 0 is a no-op; V must be >= 1 otherwise. */
+Q4_0_API int q4_0_gather(const void *W, const int32_t *ids, float *out,
+                         int64_t T, int64_t V, int64_t D, q4_0_stream_t stream);
+
+/* Quantize float32 weights X[N, K] (row-major, finite) to Q4_0 blocks W
+ * (N * K/32 * 18 bytes) by the GGUF Q4_0 rule that the pages apply offline
+ * (their quantize_tts_gguf.py, voxtral-mini-realtime-rs README, TTS section;
+ * the rule itself is not on the pages): per block of 32, m = the value of
+ * largest magnitude (the first on ties, +0 for an all-zero block),
+ * d = m / -8, id = 1/d (0 when d == 0), q = min(15, trunc(x * id + 8.5)) in
+ * float32 with the product rounded before the sum; the block stores fp16(d)
+ * rounded to nearest even.  Deterministic and bit-exact.  X and W 16-byte
+ * aligned, K % 32 == 0; N == 0 or K == 0 is a no-op. */
+Q4_0_API int q4_0_quantize(const float *X, void *W, int64_t N, int64_t K, q4_0_stream_t stream);
 
 /* One problem of a grouped launch: Y = X * dequant(W)^T, all device
  * pointers, same rules as q4_0_gemm. */

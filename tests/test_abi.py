@@ -111,3 +111,20 @@ def test_workspace_size_and_checks(q4):
     assert ws(A, A, A, 64, 8, 64, A + 4, 4096, None) == q4.Q4_ERR_MISALIGNED
     assert ws(A, A, A, 64, 8, 64, A, -1, None) == q4.Q4_ERR_INVALID_ARG
     assert ws(None, None, None, 0, 8, 64, None, 0, None) == q4.Q4_OK
+
+
+def test_gather_quantize_argument_checks(q4):
+    g, qz = q4.lib.q4_0_gather, q4.lib.q4_0_quantize
+    assert g(A, A, A, 4, 10, 48, None) == q4.Q4_ERR_INVALID_ARG      # D % 32
+    assert g(A, A, A, -1, 10, 64, None) == q4.Q4_ERR_INVALID_ARG     # T < 0
+    assert g(A, A, A, 4, 0, 64, None) == q4.Q4_ERR_INVALID_ARG       # no rows to gather from
+    assert g(None, A, A, 4, 10, 64, None) == q4.Q4_ERR_INVALID_ARG
+    assert g(A, None, A, 4, 10, 64, None) == q4.Q4_ERR_INVALID_ARG
+    assert g(A + 2, A, A, 4, 10, 64, None) == q4.Q4_ERR_MISALIGNED
+    assert g(A, A + 2, A, 4, 10, 64, None) == q4.Q4_ERR_MISALIGNED
+    assert g(A, A, A + 4, 4, 10, 64, None) == q4.Q4_ERR_MISALIGNED
+    assert g(None, None, None, 0, 10, 64, None) == q4.Q4_OK         # nothing to do
+    assert qz(A, A, 4, 40, None) == q4.Q4_ERR_INVALID_ARG
+    assert qz(None, A, 4, 64, None) == q4.Q4_ERR_INVALID_ARG
+    assert qz(A + 4, A, 4, 64, None) == q4.Q4_ERR_MISALIGNED
+    assert qz(None, None, 0, 64, None) == q4.Q4_OK

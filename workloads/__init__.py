@@ -199,3 +199,32 @@ def workload(name: str, layers: Optional[List[int]] = None) -> Workload:
 
 
 WORKLOADS = ["gemv", "layer", "cfg_decode", "concurrent", "adapter", "qkv_prefill"]
+
+# ---------------------------------------------------------------------------
+# the two utilities around the product (row gather, quantization)
+# ---------------------------------------------------------------------------
+
+T_IDS = 6
+T_WEIGHTS = 7
+
+EMBED_VOCAB, EMBED_DIM, EMBED_TOKENS = 131072, 3072, 4096
+QUANT_N, QUANT_K = 16384, 3072
+
+
+def gen_ids(T: int, V: int, seed: int = SEED, stream: int = 0) -> np.ndarray:
+    """int32 [T] token ids, uniform in 0..V-1."""
+    return _rng(seed, 0, T_IDS, stream).integers(0, V, size=T, dtype=np.int32)
+
+
+def gen_weights(N: int, K: int, seed: int = SEED, stream: int = 0, sigma: float = 0.02) -> np.ndarray:
+    """float32 [N, K] ~ N(0, sigma^2): unquantized weights to feed q4_0_quantize."""
+    x = _rng(seed, 0, T_WEIGHTS, stream).standard_normal(size=(N, K), dtype=np.float32)
+    x *= np.float32(sigma)
+    return x
+
+
+UTIL_WORKLOADS = {
+    "embed": (f"Q4 embedding lookup: {EMBED_TOKENS} token ids uniform over a {EMBED_VOCAB} x {EMBED_DIM} "
+              f"Q4_0 table ({EMBED_VOCAB * EMBED_DIM // 32 * 18 / 2**20:.1f} MiB), rows dequantized to fp32"),
+    "quantize": f"quantize fp32 weights [{QUANT_N}, {QUANT_K}] ~ N(0, 0.02^2) to Q4_0",
+}
