@@ -77,8 +77,11 @@ constexpr int kMaxSched = 2 * kMaxItems;            // schedule entries (a split
 constexpr uint16_t kSplitFlag = 0x8000;
 
 // NT = n8 tiles of X rows (M <= 8*NT)
-template <int NT> constexpr int raw_bytes() { return kRawW + 8 * NT * kXPitch; }
-template <int NT> constexpr int ring() { return NT == 4 ? 4 : 6; }
+template <int NT> constexpr int raw_bytes() { return kRawW + 8 * NT * kXPitch; }   // one 256-k stage
+// 256-k stages per ring slot: two for M <= 8, so that every wait, arrival and
+// walk step of every warp covers 512 k (halving that overhead per byte)
+template <int NT> constexpr int subs() { return NT == 1 ? 2 : 1; }
+template <int NT> constexpr int ring() { return NT == 2 ? 6 : 4; }   // slots
 
 // Partner sums in split mode: written remotely by CTA 1 of a cluster into
 // CTA 0's copy (two buffers, by item parity).
@@ -92,8 +95,8 @@ struct XComb<NT, false> {};
 
 template <int NT, bool SPLIT>
 struct Smem {
-    uint8_t raw[ring<NT>()][raw_bytes<NT>()];   // W rows (pitch 144) then X rows (pitch 528)
-    uint2 xf[kXBufs][16][NT][32];               // B fragments: [mma u][n tile][lane]
+    uint8_t raw[ring<NT>()][subs<NT>()][raw_bytes<NT>()];   // per stage: W rows (pitch 144), X rows (pitch 528)
+    uint2 xf[kXBufs][subs<NT>()][16][NT][32];               // B fragments: [stage][mma u][n tile][lane]
     float comb[8][NT][4][32];                   // group-1 sums handed to group 0 at an item's end
     uint64_t raw_full[ring<NT>()], raw_empty[ring<NT>()];
     uint64_t xf_full[kXBufs], xf_empty[kXBufs];
@@ -215,9 +218,9 @@ __device__ __forceinline__ bool wait_cluster_or_abort(uint64_t *bar, uint32_t pa
 // to the CTAs in boustrophedon order.  Split mode: the CTA's list from the
 // host; of a split n-stage item rank 0 takes the first ceil(n/2) stages and
 // rank 1 the rest.
-template <bool SPLIT>
+template <bool SPLIT, int SUBS>
 struct Walk {
-    int round, idx, item, prob, row0, stage, end;
+    int round, idx, item, prob, row0, stage, end, cnt;   // this step covers stages [stage, stage + cnt)
     bool split;
     template <int CAP>
     __device__ __forceinline__ void load(const DecodeParams<CAP> &D, uint32_t rank) {
@@ -243,6 +246,7 @@ struct Walk {
             end = split && rank == 0 ? n0 : n;
         }
         row0 = (item - P.p[prob].item_begin) * kItemRows;
+        cnt = SUBS == 1 || end - stage >= SUBS ? SUBS : end - stage;   // every item has >= 1 stage here
     }
     template <int CAP>
     __device__ __forceinline__ void start(const DecodeParams<CAP> &D, uint32_t rank) {
@@ -253,7 +257,11 @@ struct Walk {
     }
     template <int CAP>
     __device__ __forceinline__ void next(const DecodeParams<CAP> &D, uint32_t rank) {
-        if (++stage < end) return;
+        stage += cnt;
+        if (stage < end) {
+            cnt = SUBS == 1 || end - stage >= SUBS ? SUBS : end - stage;
+            return;
+        }
         ++round;
         ++idx;
         load(D, rank);
@@ -263,6 +271,7 @@ struct Walk {
 template <int NT, int CAP, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_constant__ DecodeParams<CAP> D) {
     constexpr int RS = ring<NT>();
+    constexpr int SUB = subs<NT>();
     const GroupParams<CAP> &P = D.g;
     extern __shared__ uint8_t smem_raw[];
     using SM = Smem<NT, SPLIT>;
@@ -300,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
 
     if (warp == kWarpProd) {
         // ---------------------------------------------------------------- loads
-        Walk<SPLIT> q{};
+        Walk<SPLIT, SUB> q{};
         q.start(D, rank);
         for (; q.item >= 0; q.next(D, rank)) {
             const GroupProblem &pr = P.p[q.prob];
@@ -309,16 +318,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
             bool ok = true;
             if (lane == 0) ok = wait_or_abort(&S.raw_empty[slot], ((g / RS) & 1) ^ 1, &S.abort_flag, P.err);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            // weights: one TMA box (rows past N are zero-filled and still counted)
+            // weights: one TMA box per stage (rows past N are zero-filled and still counted)
             if (lane == 0) {
-                mbar_arrive_expect_tx(&S.raw_full[slot], kRawW + pr.M * kXRow);
-                tma_load_2d(S.raw[slot], &P.wmap[q.prob], q.stage * kStageRowBytes, q.row0, &S.raw_full[slot]);
+                mbar_arrive_expect_tx(&S.raw_full[slot], q.cnt * (kRawW + pr.M * kXRow));
+                for (int i = 0; i < q.cnt; ++i)
+                    tma_load_2d(S.raw[slot][i], &P.wmap[q.prob], (q.stage + i) * kStageRowBytes, q.row0,
+                                &S.raw_full[slot]);
             }
             __syncwarp();
-            for (int m = lane; m < pr.M; m += 32)
-                bulk_g2s(S.raw[slot] + kRawW + m * kXPitch,
-                         pr.X + static_cast<int64_t>(m) * pr.K + static_cast<int64_t>(q.stage) * kStageK, kXRow,
-                         &S.raw_full[slot]);
+            for (int i = 0; i < q.cnt; ++i)
+                for (int m = lane; m < pr.M; m += 32)
+                    bulk_g2s(S.raw[slot][i] + kRawW + m * kXPitch,
+                             pr.X + static_cast<int64_t>(m) * pr.K + static_cast<int64_t>(q.stage + i) * kStageK,
+                             kXRow, &S.raw_full[slot]);
             ++prod_issued;
         }
     } else if (warp < kWarp0) {
@@ -330,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
         const int G = warp - kWarpX0;
         const int gx = lane >> 2, tx = lane & 3;
         uint32_t g = 0;
-        Walk<SPLIT> q{};
+        Walk<SPLIT, SUB> q{};
         q.start(D, rank);
         for (; q.item >= 0; q.next(D, rank), ++g) {
             if ((g & 1) != static_cast<uint32_t>(G)) continue;
@@ -342,24 +354,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
                 if (ok) ok = wait_or_abort(&S.xf_empty[xb], ((g / kXBufs) & 1) ^ 1, &S.abort_flag, P.err);
             }
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            const uint8_t *xr = S.raw[slot] + kRawW;
             #pragma unroll
-            for (int j = 0; j < NT; ++j) {
-                const int m = 8 * j + gx;
+            for (int i = 0; i < SUB; ++i) {
+                if (i >= q.cnt) break;
+                const uint8_t *xr = S.raw[slot][i] + kRawW;
                 #pragma unroll
-                for (int xw = 0; xw < 2; ++xw)
+                for (int j = 0; j < NT; ++j) {
+                    const int m = 8 * j + gx;
                     #pragma unroll
-                    for (int h = 0; h < 2; ++h)
+                    for (int xw = 0; xw < 2; ++xw)
                         #pragma unroll
-                        for (int wp = 0; wp < 2; ++wp) {
-                            uint4 o = make_uint4(0u, 0u, 0u, 0u);
-                            if (m < pr.M) {
-                                const int k = 32 * (2 * tx + xw) + 16 * h + 8 * wp;
-                                o = x8_to_fp16_permuted(*reinterpret_cast<const uint4 *>(xr + m * kXPitch + 2 * k));
+                        for (int h = 0; h < 2; ++h)
+                            #pragma unroll
+                            for (int wp = 0; wp < 2; ++wp) {
+                                uint4 o = make_uint4(0u, 0u, 0u, 0u);
+                                if (m < pr.M) {
+                                    const int k = 32 * (2 * tx + xw) + 16 * h + 8 * wp;
+                                    o = x8_to_fp16_permuted(
+                                        *reinterpret_cast<const uint4 *>(xr + m * kXPitch + 2 * k));
+                                }
+                                S.xf[xb][i][8 * xw + 4 * wp + h][j][lane] = make_uint2(o.x, o.y);
+                                S.xf[xb][i][8 * xw + 4 * wp + 2 + h][j][lane] = make_uint2(o.z, o.w);
                             }
-                            S.xf[xb][8 * xw + 4 * wp + h][j][lane] = make_uint2(o.x, o.y);
-                            S.xf[xb][8 * xw + 4 * wp + 2 + h][j][lane] = make_uint2(o.z, o.w);
-                        }
+                }
             }
             __syncwarp();
             if (lane == 0) {
@@ -378,31 +395,39 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
             #pragma unroll
             for (int j = 0; j < NT; ++j) acc[c][j][0] = acc[c][j][1] = acc[c][j][2] = acc[c][j][3] = 0.f;
         uint32_t g = 0, items_done = 0, split_done = 0;
-        Walk<SPLIT> q{};
+        Walk<SPLIT, SUB> q{};
         q.start(D, rank);
         for (; q.item >= 0; q.next(D, rank), ++g) {
             if ((g & 1) == static_cast<uint32_t>(G)) {
                 const int slot = g % RS, xb = g % kXBufs;
                 if (!wait_or_abort(&S.raw_full[slot], (g / RS) & 1, &S.abort_flag, P.err)) break;
-                const uint8_t *rowg = S.raw[slot] + (16 * tile + gq) * kStageRowBytes;
-                uint32_t rg[9], rg8[9];
-                load_blocks(rowg, t, rg);
-                load_blocks(rowg + 8 * kStageRowBytes, t, rg8);
+                uint32_t rg[SUB][9], rg8[SUB][9];
+                #pragma unroll
+                for (int i = 0; i < SUB; ++i) {
+                    if (i >= q.cnt) break;
+                    const uint8_t *rowg = S.raw[slot][i] + (16 * tile + gq) * kStageRowBytes;
+                    load_blocks(rowg, t, rg[i]);
+                    load_blocks(rowg + 8 * kStageRowBytes, t, rg8[i]);
+                }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.raw_empty[slot]);
                 if (!wait_or_abort(&S.xf_full[xb], (g / kXBufs) & 1, &S.abort_flag, P.err)) break;
-                word_mma<NT, 0, 0>(rg, rg8, S.xf[xb], lane, acc);
-                word_mma<NT, 0, 1>(rg, rg8, S.xf[xb], lane, acc);
-                word_mma<NT, 0, 2>(rg, rg8, S.xf[xb], lane, acc);
-                word_mma<NT, 0, 3>(rg, rg8, S.xf[xb], lane, acc);
-                word_mma<NT, 1, 0>(rg, rg8, S.xf[xb], lane, acc);
-                word_mma<NT, 1, 1>(rg, rg8, S.xf[xb], lane, acc);
-                word_mma<NT, 1, 2>(rg, rg8, S.xf[xb], lane, acc);
-                word_mma<NT, 1, 3>(rg, rg8, S.xf[xb], lane, acc);
+                #pragma unroll
+                for (int i = 0; i < SUB; ++i) {
+                    if (i >= q.cnt) break;
+                    word_mma<NT, 0, 0>(rg[i], rg8[i], S.xf[xb][i], lane, acc);
+                    word_mma<NT, 0, 1>(rg[i], rg8[i], S.xf[xb][i], lane, acc);
+                    word_mma<NT, 0, 2>(rg[i], rg8[i], S.xf[xb][i], lane, acc);
+                    word_mma<NT, 0, 3>(rg[i], rg8[i], S.xf[xb][i], lane, acc);
+                    word_mma<NT, 1, 0>(rg[i], rg8[i], S.xf[xb][i], lane, acc);
+                    word_mma<NT, 1, 1>(rg[i], rg8[i], S.xf[xb][i], lane, acc);
+                    word_mma<NT, 1, 2>(rg[i], rg8[i], S.xf[xb][i], lane, acc);
+                    word_mma<NT, 1, 3>(rg[i], rg8[i], S.xf[xb][i], lane, acc);
+                }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.xf_empty[xb]);
             }
-            if (q.stage == q.end - 1) {
+            if (q.stage + q.cnt == q.end) {
                 // end of the item: the two groups add their sums
                 const GroupProblem &pr = P.p[q.prob];
                 const uint32_t par = items_done & 1;
@@ -487,6 +512,7 @@ template <int NT, bool SPLIT>
 constexpr size_t smem_bytes() { return sizeof(Smem<NT, SPLIT>) + 128; }
 static_assert(smem_bytes<4, false>() <= 232448, "shared memory budget");
 static_assert(smem_bytes<1, true>() <= 232448, "shared memory budget");
+static_assert(smem_bytes<2, false>() <= 232448, "shared memory budget");
 
 template <int NT, int CAP, bool SPLIT>
 cudaError_t configure(const q4::DeviceInfo &dev) {
