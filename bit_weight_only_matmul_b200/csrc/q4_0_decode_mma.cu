@@ -28,6 +28,9 @@
 //    pairs and feeds them as A fragments of 16 mma.sync per stage: with the
 //    scale folded into each weight, one MMA may mix blocks, so every byte a
 //    thread loads is its own;
+//  * for M > 8 the stage's X rows come as four TMA boxes (64 k x 8*NT rows,
+//    128-byte swizzle, rows past M zero-filled) instead of one 1-D copy per
+//    row: 32 copies per stage would cap the stream near 2.2 TB/s;
 //  * the X warps convert the stage's X rows to fp16 straight into the
 //    matching mma.sync B fragments (two buffers per group), one 8-byte shared
 //    load per fragment for the compute threads;
@@ -77,7 +80,12 @@ constexpr int kMaxSched = 2 * kMaxItems;            // schedule entries (a split
 constexpr uint16_t kSplitFlag = 0x8000;
 
 // NT = n8 tiles of X rows (M <= 8*NT)
-template <int NT> constexpr int raw_bytes() { return kRawW + 8 * NT * kXPitch; }   // one 256-k stage
+// X by TMA boxes (M > 8): four boxes of 64 k x 8*NT rows, 128 bytes a row
+template <int NT> constexpr bool xmap() { return NT >= 2; }
+template <int NT> constexpr int xbox_bytes() { return 8 * NT * 128; }
+template <int NT> constexpr int raw_bytes() {   // one 256-k stage
+    return kRawW + (xmap<NT>() ? 4 * xbox_bytes<NT>() : 8 * NT * kXPitch);
+}
 // 256-k stages per ring slot: two for M <= 8, so that every wait, arrival and
 // walk step of every warp covers 512 k (halving that overhead per byte)
 template <int NT> constexpr int subs() { return NT == 1 ? 2 : 1; }
@@ -154,9 +162,12 @@ __device__ __forceinline__ void word_mma(const uint32_t (&rg)[9], const uint32_t
     }
 }
 
+constexpr int kXMapCap = 64;   // problems per launch when X maps are passed (M > 8)
+
 template <int CAP>
 struct DecodeParams {
     GroupParams<CAP> g;
+    CUtensorMap xmap[CAP <= kXMapCap ? CAP : 1];   // M > 8: X as bf16 [M, K], box 64 x 8*NT, 128-byte swizzle
     // split mode: CTA b runs sched[sched_begin[b] .. sched_begin[b+1]), each
     // entry an item index, with kSplitFlag set for a half of a split item
     uint16_t sched_begin[kMaxSplitCtas + 1];
@@ -275,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
     const GroupParams<CAP> &P = D.g;
     extern __shared__ uint8_t smem_raw[];
     using SM = Smem<NT, SPLIT>;
-    SM &S = *reinterpret_cast<SM *>(align_smem<128>(smem_raw));
+    SM &S = *reinterpret_cast<SM *>(align_smem<1024>(smem_raw));   // swizzled X boxes want 1024
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -319,18 +330,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
             if (lane == 0) ok = wait_or_abort(&S.raw_empty[slot], ((g / RS) & 1) ^ 1, &S.abort_flag, P.err);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             // weights: one TMA box per stage (rows past N are zero-filled and still counted)
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&S.raw_full[slot], q.cnt * (kRawW + pr.M * kXRow));
+            if constexpr (xmap<NT>()) {
+                if (lane == 0) {
+                    // full boxes are counted, zero-filled rows included
+                    mbar_arrive_expect_tx(&S.raw_full[slot], q.cnt * (kRawW + 4 * xbox_bytes<NT>()));
+                    for (int i = 0; i < q.cnt; ++i) {
+                        tma_load_2d(S.raw[slot][i], &P.wmap[q.prob], (q.stage + i) * kStageRowBytes, q.row0,
+                                    &S.raw_full[slot]);
+                        for (int b = 0; b < 4; ++b)
+                            tma_load_2d(S.raw[slot][i] + kRawW + b * xbox_bytes<NT>(), &D.xmap[q.prob],
+                                        (q.stage + i) * kStageK + 64 * b, 0, &S.raw_full[slot]);
+                    }
+                }
+            } else {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&S.raw_full[slot], q.cnt * (kRawW + pr.M * kXRow));
+                    for (int i = 0; i < q.cnt; ++i)
+                        tma_load_2d(S.raw[slot][i], &P.wmap[q.prob], (q.stage + i) * kStageRowBytes, q.row0,
+                                    &S.raw_full[slot]);
+                }
+                __syncwarp();
                 for (int i = 0; i < q.cnt; ++i)
-                    tma_load_2d(S.raw[slot][i], &P.wmap[q.prob], (q.stage + i) * kStageRowBytes, q.row0,
-                                &S.raw_full[slot]);
+                    for (int m = lane; m < pr.M; m += 32)
+                        bulk_g2s(S.raw[slot][i] + kRawW + m * kXPitch,
+                                 pr.X + static_cast<int64_t>(m) * pr.K + static_cast<int64_t>(q.stage + i) * kStageK,
+                                 kXRow, &S.raw_full[slot]);
             }
-            __syncwarp();
-            for (int i = 0; i < q.cnt; ++i)
-                for (int m = lane; m < pr.M; m += 32)
-                    bulk_g2s(S.raw[slot][i] + kRawW + m * kXPitch,
-                             pr.X + static_cast<int64_t>(m) * pr.K + static_cast<int64_t>(q.stage + i) * kStageK,
-                             kXRow, &S.raw_full[slot]);
             ++prod_issued;
         }
     } else if (warp < kWarp0) {
@@ -370,8 +395,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
                                 uint4 o = make_uint4(0u, 0u, 0u, 0u);
                                 if (m < pr.M) {
                                     const int k = 32 * (2 * tx + xw) + 16 * h + 8 * wp;
-                                    o = x8_to_fp16_permuted(
-                                        *reinterpret_cast<const uint4 *>(xr + m * kXPitch + 2 * k));
+                                    // box tx holds k 64tx..64tx+63; its 16-byte chunk c of row m
+                                    // sits at chunk c ^ (m & 7) (128-byte swizzle)
+                                    const uint8_t *src =
+                                        xmap<NT>() ? xr + tx * xbox_bytes<NT>() + m * 128 +
+                                                         ((((k & 63) >> 3) ^ (m & 7)) << 4)
+                                                   : xr + m * kXPitch + 2 * k;
+                                    o = x8_to_fp16_permuted(*reinterpret_cast<const uint4 *>(src));
                                 }
                                 S.xf[xb][i][8 * xw + 4 * wp + h][j][lane] = make_uint2(o.x, o.y);
                                 S.xf[xb][i][8 * xw + 4 * wp + 2 + h][j][lane] = make_uint2(o.z, o.w);
@@ -509,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
 }
 
 template <int NT, bool SPLIT>
-constexpr size_t smem_bytes() { return sizeof(Smem<NT, SPLIT>) + 128; }
+constexpr size_t smem_bytes() { return sizeof(Smem<NT, SPLIT>) + 1024; }
 static_assert(smem_bytes<4, false>() <= 232448, "shared memory budget");
 static_assert(smem_bytes<1, true>() <= 232448, "shared memory budget");
 static_assert(smem_bytes<2, false>() <= 232448, "shared memory budget");
@@ -672,7 +702,20 @@ cudaError_t launch_cap(const q4::Problem *probs, const int *order, int count, co
             return cudaErrorInvalidValue;
     }
     P.total_items = items;
-    if (maxM <= 8) {
+    if (maxM > 8) {
+        if constexpr (CAP <= kXMapCap) {
+            for (int i = 0; i < count; ++i) {
+                const q4::Problem &q = probs[order[i]];
+                if (!q4::get_tensor_map(&D.xmap[i], q.X, q.M, q.K, maxM <= 16 ? q4::kMapXDecode16 : q4::kMapXDecode32))
+                    return cudaErrorInvalidValue;
+            }
+            if (maxM <= 16) return launch_plain<2, CAP>(D, dev, s);
+            return launch_plain<4, CAP>(D, dev, s);
+        } else {
+            return cudaErrorInvalidValue;   // the caller sends M > 8 groups in chunks of kXMapCap
+        }
+    }
+    {
         // fewer items than SMs: each CTA has at most one item and the launch is
         // latency-bound, where the hand-over between a pair costs more than it
         // saves (measured on a single 3072 x 3072 GEMV)
@@ -682,8 +725,6 @@ cudaError_t launch_cap(const q4::Problem *probs, const int *order, int count, co
         }
         return launch_plain<1, CAP>(D, dev, s);
     }
-    if (maxM <= 16) return launch_plain<2, CAP>(D, dev, s);
-    return launch_plain<4, CAP>(D, dev, s);
 }
 
 constexpr int kSmallCap = 8, kLargeCap = 128;
@@ -704,10 +745,14 @@ cudaError_t launch_decode_mma(const Problem *probs, int count, const DeviceInfo 
     order.resize(count);
     for (int i = 0; i < count; ++i) order[i] = i;
     std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return probs[a].K > probs[b].K; });
+    int64_t maxM = 1;
+    for (int i = 0; i < count; ++i) maxM = std::max(maxM, probs[i].M);
+    const int cap = maxM > 8 ? kXMapCap : kLargeCap;   // X maps for M > 8 take parameter space
     for (int done = 0; done < count;) {
-        const int n = std::min(count - done, kLargeCap);
+        const int n = std::min(count - done, cap);
         cudaError_t e = n <= kSmallCap ? launch_cap<kSmallCap>(probs, order.data() + done, n, dev, s)
-                                       : launch_cap<kLargeCap>(probs, order.data() + done, n, dev, s);
+                        : cap == kXMapCap ? launch_cap<kXMapCap>(probs, order.data() + done, n, dev, s)
+                                          : launch_cap<kLargeCap>(probs, order.data() + done, n, dev, s);
         if (e != cudaSuccess) return e;
         done += n;
     }

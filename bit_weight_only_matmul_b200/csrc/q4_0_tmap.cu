@@ -59,11 +59,14 @@ bool encode(CUtensorMap *out, const Key &k) {
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
     }
-    if (k.kind == q4::kMapActivationsSw128 || k.kind == q4::kMapActivationsF16Sw128) {
-        // bf16 or fp16 [rows = M, cols = K], box 64 x 256, 128-byte swizzle
+    if (k.kind == q4::kMapActivationsSw128 || k.kind == q4::kMapActivationsF16Sw128 ||
+        k.kind == q4::kMapXDecode16 || k.kind == q4::kMapXDecode32) {
+        // bf16 or fp16 [rows = M, cols = K], box 64 x (256, 16 or 32), 128-byte swizzle; rows
+        // past M read as zero
         const cuuint64_t dims[2] = {static_cast<cuuint64_t>(k.cols), static_cast<cuuint64_t>(k.rows)};
         const cuuint64_t strides[1] = {static_cast<cuuint64_t>(k.cols) * 2};
-        const cuuint32_t box[2] = {64, 256};
+        const cuuint32_t rows = k.kind == q4::kMapXDecode16 ? 16 : k.kind == q4::kMapXDecode32 ? 32 : 256;
+        const cuuint32_t box[2] = {64, rows};
         const CUtensorMapDataType t = k.kind == q4::kMapActivationsSw128 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                                          : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
         return enc(out, t, 2, const_cast<void *>(k.ptr), dims, strides, box, estr,
