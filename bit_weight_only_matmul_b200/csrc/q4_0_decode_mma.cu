@@ -316,6 +316,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
     } else {
         __syncthreads();
     }
+    // Programmatic dependent launch: the next kernel on the stream may start
+    // its CTAs as this grid's CTAs leave the SMs, and this grid touches no
+    // global memory before the previous kernel on the stream has completed
+    // (both are no-ops for launches without the attribute).
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     uint32_t prod_issued = 0;
 
     if (warp == kWarpProd) {
@@ -560,8 +566,17 @@ cudaError_t launch_plain(DecodeParams<CAP> &D, const q4::DeviceInfo &dev, cudaSt
     cudaError_t e = configure<NT, CAP, false>(dev);
     if (e != cudaSuccess) return e;
     const int grid = std::max(1, std::min(dev.sm_count, D.g.total_items));
-    decode_mma_kernel<NT, CAP, false><<<grid, kThreads, smem_bytes<NT, false>(), s>>>(D);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem_bytes<NT, false>();
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_mma_kernel<NT, CAP, false>, D);
 }
 
 cudaLaunchConfig_t cluster_config(int clusters, cudaStream_t s, cudaLaunchAttribute *attr) {
@@ -574,8 +589,10 @@ cudaLaunchConfig_t cluster_config(int clusters, cudaStream_t s, cudaLaunchAttrib
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cfg;
 }
 
@@ -586,7 +603,7 @@ int split_clusters(const q4::DeviceInfo &dev) {
     if (cached_device == dev.device) return cached;
     int n = 0;
     if (configure<1, CAP, true>(dev) == cudaSuccess) {
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         cudaLaunchConfig_t cfg = cluster_config(std::max(1, dev.sm_count / 2), nullptr, attr);
         if (cudaOccupancyMaxActiveClusters(&n, decode_mma_kernel<1, CAP, true>, &cfg) != cudaSuccess) n = 0;
     }
@@ -670,7 +687,7 @@ cudaError_t launch_split(DecodeParams<CAP> &D, int clusters, cudaStream_t s) {
         build_schedule(D, clusters);
         last = sig;
     }
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = cluster_config(clusters, s, attr);
     return cudaLaunchKernelEx(&cfg, decode_mma_kernel<1, CAP, true>, D);
 }
