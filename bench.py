@@ -12,7 +12,9 @@ step, so every step streams its weights from HBM.
 
 The metric is effective HBM bandwidth: algorithmic bytes (every Q4_0 weight
 byte once + X and Y once) / time.  Other workloads (--workload): gemv, layer,
-cfg_decode (M=2, 26 layers), concurrent (M=32, 26 layers) in GB/s; adapter,
+cfg_decode (M=2, 26 layers), concurrent (M=32, 26 layers), flow_head (M=2,
+one Euler step of the 3-layer flow head) in GB/s; embed, quantize (the row
+gather and the quantizer) in GB/s; adapter,
 qkv_prefill (M=4096) in TFLOP/s.
 
 N > 1 (torchrun, one process per GPU): every rank runs an independent
@@ -52,6 +54,7 @@ DOMINANT = {
     "layer": ("decode_mma_kernel", "q4_0_decode_mma.cu"),
     "cfg_decode": ("decode_mma_kernel", "q4_0_decode_mma.cu"),
     "concurrent": ("decode_mma_kernel", "q4_0_decode_mma.cu"),
+    "flow_head": ("decode_mma_kernel", "q4_0_decode_mma.cu"),
     "adapter": ("prefill_kernel", "q4_0_prefill.cu"),
     "qkv_prefill": ("prefill_kernel", "q4_0_prefill.cu"),
 }

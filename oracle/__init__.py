@@ -73,6 +73,8 @@ class Oracle:
         L.oracle_float_to_half.argtypes = [ctypes.c_float]
         L.oracle_q4_0_quantize.restype = None
         L.oracle_q4_0_quantize.argtypes = [_p, _p, _i64, _i64]
+        L.oracle_swiglu.restype = None
+        L.oracle_swiglu.argtypes = [_p, _p, _p, _i64]
 
     # -- scalar decoders -------------------------------------------------
     def half_to_double(self, h: int) -> float:
@@ -170,6 +172,17 @@ class Oracle:
         W = np.empty((N, K // 32 * 18), np.uint8)
         self._lib.oracle_q4_0_quantize(X.ctypes.data, W.ctypes.data, N, K)
         return W
+
+
+    def swiglu(self, g: np.ndarray, u: np.ndarray) -> np.ndarray:
+        """silu(g) * u elementwise in float64 (same shapes)."""
+        g = self._c(g, np.float64)
+        u = self._c(u, np.float64)
+        if g.shape != u.shape:
+            raise ValueError("g and u differ in shape")
+        out = np.empty(g.shape, np.float64)
+        self._lib.oracle_swiglu(g.ctypes.data, u.ctypes.data, out.ctypes.data, g.size)
+        return out
 
 
 _default = None

@@ -29,8 +29,17 @@
  *
  * Every product (q-8)*d*x is exact in float64 (4 + 11 + 8 significant bits).
  *
- * Two more operations around the product (the next steps the survey ranks,
- * not the hot path itself):
+ * Operations around the product (the next steps the survey ranks, not the
+ * hot path itself):
+ *   swiglu   -- the activation between the fused gate/up projection and the
+ *               down projection of a decoder layer's feed-forward block:
+ *               out = silu(g) * u with silu(g) = g / (1 + exp(-g)), in
+ *               float64 (the pages name the fused gate/up projection,
+ *               voxtral-mini-realtime-rs (Shannon-Prime fork) README, TTS
+ *               section, optimizations; the SwiGLU form of the Mistral-family
+ *               feed-forward block is the reading taken, not printed there);
+ *   residual -- Y + R, the residual connection after the O and down
+ *               projections (same reading);
  *   gather   -- rows ids[t] of a Q4_0 matrix W[V, D] dequantized to float32:
  *               the Q4 embedding lookup the pages run on the CPU instead of
  *               keeping a 1.5 GiB fp32 table (hakusoku.com story 5135, linear
@@ -336,5 +345,18 @@ void oracle_q4_0_quantize(const float *X, uint8_t *W, int64_t N, int64_t K)
             for (int j = 0; j < 16; j++)
                 blk[2 + j] = (uint8_t)((q[j] & 0x0f) | ((q[j + 16] & 0x0f) << 4));
         }
+    }
+}
+
+/* out[i] = silu(g[i]) * u[i], silu(g) = g / (1 + exp(-g)), float64. */
+void oracle_swiglu(const double *g, const double *u, double *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; i++) {
+#if ORACLE_MUTANT == 11
+        double s = g[i] / (1.0 + exp(g[i])); /* planted: wrong sign in the exponent */
+#else
+        double s = g[i] / (1.0 + exp(-g[i]));
+#endif
+        out[i] = s * u[i];
     }
 }

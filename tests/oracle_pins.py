@@ -23,6 +23,9 @@ What each pin is tied to:
     its reconstruction, symmetry under negation and power-of-two scaling);
   * gather: equals the pinned dequantization row by row, zero rows for ids
     out of range;
+  * swiglu: closed forms of silu (silu(0) = 0, silu(x) - silu(-x) = x,
+    silu(1) = e/(1+e) from math.exp, silu(x) -> x and -> 0 at the ends) and
+    the product with u;
   * sizes: 4.5 bits per weight, cross-checked with the pages' 1.5 GiB fp32
     embedding table that becomes 216 MB in Q4 (hakusoku.com story 5135,
     linear ops and embeddings; voxtral-mini-realtime-rs README, "WASM
@@ -360,6 +363,19 @@ def pin_gather_matches_dequant(o):
     assert not out[[0, 2, 3]].any()
 
 
+def pin_swiglu_closed_forms(o):
+    g = np.array([0.0, 1.0, -1.0, 2.5, -2.5, 40.0, -40.0, 1e-9])
+    u = np.array([3.0, 1.0, 1.0, 1.0, 1.0, 1.0, 1.0, 1.0])
+    out = o.swiglu(g, u)
+    assert out[0] == 0.0
+    assert abs(out[1] - math.e / (1 + math.e)) <= 1e-15
+    assert abs(out[1] - out[2] - 1.0) <= 1e-15 and abs(out[3] - out[4] - 2.5) <= 1e-15
+    assert abs(out[5] - 40.0) <= 1e-12 and abs(out[6]) <= 1e-15
+    assert abs(out[7] - 0.5e-9) <= 1e-18          # silu(e) = e/2 + e^2/4 + ...
+    gg = np.linspace(-8, 8, 33)
+    assert np.allclose(o.swiglu(gg, np.full(33, -2.0)), -2.0 * o.swiglu(gg, np.ones(33)), rtol=0, atol=0)
+
+
 ALL_PINS = [
     pin_half_decoder,
     pin_bf16_decoder,
@@ -378,4 +394,5 @@ ALL_PINS = [
     pin_quantize_rounding_bound,
     pin_quantize_sign_and_scale,
     pin_gather_matches_dequant,
+    pin_swiglu_closed_forms,
 ]

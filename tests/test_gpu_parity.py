@@ -236,7 +236,7 @@ def test_forced_warp_mma_decode(q4, M, N, K):
     run_gemm(q4, M, N, K, path=q4.PATH_DECODE_EXACT)
 
 
-@pytest.mark.parametrize("name,layers", [("cfg_decode", [0, 13, 25]), ("concurrent", [0, 25])])
+@pytest.mark.parametrize("name,layers", [("cfg_decode", [0, 13, 25]), ("concurrent", [0, 25]), ("flow_head", None)])
 def test_decode_workloads_sampled(q4, name, layers):
     b = build_workload(q4, workloads.workload(name, layers=layers), samples=400)
     q4.q4_0_gemm_grouped(b.problems())

@@ -28,6 +28,7 @@ MUTANTS = {
     8: "quantization scale with the wrong sign",
     9: "quantization takes the last of equal extreme magnitudes",
     10: "quantization truncates instead of rounding",
+    11: "silu with the wrong sign in the exponent",
 }
 
 

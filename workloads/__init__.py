@@ -139,6 +139,8 @@ N_LAYERS = 26
 FFN = 8192
 Q_DIM, KV_DIM = 3072, 1024
 ADAPTER_IN = 5120
+FLOW_LAYERS = 3
+FLOW_LAYER0 = 100   # stream ids of the flow head's layers, apart from the decoder's
 
 
 def decoder_layer(layer: int, M: int, **xkw) -> List[Linear]:
@@ -189,6 +191,14 @@ def workload(name: str, layers: Optional[List[int]] = None) -> Workload:
         ls = range(N_LAYERS) if layers is None else layers
         return Workload(name, "concurrent decode, M=32, 26 stacked layers, 3 of 32 X rows x8",
                         [l for i in ls for l in decoder_layer(i, 32, outlier_rows=3)])
+    if name == "flow_head":
+        # the flow-matching head: 3 transformer layers run once per Euler step
+        # on the batch-2 CFG rows (the pages give no width for it; reading:
+        # the decoder's linear shapes, since it consumes the decoder's hidden
+        # states); one step = one Euler step = the 3 layers' 12 GEMMs
+        ls = range(FLOW_LAYERS) if layers is None else layers
+        return Workload(name, "flow-head Euler step, M=2 (CFG), 3 layers of the decoder linear set",
+                        [l for i in ls for l in decoder_layer(FLOW_LAYER0 + i, 2, row_scale=True)])
     if name == "adapter":
         return Workload(name, "adapter/prefill GEMM M=4096, K=5120, N=3072, X ~ N(0, 0.5^2)",
                         [Linear("adapter", D_MODEL, ADAPTER_IN, 0, 0, 4096, sigma=0.5)])
@@ -198,7 +208,7 @@ def workload(name: str, layers: Optional[List[int]] = None) -> Workload:
     raise KeyError(name)
 
 
-WORKLOADS = ["gemv", "layer", "cfg_decode", "concurrent", "adapter", "qkv_prefill"]
+WORKLOADS = ["gemv", "layer", "cfg_decode", "concurrent", "flow_head", "adapter", "qkv_prefill"]
 
 # ---------------------------------------------------------------------------
 # the two utilities around the product (row gather, quantization)
