@@ -29,6 +29,7 @@ Q4_DEVERR_BAD_INDEX = 2
 
 Q4_0_MAX_GROUP = 256
 Q4_0_STATIC_WS_BYTES = 64 << 20
+Q4_0_EPI_NONE, Q4_0_EPI_RESIDUAL, Q4_0_EPI_SWIGLU = 0, 1, 2
 
 PATH_AUTO, PATH_GENERIC, PATH_DECODE, PATH_TENSOR, PATH_DECODE_EXACT, PATH_DECODE_TMEM = 0, 1, 2, 3, 4, 5
 
@@ -44,6 +45,8 @@ EXPORTS = (
     "q4_0_gemm_ws",
     "q4_0_gemm_static_ws",
     "q4_0_gemm_grouped",
+    "q4_0_gemm_grouped_ex",
+    "q4_0_interleave_gate_up",
     "q4_0_gather",
     "q4_0_quantize",
     "q4_0_device_error",
@@ -65,6 +68,12 @@ class q4_0_problem(ctypes.Structure):
                 ("M", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
 
 
+class q4_0_problem_ex(ctypes.Structure):
+    _fields_ = [("W", ctypes.c_void_p), ("X", ctypes.c_void_p), ("Y", ctypes.c_void_p),
+                ("M", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("R", ctypes.c_void_p), ("epilogue", ctypes.c_int32)]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with `python bit_weight_only_matmul_b200/build.py`")
@@ -81,6 +90,8 @@ def _load() -> ctypes.CDLL:
         "q4_0_gemm_ws": (i32, [vp, vp, vp, i64, i64, i64, vp, i64, vp]),
         "q4_0_gemm_static_ws": (i32, [vp, vp, vp, i64, i64, i64, vp]),
         "q4_0_gemm_grouped": (i32, [ctypes.POINTER(q4_0_problem), i32, vp]),
+        "q4_0_gemm_grouped_ex": (i32, [ctypes.POINTER(q4_0_problem_ex), i32, vp]),
+        "q4_0_interleave_gate_up": (i32, [vp, vp, vp, i64, i64, vp]),
         "q4_0_gather": (i32, [vp, vp, vp, i64, i64, i64, vp]),
         "q4_0_quantize": (i32, [vp, vp, i64, i64, vp]),
         "q4_0_device_error": (i32, [ctypes.POINTER(ctypes.c_uint32), i32]),
@@ -179,6 +190,29 @@ def q4_0_gemm_grouped(problems, count: Optional[int] = None, stream=None) -> Non
     elif count is None:
         count = len(problems)
     _check(_lib.q4_0_gemm_grouped(problems, count, _stream(stream)), "q4_0_gemm_grouped")
+
+
+def make_problems_ex(problems: Sequence) -> ctypes.Array:
+    """Build a q4_0_problem_ex array from (W, X, Y, M, N, K, R, epilogue) tuples."""
+    arr = (q4_0_problem_ex * max(1, len(problems)))()
+    for i, (W, X, Y, M, N, K, R, epi) in enumerate(problems):
+        arr[i] = q4_0_problem_ex(_ptr(W), _ptr(X), _ptr(Y), M, N, K, _ptr(R), epi)
+    return arr
+
+
+def q4_0_gemm_grouped_ex(problems, count: Optional[int] = None, stream=None) -> None:
+    """`problems`: a q4_0_problem_ex array or (W, X, Y, M, N, K, R, epilogue) tuples."""
+    if not isinstance(problems, ctypes.Array):
+        count = len(problems)
+        problems = make_problems_ex(problems)
+    elif count is None:
+        count = len(problems)
+    _check(_lib.q4_0_gemm_grouped_ex(problems, count, _stream(stream)), "q4_0_gemm_grouped_ex")
+
+
+def q4_0_interleave_gate_up(W_gate, W_up, W_gu, F: int, K: int, stream=None) -> None:
+    _check(_lib.q4_0_interleave_gate_up(_ptr(W_gate), _ptr(W_up), _ptr(W_gu), F, K, _stream(stream)),
+           "q4_0_interleave_gate_up")
 
 
 def q4_0_gather(W, ids, out, T: int, V: int, D: int, stream=None) -> None:

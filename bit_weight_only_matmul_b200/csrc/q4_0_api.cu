@@ -258,6 +258,55 @@ int q4_0_quantize(const float *X, void *W, int64_t N, int64_t K, q4_0_stream_t s
     return e == cudaSuccess ? Q4_OK : cuda_fail(e);
 }
 
+int q4_0_gemm_grouped_ex(const q4_0_problem_ex *problems, int count, q4_0_stream_t stream) {
+    if (count < 0 || count > Q4_0_MAX_GROUP || (count > 0 && !problems)) return Q4_ERR_INVALID_ARG;
+    if (count == 0) return Q4_OK;
+    static thread_local std::vector<q4::Problem> dec;
+    dec.clear();
+    for (int i = 0; i < count; ++i) {
+        const q4_0_problem_ex &a = problems[i];
+        const q4_0_problem base{a.W, a.X, a.Y, a.M, a.N, a.K};
+        int st = check_problem(base);
+        if (st != Q4_OK) return st;
+        if (a.M < 1 || a.M > 32 || a.N < 1 || a.K < 256 || a.K % 256 != 0) return Q4_ERR_INVALID_ARG;
+        if (a.epilogue == Q4_0_EPI_RESIDUAL) {
+            if (!a.R) return Q4_ERR_INVALID_ARG;
+            if (!aligned16(a.R)) return Q4_ERR_MISALIGNED;
+        } else if (a.epilogue == Q4_0_EPI_SWIGLU) {
+            if (a.N % 128 != 0) return Q4_ERR_INVALID_ARG;
+        } else if (a.epilogue != Q4_0_EPI_NONE) {
+            return Q4_ERR_INVALID_ARG;
+        }
+        q4::Problem p{static_cast<const uint8_t *>(a.W), a.X, a.Y, a.M, a.N, a.K};
+        p.R = a.epilogue == Q4_0_EPI_RESIDUAL ? a.R : nullptr;
+        p.epi = a.epilogue;
+        dec.push_back(p);
+    }
+    const q4::DeviceInfo *dev = nullptr;
+    int st = current_device(&dev);
+    if (st != Q4_OK) return st;
+    for (const q4::Problem &p : dec)
+        if (!q4::decode_mma_supports(p)) return Q4_ERR_INVALID_ARG;
+    const cudaError_t e = q4::launch_decode_mma(dec.data(), count, *dev, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? Q4_OK : cuda_fail(e);
+}
+
+int q4_0_interleave_gate_up(const void *W_gate, const void *W_up, void *W_gu, int64_t F, int64_t K,
+                            q4_0_stream_t stream) {
+    int st = check_dims(2 * F, K);
+    if (st != Q4_OK || F < 0 || F % 64 != 0 || K % 256 != 0) return Q4_ERR_INVALID_ARG;
+    if (F == 0 || K == 0) return Q4_OK;
+    if (!W_gate || !W_up || !W_gu) return Q4_ERR_INVALID_ARG;
+    if (!aligned16(W_gate) || !aligned16(W_up) || !aligned16(W_gu)) return Q4_ERR_MISALIGNED;
+    const q4::DeviceInfo *dev = nullptr;
+    st = current_device(&dev);
+    if (st != Q4_OK) return st;
+    const cudaError_t e = q4::launch_interleave_gate_up(static_cast<const uint8_t *>(W_gate),
+                                                         static_cast<const uint8_t *>(W_up), static_cast<uint8_t *>(W_gu),
+                                                         F, K, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? Q4_OK : cuda_fail(e);
+}
+
 int q4_0_gemm_grouped(const q4_0_problem *problems, int count, q4_0_stream_t stream) {
     if (count < 0 || count > Q4_0_MAX_GROUP) return Q4_ERR_INVALID_ARG;
     if (count == 0) return Q4_OK;

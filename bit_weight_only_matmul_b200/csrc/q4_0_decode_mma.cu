@@ -34,6 +34,10 @@
 //  * the X warps convert the stage's X rows to fp16 straight into the
 //    matching mma.sync B fragments (two buffers per group), one 8-byte shared
 //    load per fragment for the compute threads;
+//  * fused epilogues (decode only): Y = sums + R, or, for a gate/up weight
+//    whose items hold 64 gate rows then the same 64 features' up rows,
+//    Y[m, f] = silu(gate) * up with the up tiles' sums handed to the gate
+//    tiles through shared memory -- the intermediate never reaches HBM;
 //  * the accumulators (two chains per n-tile) live across the whole item; at
 //    its end the group-1 warp hands its sums through shared memory to the
 //    group-0 warp of the same rows, which stores Y[m, n].
@@ -109,6 +113,8 @@ struct Smem {
     uint64_t raw_full[ring<NT>()], raw_empty[ring<NT>()];
     uint64_t xf_full[kXBufs], xf_empty[kXBufs];
     uint64_t comb_full, comb_empty;
+    float epi[4][NT][4][32];                    // SwiGLU: up-row sums handed to the gate rows
+    uint64_t epi_full, epi_empty;
     XComb<NT, SPLIT> x;
     int abort_flag;
 };
@@ -300,6 +306,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
         }
         mbar_init(&S.comb_full, kGroupWarps);
         mbar_init(&S.comb_empty, kGroupWarps);
+        mbar_init(&S.epi_full, kGroupWarps / 2);
+        mbar_init(&S.epi_empty, kGroupWarps / 2);
         if constexpr (SPLIT) {
             for (int s = 0; s < 2; ++s) {
                 mbar_init(&S.x.full[s], 32 * kGroupWarps);    // every thread of the partner's group 0
@@ -430,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
         for (int c = 0; c < 2; ++c)
             #pragma unroll
             for (int j = 0; j < NT; ++j) acc[c][j][0] = acc[c][j][1] = acc[c][j][2] = acc[c][j][3] = 0.f;
-        uint32_t g = 0, items_done = 0, split_done = 0;
+        uint32_t g = 0, items_done = 0, split_done = 0, swiglu_done = 0;
         Walk<SPLIT, SUB> q{};
         q.start(D, rank);
         for (; q.item >= 0; q.next(D, rank), ++g) {
@@ -509,14 +517,46 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
                         }
                     }
                     // thread holds rows gq / gq+8 of the tile x columns 8j+2t, 8j+2t+1
-                    if (!q.split || rank == 0) {
+                    if ((!q.split || rank == 0) && pr.epi == kEpiSwiGLU) {
+                        // rows 0-63 of the item are gate rows of features row0/2 .. row0/2+63,
+                        // rows 64-127 the up rows of the same features: tiles 4-7 hand their
+                        // sums to tiles 0-3, which store silu(gate) * up into Y[M, N/2]
+                        const uint32_t epar = swiglu_done & 1;
+                        ++swiglu_done;
+                        if (tile >= 4) {
+                            if (!wait_or_abort(&S.epi_empty, epar ^ 1, &S.abort_flag, P.err)) break;
+                            #pragma unroll
+                            for (int j = 0; j < NT; ++j)
+                                #pragma unroll
+                                for (int e = 0; e < 4; ++e) S.epi[tile - 4][j][e][lane] = sum[j][e];
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&S.epi_full);
+                        } else {
+                            if (!wait_or_abort(&S.epi_full, epar, &S.abort_flag, P.err)) break;
+                            const int F = pr.N >> 1;
+                            #pragma unroll
+                            for (int j = 0; j < NT; ++j)
+                                #pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const float gv = sum[j][e], uv = S.epi[tile][j][e][lane];
+                                    const int m = 8 * j + 2 * t + (e & 1);
+                                    const int f = (q.row0 >> 1) + 16 * tile + gq + ((e & 2) ? 8 : 0);
+                                    if (m < pr.M) pr.Y[static_cast<int64_t>(m) * F + f] = gv / (1.0f + expf(-gv)) * uv;
+                                }
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&S.epi_empty);
+                        }
+                    } else if (!q.split || rank == 0) {
                         #pragma unroll
                         for (int j = 0; j < NT; ++j)
                             #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 const int m = 8 * j + 2 * t + (e & 1);
                                 const int n = q.row0 + 16 * tile + gq + ((e & 2) ? 8 : 0);
-                                if (m < pr.M && n < pr.N) pr.Y[static_cast<int64_t>(m) * pr.N + n] = sum[j][e];
+                                if (m < pr.M && n < pr.N) {
+                                    const int64_t o = static_cast<int64_t>(m) * pr.N + n;
+                                    pr.Y[o] = pr.epi == kEpiResidual ? sum[j][e] + pr.R[o] : sum[j][e];
+                                }
                             }
                     }
                 }
@@ -708,6 +748,8 @@ cudaError_t launch_cap(const q4::Problem *probs, const int *order, int count, co
         t.W = q.W;
         t.X = q.X;
         t.Y = q.Y;
+        t.R = q.R;
+        t.epi = q.epi;
         t.M = static_cast<int>(q.M);
         t.N = static_cast<int>(q.N);
         t.K = static_cast<int>(q.K);

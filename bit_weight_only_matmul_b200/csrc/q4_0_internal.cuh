@@ -15,6 +15,8 @@ struct Problem {
     const uint16_t *X;
     float *Y;
     int64_t M, N, K;
+    const float *R = nullptr;   // residual (decode epilogue 1)
+    int epi = 0;                // decode epilogue: 0 none, 1 + R, 2 SwiGLU of row-interleaved gate/up
 };
 
 // Per-device facts cached by the API layer.
@@ -31,6 +33,8 @@ cudaError_t launch_pack(const uint8_t *codes, const uint16_t *scales, uint8_t *W
                         int64_t N, int64_t K, cudaStream_t s);
 cudaError_t launch_dequant(const uint8_t *W, float *out, int64_t N, int64_t K, cudaStream_t s);
 cudaError_t launch_zero(float *Y, int64_t count, cudaStream_t s);
+cudaError_t launch_interleave_gate_up(const uint8_t *Wg, const uint8_t *Wu, uint8_t *Wgu, int64_t F, int64_t K,
+                                     cudaStream_t s);
 cudaError_t launch_gather(const uint8_t *W, const int32_t *ids, float *out, int64_t T, int64_t V, int64_t D,
                           const DeviceInfo &dev, cudaStream_t s);
 cudaError_t launch_quantize(const float *X, uint8_t *W, int64_t N, int64_t K, const DeviceInfo &dev,

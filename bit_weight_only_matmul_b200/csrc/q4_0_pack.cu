@@ -59,6 +59,23 @@ __global__ void dequant_kernel(const uint8_t *__restrict__ W, float *__restrict_
     }
 }
 
+// Row-interleaved gate/up weight for the fused SwiGLU epilogue: destination
+// rows 128i .. 128i+63 are gate rows 64i .. 64i+63, rows 128i+64 .. 128i+127
+// the up rows of the same features.  One warp per destination row, 16-byte
+// copies (rows of K/32*18 bytes, a multiple of 16 when K % 256 == 0).
+__global__ void interleave_kernel(const uint8_t *__restrict__ Wg, const uint8_t *__restrict__ Wu,
+                                  uint8_t *__restrict__ Wgu, int64_t F, int64_t row_vec) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t r = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; r < 2 * F; r += warps) {
+        const int64_t i = r >> 7, w = r & 127;
+        const uint8_t *src = w < 64 ? Wg + (64 * i + w) * row_vec * 16 : Wu + (64 * i + w - 64) * row_vec * 16;
+        const uint4 *sv = reinterpret_cast<const uint4 *>(src);
+        uint4 *dv = reinterpret_cast<uint4 *>(Wgu + r * row_vec * 16);
+        for (int64_t c = lane; c < row_vec; c += 32) dv[c] = sv[c];
+    }
+}
+
 // Portable GEMM: one warp per (row n, chunk of up to 8 rows of X).  Lanes
 // stride over the blocks of the row, each block's 32 products are summed in
 // fp32 and scaled by d once, and the lanes' partial sums are combined with
@@ -139,6 +156,13 @@ cudaError_t launch_pack(const uint8_t *codes, const uint16_t *scales, uint8_t *W
 cudaError_t launch_dequant(const uint8_t *W, float *out, int64_t N, int64_t K, cudaStream_t s) {
     const int64_t nblocks = N * (K / 32);
     dequant_kernel<<<grid_for(nblocks, 256), 256, 0, s>>>(W, out, nblocks);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_interleave_gate_up(const uint8_t *Wg, const uint8_t *Wu, uint8_t *Wgu, int64_t F, int64_t K,
+                                     cudaStream_t s) {
+    const int64_t rows = 2 * F;
+    interleave_kernel<<<grid_for(rows * 32, 256), 256, 0, s>>>(Wg, Wu, Wgu, F, K / 32 * 18 / 16);
     return cudaGetLastError();
 }
 

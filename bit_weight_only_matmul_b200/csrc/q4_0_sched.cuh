@@ -27,7 +27,12 @@ struct GroupProblem {
     int M, N, K;
     int stages;        // K / 256
     int item_begin;    // first item index of this problem
+    const float *R;    // residual added to Y (epilogue kEpiResidual)
+    int epi;           // kEpi*: what the item's end does with its sums
 };
+
+// Epilogues of a decode item (values of the C ABI's Q4_0_EPI_*).
+constexpr int kEpiNone = 0, kEpiResidual = 1, kEpiSwiGLU = 2;
 
 // CAP problems per launch; the weights' TMA maps live in the kernel parameters.
 template <int CAP>

@@ -175,6 +175,45 @@ Q4_0_API int q4_0_gemm_ws(const void *W, const uint16_t *X, float *Y,
 Q4_0_API int q4_0_gemm_static_ws(const void *W, const uint16_t *X, float *Y,
                                  int64_t M, int64_t N, int64_t K, q4_0_stream_t stream);
 
+/* Fused epilogues of the decode path (q4_0_gemm_grouped_ex). */
+#define Q4_0_EPI_NONE 0      /* Y = X * dequant(W)^T */
+#define Q4_0_EPI_RESIDUAL 1  /* Y = X * dequant(W)^T + R (R [M,N] fp32; R == Y allowed) */
+#define Q4_0_EPI_SWIGLU 2    /* Y[M, N/2] = silu(gate) * up of a row-interleaved gate/up W */
+
+/* A grouped problem with a fused epilogue.  W, X, M, N, K as in
+ * q4_0_problem.  R: the residual for Q4_0_EPI_RESIDUAL (device, 16-byte
+ * aligned, [M,N] fp32), ignored otherwise.  For Q4_0_EPI_SWIGLU, W holds 2F
+ * rows (N = 2F, F % 64 == 0) in the order q4_0_interleave_gate_up writes
+ * and Y is [M, F]. */
+typedef struct q4_0_problem_ex {
+    const void *W;
+    const uint16_t *X;
+    float *Y;
+    int64_t M, N, K;
+    const float *R;
+    int32_t epilogue;
+} q4_0_problem_ex;
+
+/* q4_0_gemm_grouped with the step on either side of a decoder layer's
+ * linears fused into the store of Y, so that no intermediate makes a round
+ * trip through HBM: the residual add after the O and down projections, and
+ * the SwiGLU activation silu(g) * u (silu(g) = g / (1 + exp(-g)), fp32)
+ * between the fused gate/up projection (voxtral-mini-realtime-rs README, TTS
+ * section, optimizations) and the down projection.  The epilogues run on the
+ * decode path: every problem needs 1 <= M <= 32, K a positive multiple of 256
+ * and 16-byte aligned W, X, Y, R, else Q4_ERR_INVALID_ARG and nothing is
+ * launched.  Tolerance: the GEMM bound of each input of the epilogue, carried
+ * through it (silu' <= 1.1), plus fp32 rounding of the epilogue. */
+Q4_0_API int q4_0_gemm_grouped_ex(const q4_0_problem_ex *problems, int count, q4_0_stream_t stream);
+
+/* Row-interleaved gate/up weight for Q4_0_EPI_SWIGLU: W_gu rows 128i .. 128i+63
+ * = W_gate rows 64i .. 64i+63 and rows 128i+64 .. 128i+127 = W_up rows
+ * 64i .. 64i+63, for i < F/64.  W_gate, W_up: F rows each; W_gu: 2F rows; all
+ * Q4_0 device buffers, 16-byte aligned, not overlapping; F % 64 == 0 and
+ * K % 256 == 0. */
+Q4_0_API int q4_0_interleave_gate_up(const void *W_gate, const void *W_up, void *W_gu,
+                                     int64_t F, int64_t K, q4_0_stream_t stream);
+
 /* Row gather (a Q4 embedding lookup): out[t, :] = dequant(W)[ids[t], :] for
  * t < T, W a Q4_0 matrix of V rows by D weights, out float32 [T, D] row-major
  * (exact: each (q - 8) * d is representable in float32).  The pages keep the

@@ -128,3 +128,21 @@ def test_gather_quantize_argument_checks(q4):
     assert qz(None, A, 4, 64, None) == q4.Q4_ERR_INVALID_ARG
     assert qz(A + 4, A, 4, 64, None) == q4.Q4_ERR_MISALIGNED
     assert qz(None, None, 0, 64, None) == q4.Q4_OK
+
+
+def test_grouped_ex_argument_checks(q4):
+    def ex(M, N, K, R=A, epi=q4.Q4_0_EPI_RESIDUAL):
+        arr = (q4.q4_0_problem_ex * 1)()
+        arr[0] = q4.q4_0_problem_ex(A, A, A, M, N, K, R, epi)
+        return q4.lib.q4_0_gemm_grouped_ex(arr, 1, None)
+    assert ex(33, 128, 256) == q4.Q4_ERR_INVALID_ARG                      # decode path only: M <= 32
+    assert ex(4, 128, 288) == q4.Q4_ERR_INVALID_ARG                       # K % 256
+    assert ex(4, 128, 256, R=None) == q4.Q4_ERR_INVALID_ARG               # residual needs R
+    assert ex(4, 128, 256, R=A + 4) == q4.Q4_ERR_MISALIGNED
+    assert ex(4, 192, 256, epi=q4.Q4_0_EPI_SWIGLU) == q4.Q4_ERR_INVALID_ARG   # 2F with F % 64
+    assert ex(4, 128, 256, epi=7) == q4.Q4_ERR_INVALID_ARG
+    il = q4.lib.q4_0_interleave_gate_up
+    assert il(A, A, A, 96, 256, None) == q4.Q4_ERR_INVALID_ARG            # F % 64
+    assert il(A, A, A, 64, 288, None) == q4.Q4_ERR_INVALID_ARG            # K % 256
+    assert il(A + 8, A, A, 64, 256, None) == q4.Q4_ERR_MISALIGNED
+    assert il(None, None, None, 0, 256, None) == q4.Q4_OK
