@@ -55,6 +55,7 @@ DOMINANT = {
     "cfg_decode": ("decode_mma_kernel", "q4_0_decode_mma.cu"),
     "concurrent": ("decode_mma_kernel", "q4_0_decode_mma.cu"),
     "flow_head": ("decode_mma_kernel", "q4_0_decode_mma.cu"),
+    "layer_fused": ("decode_mma_kernel", "q4_0_decode_mma.cu"),
     "adapter": ("prefill_kernel", "q4_0_prefill.cu"),
     "qkv_prefill": ("prefill_kernel", "q4_0_prefill.cu"),
 }
@@ -177,12 +178,49 @@ class GpuWorkload:
         ws = max([q4.q4_0_gemm_workspace_size(l.M, l.N, l.K) for l in wl.linears] + [0])
         self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device="cuda")
         self.small_arrs = [q4.make_problems([probs[i] for i in self.small]) for probs, _ in self.sets]
+        self.fused_arrs = []
+        if wl.fused:
+            # the same weights with the epilogues fused: gate/up re-laid out
+            # row-interleaved (gate rows 0..F-1, up rows F..2F-1 of the
+            # concatenated weight), Y of width F; O and down add a residual
+            self.keep = []
+            self.fused_ys = []
+            for probs, _ in self.sets:
+                ex, ys = [], []
+                for (W, X, Y, M, N, K), lin in zip(probs, wl.linears):
+                    if lin.name == "gate_up":
+                        F = N // 2
+                        half = F * (K // 32) * 18
+                        Wgu = torch.empty_like(W)
+                        q4.q4_0_interleave_gate_up(W[:half], W[half:], Wgu, F, K)
+                        Yf = torch.empty((M, F), dtype=torch.float32, device="cuda")
+                        self.keep += [Wgu, Yf]
+                        ys.append(Yf)
+                        ex.append((Wgu, X, Yf, M, N, K, None, q4.Q4_0_EPI_SWIGLU))
+                    elif lin.name in ("o", "down"):
+                        R = torch.randn((M, N), device="cuda")
+                        self.keep.append(R)
+                        ys.append(Y)
+                        ex.append((W, X, Y, M, N, K, R, q4.Q4_0_EPI_RESIDUAL))
+                    else:
+                        ys.append(Y)
+                        ex.append((W, X, Y, M, N, K, None, q4.Q4_0_EPI_NONE))
+                self.fused_arrs.append(q4.make_problems_ex(ex))
+                self.fused_ys.append(ys)
         self.operand_bytes = sum(W.numel() + X.numel() * 2 + Y.numel() * 4 for W, X, Y, *_ in self.sets[0][0])
         torch.cuda.synchronize()
+
+    def outputs(self, step: int):
+        """The Y tensors a step writes."""
+        k = step % len(self.sets)
+        return self.fused_ys[k] if self.fused_arrs else [p[2] for p in self.sets[k][0]]
 
     def launch(self, q4, step: int):
         k = step % len(self.sets)
         probs, _ = self.sets[k]
+        if self.fused_arrs:
+            q4.q4_0_gemm_grouped_ex(self.fused_arrs[k], len(probs))
+            return
         if self.small:
             q4.q4_0_gemm_grouped(self.small_arrs[k], len(self.small))
         for i in self.large:
@@ -272,7 +310,7 @@ def run_ours(args, rank: int, world: int):
     # end to end through the public API: host X -> device, grouped GEMM, Y -> host
     probs0 = G.sets[0][0]
     hx = [torch.empty(p[1].shape, dtype=p[1].dtype, pin_memory=True).copy_(p[1].cpu()) for p in probs0]
-    hy = [torch.empty(p[2].shape, dtype=p[2].dtype, pin_memory=True) for p in probs0]
+    hy = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for y in G.outputs(0)]
     h2d = sum(t.numel() * t.element_size() for t in hx)
     d2h = sum(t.numel() * t.element_size() for t in hy)
     e0 = torch.cuda.Event(enable_timing=True)
@@ -283,7 +321,7 @@ def run_ours(args, rank: int, world: int):
         for (W, X, Y, *_), h in zip(probs, hx):
             X.copy_(h, non_blocking=True)
         G.launch(q4, k)
-        for (W, X, Y, *_), h in zip(probs, hy):
+        for Y, h in zip(G.outputs(k), hy):
             h.copy_(Y, non_blocking=True)
 
     for i in range(args.warmup):

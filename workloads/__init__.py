@@ -159,6 +159,7 @@ class Workload:
     name: str
     description: str
     linears: List[Linear] = field(default_factory=list)
+    fused: bool = False   # gate/up -> SwiGLU (Y is half as wide), O and down + a residual read
 
     @property
     def weight_bytes(self) -> int:
@@ -166,8 +167,17 @@ class Workload:
 
     @property
     def hbm_bytes(self) -> int:
-        """Algorithmic bytes: every weight byte once plus X and Y once."""
-        return sum(l.weight_bytes + l.act_bytes for l in self.linears)
+        """Algorithmic bytes: every weight byte once plus X and Y once (with
+        the fused epilogues: the gate/up output is N/2 wide and the O and
+        down outputs also read a residual of their own size)."""
+        total = sum(l.weight_bytes + l.act_bytes for l in self.linears)
+        if self.fused:
+            for l in self.linears:
+                if l.name == "gate_up":
+                    total -= l.M * (l.N // 2) * 4
+                elif l.name in ("o", "down"):
+                    total += l.M * l.N * 4
+        return total
 
     @property
     def flops(self) -> int:
@@ -191,6 +201,9 @@ def workload(name: str, layers: Optional[List[int]] = None) -> Workload:
         ls = range(N_LAYERS) if layers is None else layers
         return Workload(name, "concurrent decode, M=32, 26 stacked layers, 3 of 32 X rows x8",
                         [l for i in ls for l in decoder_layer(i, 32, outlier_rows=3)])
+    if name == "layer_fused":
+        return Workload(name, "the layer set at M=1 with fused epilogues: O and down + residual, "
+                              "gate/up -> SwiGLU (one grouped launch)", decoder_layer(0, 1), fused=True)
     if name == "flow_head":
         # the flow-matching head: 3 transformer layers run once per Euler step
         # on the batch-2 CFG rows (the pages give no width for it; reading:
@@ -208,7 +221,7 @@ def workload(name: str, layers: Optional[List[int]] = None) -> Workload:
     raise KeyError(name)
 
 
-WORKLOADS = ["gemv", "layer", "cfg_decode", "concurrent", "flow_head", "adapter", "qkv_prefill"]
+WORKLOADS = ["gemv", "layer", "layer_fused", "cfg_decode", "concurrent", "flow_head", "adapter", "qkv_prefill"]
 
 # ---------------------------------------------------------------------------
 # the two utilities around the product (row gather, quantization)
