@@ -20,8 +20,10 @@
 // compute warps; X warp G and compute group G take the stages g with
 // g mod 2 == G, so that two stages are worked on at once.
 //  * stage = 256 k of an item (128 weight rows x 144 bytes, one TMA box) plus
-//    the same 256 k of every row of X (1-D bulk copies), in a 4-6-deep ring;
-//    the TMA box pattern alone streams at ~6.9 TB/s (measured);
+//    the same 256 k of every row of X (1-D bulk copies), in a ring of 4-6
+//    slots; for M <= 8 a slot holds two stages, so that every wait, arrival
+//    and walk step covers 512 k; the TMA box pattern alone streams at
+//    ~6.9 TB/s (measured);
 //  * compute warp w of a group owns rows 16w .. 16w+15; thread (g, t) reads
 //    the 36 contiguous bytes of blocks 2t and 2t+1 of rows g and g+8 (nine
 //    conflict-free 4-byte loads per row), turns them into fp16 (q - 8) * d
@@ -51,6 +53,9 @@
 // Y.  The other items stay whole, each on one CTA.  The host deals the split
 // items to the clusters and then the whole items to the CTAs, longest first
 // onto the least loaded.
+// Launches use programmatic stream serialization: the next grid on the
+// stream may start as this grid's CTAs leave, and every CTA waits for the
+// previous grid before its first global access.
 // Numerics: each weight is rounded once to fp16 (relative error <= 2^-11,
 // inside the 1e-3 tolerance of the method); X is exact in fp16 within its
 // normal range; products are exact and accumulation is fp32.  Operands beyond

@@ -29,7 +29,7 @@
  *
  * Every product (q-8)*d*x is exact in float64 (4 + 11 + 8 significant bits).
  *
- * Operations around the product (the next steps the survey ranks, not the
+ * Operations around the product (the steps next to it in a decoder, not the
  * hot path itself):
  *   swiglu   -- the activation between the fused gate/up projection and the
  *               down projection of a decoder layer's feed-forward block:
