@@ -49,6 +49,7 @@ EXPORTS = (
     "q4_0_interleave_gate_up",
     "q4_0_gather",
     "q4_0_quantize",
+    "q4_0_selftest_wait_timeout",
     "q4_0_device_error",
     "q4_0_force_path",
 )
@@ -95,6 +96,7 @@ def _load() -> ctypes.CDLL:
         "q4_0_gather": (i32, [vp, vp, vp, i64, i64, i64, vp]),
         "q4_0_quantize": (i32, [vp, vp, i64, i64, vp]),
         "q4_0_device_error": (i32, [ctypes.POINTER(ctypes.c_uint32), i32]),
+        "q4_0_selftest_wait_timeout": (i32, [ctypes.c_uint32, vp]),
         "q4_0_force_path": (i32, [i32]),
     }
     for name, (res, args) in sig.items():

@@ -307,6 +307,16 @@ int q4_0_interleave_gate_up(const void *W_gate, const void *W_up, void *W_gu, in
     return e == cudaSuccess ? Q4_OK : cuda_fail(e);
 }
 
+int q4_0_selftest_wait_timeout(uint32_t limit_us, q4_0_stream_t stream) {
+    if (limit_us < 1 || limit_us > 1000000) return Q4_ERR_INVALID_ARG;
+    const q4::DeviceInfo *dev = nullptr;
+    int st = current_device(&dev);
+    if (st != Q4_OK) return st;
+    const cudaError_t e = q4::launch_selftest_wait(*dev, static_cast<unsigned long long>(limit_us) * 1000ull,
+                                                   reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? Q4_OK : cuda_fail(e);
+}
+
 int q4_0_gemm_grouped(const q4_0_problem *problems, int count, q4_0_stream_t stream) {
     if (count < 0 || count > Q4_0_MAX_GROUP) return Q4_ERR_INVALID_ARG;
     if (count == 0) return Q4_OK;

@@ -33,6 +33,9 @@ cudaError_t launch_pack(const uint8_t *codes, const uint16_t *scales, uint8_t *W
                         int64_t N, int64_t K, cudaStream_t s);
 cudaError_t launch_dequant(const uint8_t *W, float *out, int64_t N, int64_t K, cudaStream_t s);
 cudaError_t launch_zero(float *Y, int64_t count, cudaStream_t s);
+// One CTA whose thread 0 waits, bounded by limit_ns, on a barrier nothing
+// arrives on (self-test of the bounded waits).
+cudaError_t launch_selftest_wait(const DeviceInfo &dev, unsigned long long limit_ns, cudaStream_t s);
 cudaError_t launch_interleave_gate_up(const uint8_t *Wg, const uint8_t *Wu, uint8_t *Wgu, int64_t F, int64_t K,
                                      cudaStream_t s);
 cudaError_t launch_gather(const uint8_t *W, const int32_t *ids, float *out, int64_t T, int64_t V, int64_t D,
@@ -141,13 +144,14 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t pa
 }
 
 // Wait for phase `parity` of an mbarrier to complete, for at most
-// kWaitLimitNs.  Returns false (and ORs Q4_DEVERR_WAIT_TIMEOUT into *err) if
-// the wait ran out.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned *err) {
+// kWaitLimitNs (or `limit_ns`).  Returns false (and ORs
+// Q4_DEVERR_WAIT_TIMEOUT into *err) if the wait ran out.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned *err,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     while (!mbar_try_wait_suspend(bar, parity)) {
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (global_ns() - t0 > limit_ns) {
             atomicOr(err, (unsigned)Q4_DEVERR_WAIT_TIMEOUT);
             return false;
         }

@@ -76,6 +76,20 @@ __global__ void interleave_kernel(const uint8_t *__restrict__ Wg, const uint8_t 
     }
 }
 
+// Self-test of the failure detection: thread 0 waits on an mbarrier that no
+// one arrives on.  The bounded wait must give up after limit_ns, set
+// Q4_DEVERR_WAIT_TIMEOUT in the device error word and let the kernel return;
+// no copy or MMA is in flight, so nothing else needs to land first.
+__global__ void selftest_wait_kernel(unsigned *err, unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        q4dev::mbar_init(&bar, 1);
+        q4dev::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)q4dev::mbar_wait(&bar, 0, err, limit_ns);
+}
+
 // Portable GEMM: one warp per (row n, chunk of up to 8 rows of X).  Lanes
 // stride over the blocks of the row, each block's 32 products are summed in
 // fp32 and scaled by d once, and the lanes' partial sums are combined with
@@ -163,6 +177,11 @@ cudaError_t launch_interleave_gate_up(const uint8_t *Wg, const uint8_t *Wu, uint
                                      cudaStream_t s) {
     const int64_t rows = 2 * F;
     interleave_kernel<<<grid_for(rows * 32, 256), 256, 0, s>>>(Wg, Wu, Wgu, F, K / 32 * 18 / 16);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_wait(const DeviceInfo &dev, unsigned long long limit_ns, cudaStream_t s) {
+    selftest_wait_kernel<<<1, 32, 0, s>>>(dev.err, limit_ns);
     return cudaGetLastError();
 }
 

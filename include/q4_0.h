@@ -214,6 +214,14 @@ Q4_0_API int q4_0_gemm_grouped_ex(const q4_0_problem_ex *problems, int count, q4
 Q4_0_API int q4_0_interleave_gate_up(const void *W_gate, const void *W_up, void *W_gu,
                                      int64_t F, int64_t K, q4_0_stream_t stream);
 
+/* Self-test of the failure detection (no counterpart on the pages): one
+ * CTA waits on an on-chip barrier that nothing arrives on, bounded by
+ * limit_us (1 .. 1000000); the wait gives up, ORs Q4_DEVERR_WAIT_TIMEOUT into
+ * q4_0_device_error and the kernel returns, leaving the context usable.  It
+ * lets a test show that a bounded wait ends and reports, without any fault.
+ * Asynchronous on `stream` like every call. */
+Q4_0_API int q4_0_selftest_wait_timeout(uint32_t limit_us, q4_0_stream_t stream);
+
 /* Row gather (a Q4 embedding lookup): out[t, :] = dequant(W)[ids[t], :] for
  * t < T, W a Q4_0 matrix of V rows by D weights, out float32 [T, D] row-major
  * (exact: each (q - 8) * d is representable in float32).  The pages keep the

@@ -146,3 +146,8 @@ def test_grouped_ex_argument_checks(q4):
     assert il(A, A, A, 64, 288, None) == q4.Q4_ERR_INVALID_ARG            # K % 256
     assert il(A + 8, A, A, 64, 256, None) == q4.Q4_ERR_MISALIGNED
     assert il(None, None, None, 0, 256, None) == q4.Q4_OK
+
+
+def test_selftest_argument_checks(q4):
+    assert q4.lib.q4_0_selftest_wait_timeout(0, None) == q4.Q4_ERR_INVALID_ARG
+    assert q4.lib.q4_0_selftest_wait_timeout(1000001, None) == q4.Q4_ERR_INVALID_ARG
