@@ -1,6 +1,7 @@
-// q4_0_sched.cuh -- work distribution shared by the persistent decode kernels:
-// the grouped-problem parameter block, the (item, stage) walk of one CTA, and
-// a bounded mbarrier wait that also stops when another role has aborted.
+// q4_0_sched.cuh -- pieces of the persistent decode kernel's work
+// distribution: the grouped-problem parameter block, the search of an item's
+// problem, and a bounded mbarrier wait that also stops when another role has
+// aborted.
 //
 // An item is 128 weight rows x all of K of one problem.  Problems are sorted
 // by K (largest first) on the host, so items with long rows come first, and
@@ -53,32 +54,6 @@ __device__ __forceinline__ int find_problem(const TP &P, int item) {
     }
     return lo;
 }
-
-// One CTA's sequence of (item, stage).
-struct Seq {
-    int round, item, prob, row0, stage, nstages;
-    uint32_t nitems;   // items this CTA finished before the current one
-    template <class TP>
-    __device__ __forceinline__ void load(const TP &P) {
-        const int G = gridDim.x;
-        const int pos = (round & 1) ? (G - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
-        item = round * G + pos;
-        if (item >= P.total_items) { item = -1; return; }
-        prob = find_problem(P, item);
-        row0 = (item - P.p[prob].item_begin) * kItemRows;
-        stage = 0;
-        nstages = P.p[prob].stages;
-    }
-    template <class TP>
-    __device__ __forceinline__ void start(const TP &P) { round = 0; nitems = 0; load(P); }
-    template <class TP>
-    __device__ __forceinline__ void next(const TP &P) {
-        if (++stage < nstages) return;
-        ++round;
-        ++nitems;
-        load(P);
-    }
-};
 
 // Bounded wait (kWaitLimitNs) that gives up early once *abort_flag is set, and
 // sets it (with Q4_DEVERR_WAIT_TIMEOUT in *err) when it runs out itself.

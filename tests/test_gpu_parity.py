@@ -341,3 +341,15 @@ def test_workspace_too_small_falls_back(q4):
 @pytest.mark.parametrize("M,N,K", [(1, 100, 1024), (2, 129, 3072), (16, 33, 2048), (32, 70, 512)])
 def test_forced_tmem_decode(q4, M, N, K):
     run_gemm(q4, M, N, K, path=q4.PATH_DECODE_TMEM)
+
+
+@pytest.mark.parametrize("name", ["concurrent", "cfg_decode"])
+def test_forced_tmem_decode_workload(q4, name):
+    b = build_workload(q4, workloads.workload(name, layers=[0, 1]), samples=300)
+    q4.q4_0_force_path(q4.PATH_DECODE_TMEM)
+    try:
+        q4.q4_0_gemm_grouped(b.problems())
+    finally:
+        q4.q4_0_force_path(0)
+    check_built(b, f"{name} layers 0-1, tcgen05 decode")
+    no_device_error(q4)
