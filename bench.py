@@ -158,19 +158,35 @@ class GpuWorkload:
         import torch
         self.wl = wl
         self.sets = []
+        # a step's X (and Y) tensors are views of one contiguous buffer per
+        # copy, so that the end-to-end step moves them with one copy each way
+        def offsets(sizes):
+            out, at = [], 0
+            for n in sizes:
+                out.append(at)
+                at += -(-n // 64) * 64   # 64-element steps keep every view 16-byte aligned
+            return out, at
+        x_off, x_total = offsets([l.M * l.K for l in wl.linears])
+        y_off, y_total = offsets([l.M * l.N for l in wl.linears])
+        self.xbufs, self.ybufs = [], []
         for c in range(copies):
             probs = []
-            for lin in wl.linears:
+            xbuf = torch.zeros(x_total, dtype=torch.int16, device="cuda")
+            ybuf = torch.empty(y_total, dtype=torch.float32, device="cuda")
+            for lin, xo, yo in zip(wl.linears, x_off, y_off):
                 s = seed + 7919 * c
                 codes = torch.from_numpy(lin.codes(s)).cuda()
                 scales = torch.from_numpy(lin.scales(s).view(np.int16)).cuda()
                 W = torch.empty(q4.q4_0_bytes(lin.N, lin.K), dtype=torch.uint8, device="cuda")
                 q4.q4_0_pack(codes, scales, W, lin.N, lin.K)
                 del codes, scales
-                X = torch.from_numpy(lin.x(s).view(np.int16)).cuda()
-                Y = torch.empty((lin.M, lin.N), dtype=torch.float32, device="cuda")
+                X = xbuf[xo:xo + lin.M * lin.K].view(lin.M, lin.K)
+                X.copy_(torch.from_numpy(lin.x(s).view(np.int16)))
+                Y = ybuf[yo:yo + lin.M * lin.N].view(lin.M, lin.N)
                 probs.append((W, X, Y, lin.M, lin.N, lin.K))
             self.sets.append((probs, q4.make_problems(probs)))
+            self.xbufs.append(xbuf)
+            self.ybufs.append(ybuf)
         # the M > 32 GEMMs run through q4_0_gemm_ws with one shared workspace
         # (X converted to fp16 once per GEMM); the M <= 32 ones in one grouped launch
         self.small = [i for i, l in enumerate(wl.linears) if l.M <= 32]
@@ -308,20 +324,20 @@ def run_ours(args, rank: int, world: int):
         raise RuntimeError(f"device error word {dev_err:#x} after the timed region")
 
     # end to end through the public API: host X -> device, grouped GEMM, Y -> host
-    probs0 = G.sets[0][0]
-    hx = [torch.empty(p[1].shape, dtype=p[1].dtype, pin_memory=True).copy_(p[1].cpu()) for p in probs0]
-    hy = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for y in G.outputs(0)]
+    # (one pinned copy each way: a step's X and Y live in one buffer each)
+    hx = [torch.empty(G.xbufs[0].shape, dtype=G.xbufs[0].dtype, pin_memory=True).copy_(G.xbufs[0].cpu())]
+    outs0 = [G.ybufs[0]] if not G.fused_arrs else G.outputs(0)
+    hy = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for y in outs0]
     h2d = sum(t.numel() * t.element_size() for t in hx)
     d2h = sum(t.numel() * t.element_size() for t in hy)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
 
     def e2e_step(k):
-        probs, _ = G.sets[k % len(G.sets)]
-        for (W, X, Y, *_), h in zip(probs, hx):
-            X.copy_(h, non_blocking=True)
+        c = k % len(G.sets)
+        G.xbufs[c].copy_(hx[0], non_blocking=True)
         G.launch(q4, k)
-        for Y, h in zip(G.outputs(k), hy):
+        for Y, h in zip([G.ybufs[c]] if not G.fused_arrs else G.outputs(k), hy):
             h.copy_(Y, non_blocking=True)
 
     for i in range(args.warmup):
