@@ -353,3 +353,43 @@ def test_forced_tmem_decode_workload(q4, name):
         q4.q4_0_force_path(0)
     check_built(b, f"{name} layers 0-1, tcgen05 decode")
     no_device_error(q4)
+
+
+def test_decode_vocab_sized_gemv_sampled(q4):
+    """M=1 against a 131072-row weight (an LM-head / embedding-table shape): 1024
+    items, the edge of split mode, checked at sampled outputs including the
+    last row."""
+    M, N, K = 1, 131072, 3072
+    rng = np.random.default_rng(12)
+    o = oracle.get()
+    codes = workloads.gen_codes(N, K, layer=77)
+    scales = workloads.gen_scales(N, K, layer=77)
+    X = workloads.gen_x(M, K, layer=77)
+    W_host = o.pack(codes, scales)
+    W = torch.from_numpy(W_host.reshape(-1)).cuda()
+    del codes
+    Y = torch.full((M, N), float("nan"), device="cuda")
+    q4.q4_0_gemm(W, dev(X), Y, M, N, K)
+    ns = np.concatenate([rng.integers(0, N, 300), [0, N - 1, 128 * 1023, 128 * 1023 + 127]])
+    ms = np.zeros_like(ns)
+    Y_or, B_or = o.gemm_sampled(W_host, X, M, N, K, ms, ns)
+    check_gemm(Y.cpu().numpy()[ms, ns], Y_or, B_or, "vocab-sized gemv")
+    no_device_error(q4)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 200, 1024), (2, 300, 3072), (24, 129, 512), (64, 256, 512)])
+def test_subnormal_scales(q4, M, N, K):
+    """Scales in the fp16 subnormal range: every (q - 8) * d is then an exact
+    fp16 subnormal, on the decode and the tensor-core paths alike."""
+    rng = np.random.default_rng(M * 13 + N + K)
+    codes = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
+    scales = rng.integers(1, 0x400, size=(N, K // 32)).astype(np.uint16)   # positive subnormals
+    scales[::3] |= 0x8000                                                   # and negative ones
+    X = workloads.fp32_to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    W = pack_on_gpu(q4, codes, scales)
+    Y = torch.full((M, N), float("nan"), device="cuda")
+    q4.q4_0_gemm(W, dev(X), Y, M, N, K)
+    o = oracle.get()
+    Y_or, B_or = o.gemm(o.pack(codes, scales), X, M, N, K)
+    check_gemm(Y.cpu().numpy(), Y_or, B_or, "subnormal scales")
+    no_device_error(q4)
