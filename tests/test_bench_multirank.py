@@ -45,3 +45,18 @@ def test_whole_job_rate_is_weak_scaling():
     # 2 ranks x 10 steps x 1e9 bytes in 20 ms (slowest rank) = 1e12 B/s
     assert bench.whole_job_rate(1e9, 10, 2, 20.0) == pytest.approx(1e12)
     assert bench.max_over_ranks([1.0, 2.0], 1, "cpu") == [1.0, 2.0]
+
+
+def test_workload_byte_accounting():
+    """The bench's algorithmic bytes: every weight byte once plus X and Y once;
+    the fused layer writes half of the gate/up output and reads two residuals."""
+    import workloads
+    layer = workloads.workload("layer")
+    W = sum(l.N * (l.K // 32) * 18 for l in layer.linears)
+    XY = sum(l.M * l.K * 2 + l.M * l.N * 4 for l in layer.linears)
+    assert layer.hbm_bytes == W + XY == 56768512
+    fused = workloads.workload("layer_fused")
+    assert fused.hbm_bytes == layer.hbm_bytes - 1 * 8192 * 4 + 2 * 1 * 3072 * 4
+    cfg = workloads.workload("cfg_decode")
+    assert cfg.hbm_bytes == 1479761920
+    assert workloads.workload("adapter").flops == 2 * 4096 * 3072 * 5120
