@@ -15,8 +15,9 @@
 //
 // Quantize: the GGUF Q4_0 rule the pages apply offline (their
 // quantize_tts_gguf.py, named in the voxtral-mini-realtime-rs README, TTS
-// section), one warp per block of 32: the value of largest magnitude (the
-// first on ties) by a shuffle reduction, d = m / -8, id = 1/d (0 if d == 0),
+// section), four blocks per warp step (a float4 per lane): the value of
+// largest magnitude (the first on ties) over each block's eight lanes by a
+// shuffle reduction, d = m / -8, id = 1/d (0 if d == 0),
 // q = min(15, trunc(x * id + 8.5)) with the product and the sum rounded
 // separately (no fused multiply-add), fp16(d) rounded to nearest even.
 #include <cuda_fp16.h>
@@ -27,7 +28,6 @@ namespace {
 
 constexpr int kBlockBytes = 18;
 
-constexpr int kUnroll = 4;   // blocks per warp step in quantize, loads issued first
 
 __global__ void gather_kernel(const uint8_t *__restrict__ W, const int32_t *__restrict__ ids,
                               float *__restrict__ out, int64_t T, int64_t V, int64_t nb, unsigned *err) {
@@ -60,44 +60,50 @@ __global__ void gather_kernel(const uint8_t *__restrict__ W, const int32_t *__re
 }
 
 __global__ void quantize_kernel(const float *__restrict__ X, uint8_t *__restrict__ W, int64_t nblocks) {
-    const int lane = threadIdx.x & 31;
+    // a warp takes four blocks per step: lane (b, c) holds values 4c..4c+3 of block b
+    const int lane = threadIdx.x & 31, c = lane & 7;
     const int64_t warp0 = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t b0 = warp0; b0 < nblocks; b0 += kUnroll * warps) {
-        float x[kUnroll];
+    const int64_t quads = (nblocks + 3) / 4;
+    for (int64_t qd = warp0; qd < quads; qd += warps) {
+        const int64_t b = qd * 4 + (lane >> 3);
+        const bool live = b < nblocks;
+        const float4 v = live ? reinterpret_cast<const float4 *>(X + b * 32)[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float x[4] = {v.x, v.y, v.z, v.w};
+        // the first of the largest magnitudes: in the lane, then over the block's 8 lanes
+        float a = fabsf(x[0]), m = x[0];
+        int at = 4 * c;
         #pragma unroll
-        for (int i = 0; i < kUnroll; ++i) {
-            const int64_t b = b0 + i * warps;
-            x[i] = b < nblocks ? X[b * 32 + lane] : 0.0f;
+        for (int i = 1; i < 4; ++i) {
+            const float ai = fabsf(x[i]);
+            if (ai > a) { a = ai; m = x[i]; at = 4 * c + i; }
         }
         #pragma unroll
-        for (int i = 0; i < kUnroll; ++i) {
-            const int64_t b = b0 + i * warps;
-            if (b >= nblocks) break;   // warp-uniform
-            // the first of the largest magnitudes
-            float a = fabsf(x[i]);
-            int at = lane;
-            #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float a2 = __shfl_xor_sync(0xffffffffu, a, off);
-                const int at2 = __shfl_xor_sync(0xffffffffu, at, off);
-                if (a2 > a || (a2 == a && at2 < at)) {
-                    a = a2;
-                    at = at2;
-                }
-            }
-            float m = __shfl_sync(0xffffffffu, x[i], at);
-            if (a == 0.0f) m = 0.0f;   // an all-zero block (of either sign) has m = +0
-            const float d = __fdiv_rn(m, -8.0f);
-            const float id = d != 0.0f ? __frcp_rn(d) : 0.0f;
+        for (int off = 4; off > 0; off >>= 1) {
+            const float a2 = __shfl_xor_sync(0xffffffffu, a, off);
+            const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+            const int at2 = __shfl_xor_sync(0xffffffffu, at, off);
+            if (a2 > a || (a2 == a && at2 < at)) { a = a2; m = m2; at = at2; }
+        }
+        if (a == 0.0f) m = 0.0f;   // an all-zero block (of either sign) has m = +0
+        const float d = __fdiv_rn(m, -8.0f);
+        const float id = d != 0.0f ? __frcp_rn(d) : 0.0f;
+        uint32_t qw = 0;   // this lane's four codes, one per byte
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) {
             int q = __float2int_rz(__fadd_rn(__fmul_rn(x[i], id), 8.5f));
             q = q > 15 ? 15 : q;
-            const int hi = __shfl_down_sync(0xffffffffu, q, 16);
-            const uint32_t byte = static_cast<uint32_t>(q | (hi << 4)) & 0xFFu;   // qs[lane] for lane < 16
-            const uint32_t next = __shfl_down_sync(0xffffffffu, byte, 1);
+            qw |= static_cast<uint32_t>(q) << (8 * i);
+        }
+        // lane c < 4 holds codes 4c..4c+3 (low nibbles of qs bytes 4c..4c+3), lane c+4
+        // the codes 16+4c.. that go in the high nibbles of the same bytes
+        const uint32_t hiw = __shfl_down_sync(0xffffffffu, qw, 4);
+        if (live && c < 4) {
+            const uint32_t bytes = qw | (hiw << 4);
             uint16_t *blk = reinterpret_cast<uint16_t *>(W + b * kBlockBytes);
-            if (lane < 16 && (lane & 1) == 0) blk[1 + (lane >> 1)] = static_cast<uint16_t>(byte | (next << 8));
-            if (lane == 0) blk[0] = __half_as_ushort(__float2half_rn(d));
+            blk[1 + 2 * c] = static_cast<uint16_t>(bytes & 0xFFFFu);
+            blk[2 + 2 * c] = static_cast<uint16_t>(bytes >> 16);
+            if (c == 0) blk[0] = __half_as_ushort(__float2half_rn(d));
         }
     }
 }
@@ -122,7 +128,7 @@ cudaError_t launch_gather(const uint8_t *W, const int32_t *ids, float *out, int6
 cudaError_t launch_quantize(const float *X, uint8_t *W, int64_t N, int64_t K, const DeviceInfo &dev,
                             cudaStream_t s) {
     const int64_t nblocks = N * (K / 32);
-    quantize_kernel<<<grid_for((nblocks + kUnroll - 1) / kUnroll, dev.sm_count), 256, 0, s>>>(X, W, nblocks);
+    quantize_kernel<<<grid_for((nblocks + 3) / 4, dev.sm_count), 256, 0, s>>>(X, W, nblocks);
     return cudaGetLastError();
 }
 
