@@ -54,8 +54,9 @@ __global__ void gather_kernel(const uint8_t *__restrict__ W, const int32_t *__re
         } else if (b == 0 && c == 0) {
             atomicOr(err, (unsigned)Q4_DEVERR_BAD_INDEX);
         }
-        // weights 4cc..4cc+3 of the low (c < 4) or high (c >= 4) half of block b
-        reinterpret_cast<float4 *>(out + t * nb * 32 + b * 32)[c] = o;
+        // weights 4cc..4cc+3 of the low (c < 4) or high (c >= 4) half of block b; a
+        // streaming store: the rows are read by the next kernel, not by this one
+        __stcs(reinterpret_cast<float4 *>(out + t * nb * 32 + b * 32) + c, o);
     }
 }
 
