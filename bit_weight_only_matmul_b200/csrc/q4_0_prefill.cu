@@ -323,7 +323,8 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
                 if (n < P.N) {
                     #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        if (mb + j < P.M) P.Y[static_cast<int64_t>(mb + j) * P.N + n] = v[j];
+                        // streaming store: Y is not read again here, X and W tiles are
+                        if (mb + j < P.M) __stcs(P.Y + static_cast<int64_t>(mb + j) * P.N + n, v[j]);
                 }
             }
             tc_fence_before();
