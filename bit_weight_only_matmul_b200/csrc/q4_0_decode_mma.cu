@@ -43,16 +43,18 @@
 //  * the accumulators (two chains per n-tile) live across the whole item; at
 //    its end the group-1 warp hands its sums through shared memory to the
 //    group-0 warp of the same rows, which stores Y[m, n].
-// Split mode (M <= 8, between one item per SM and kMaxItems items): when a
-// launch has few items, whole items leave a tail -- one decoder layer at M=1
-// has 24 items of 32 stages next to 192 of 12, so the busiest CTA works 32
-// stages against a mean of 21.  The CTAs then run in clusters of two.  An
-// item longer than the mean load of a CTA is split: the two CTAs of a
-// cluster take its two halves, both first thing, and the second CTA's sums
-// reach the first through distributed shared memory before the first stores
-// Y.  The other items stay whole, each on one CTA.  The host deals the split
-// items to the clusters and then the whole items to the CTAs, longest first
-// onto the least loaded.
+// Split mode (M <= 8, up to kMaxItems items): when a launch has few items,
+// whole items leave a tail -- one decoder layer at M=1 has 24 items of 32
+// stages next to 192 of 12, so the busiest CTA works 32 stages against a
+// mean of 21 -- and with fewer items than SMs most SMs idle (a 3072 x 3072
+// GEMV has 24 items of 12 stages).  The CTAs then run in clusters of CL: two
+// when there is at least one item per SM, else 4, 6 or 8, whichever leaves
+// the least work on the busiest CTA.  An item longer than the mean load of
+// a CTA is split: the CL CTAs of a cluster take its CL pieces, all first
+// thing, and the sums of ranks 1..CL-1 reach rank 0 through distributed
+// shared memory before it stores Y.  The other items stay whole, each on
+// one CTA.  The host deals the split items to the clusters and then the
+// whole items to the CTAs, longest first onto the least loaded.
 // Launches use programmatic stream serialization: the next grid on the
 // stream may start as this grid's CTAs leave, and every CTA waits for the
 // previous grid before its first global access.
@@ -98,29 +100,32 @@ template <int NT> constexpr int raw_bytes() {   // one 256-k stage
 // 256-k stages per ring slot: two for M <= 8, so that every wait, arrival and
 // walk step of every warp covers 512 k (halving that overhead per byte)
 template <int NT> constexpr int subs() { return NT == 1 ? 2 : 1; }
-template <int NT> constexpr int ring() { return NT == 2 ? 6 : 4; }   // slots
+// ring slots; clusters of CL >= 4 (launches of few items, where a CTA works
+// a few stages) give part of the ring to the partner sums
+template <int NT, int CL> constexpr int ring() { return CL >= 6 ? 2 : CL == 4 ? 3 : NT == 2 ? 6 : 4; }
 
-// Partner sums in split mode: written remotely by CTA 1 of a cluster into
-// CTA 0's copy (two buffers, by item parity).
-template <int NT, bool SPLIT>
+// Partner sums in split mode: rank r > 0 of a cluster of CL writes its
+// sums remotely into slot r - 1 of rank 0's copy (two buffers, by item
+// parity).
+template <int NT, int CL>
 struct XComb {
-    float v[2][8][NT][4][32];
+    float v[2][CL - 1][8][NT][4][32];
     uint64_t full[2], empty[2];
 };
 template <int NT>
-struct XComb<NT, false> {};
+struct XComb<NT, 1> {};
 
-template <int NT, bool SPLIT>
+template <int NT, int CL>
 struct Smem {
-    uint8_t raw[ring<NT>()][subs<NT>()][raw_bytes<NT>()];   // per stage: W rows (pitch 144), X rows (pitch 528)
+    uint8_t raw[ring<NT, CL>()][subs<NT>()][raw_bytes<NT>()];   // per stage: W rows (pitch 144), X rows (pitch 528)
     uint2 xf[kXBufs][subs<NT>()][16][NT][32];               // B fragments: [stage][mma u][n tile][lane]
     float comb[8][NT][4][32];                   // group-1 sums handed to group 0 at an item's end
-    uint64_t raw_full[ring<NT>()], raw_empty[ring<NT>()];
+    uint64_t raw_full[ring<NT, CL>()], raw_empty[ring<NT, CL>()];
     uint64_t xf_full[kXBufs], xf_empty[kXBufs];
     uint64_t comb_full, comb_empty;
     float epi[4][NT][4][32];                    // SwiGLU: up-row sums handed to the gate rows
     uint64_t epi_full, epi_empty;
-    XComb<NT, SPLIT> x;
+    XComb<NT, CL> x;
     int abort_flag;
 };
 
@@ -236,18 +241,19 @@ __device__ __forceinline__ bool wait_cluster_or_abort(uint64_t *bar, uint32_t pa
     return true;
 }
 
-// One CTA's walk over its (item, stage) sequence.  Plain mode: the items dealt
-// to the CTAs in boustrophedon order.  Split mode: the CTA's list from the
-// host; of a split n-stage item rank 0 takes the first ceil(n/2) stages and
-// rank 1 the rest.
-template <bool SPLIT, int SUBS>
+// One CTA's walk over its (item, stage) sequence.  Plain mode (CL = 1): the
+// items dealt to the CTAs in boustrophedon order.  Split mode: the CTA's list
+// from the host; of a split n-stage item rank r of the cluster of CL takes
+// stages ceil(n r / CL) .. ceil(n (r + 1) / CL) - 1 (at least one: the host
+// splits only items of n >= CL stages).
+template <int CL, int SUBS>
 struct Walk {
     int round, idx, item, prob, row0, stage, end, cnt;   // this step covers stages [stage, stage + cnt)
     bool split;
     template <int CAP>
     __device__ __forceinline__ void load(const DecodeParams<CAP> &D, uint32_t rank) {
         const GroupParams<CAP> &P = D.g;
-        if constexpr (!SPLIT) {
+        if constexpr (CL == 1) {
             const int G = gridDim.x;
             const int pos = (round & 1) ? (G - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
             item = round * G + pos;
@@ -263,9 +269,8 @@ struct Walk {
             split = (e & kSplitFlag) != 0;
             prob = find_problem(P, item);
             const int n = P.p[prob].stages;
-            const int n0 = (n + 1) / 2;
-            stage = split && rank == 1 ? n0 : 0;
-            end = split && rank == 0 ? n0 : n;
+            stage = split ? (n * static_cast<int>(rank) + CL - 1) / CL : 0;
+            end = split ? (n * static_cast<int>(rank + 1) + CL - 1) / CL : n;
         }
         row0 = (item - P.p[prob].item_begin) * kItemRows;
         cnt = SUBS == 1 || end - stage >= SUBS ? SUBS : end - stage;   // every item has >= 1 stage here
@@ -274,7 +279,7 @@ struct Walk {
     __device__ __forceinline__ void start(const DecodeParams<CAP> &D, uint32_t rank) {
         round = 0;
         idx = 0;
-        if constexpr (SPLIT) idx = D.sched_begin[blockIdx.x];
+        if constexpr (CL > 1) idx = D.sched_begin[blockIdx.x];
         load(D, rank);
     }
     template <int CAP>
@@ -290,13 +295,13 @@ struct Walk {
     }
 };
 
-template <int NT, int CAP, bool SPLIT>
+template <int NT, int CAP, int CL>
 __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_constant__ DecodeParams<CAP> D) {
-    constexpr int RS = ring<NT>();
+    constexpr int RS = ring<NT, CL>();
     constexpr int SUB = subs<NT>();
     const GroupParams<CAP> &P = D.g;
     extern __shared__ uint8_t smem_raw[];
-    using SM = Smem<NT, SPLIT>;
+    using SM = Smem<NT, CL>;
     SM &S = *reinterpret_cast<SM *>(align_smem<1024>(smem_raw));   // swizzled X boxes want 1024
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -313,33 +318,47 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
         mbar_init(&S.comb_empty, kGroupWarps);
         mbar_init(&S.epi_full, kGroupWarps / 2);
         mbar_init(&S.epi_empty, kGroupWarps / 2);
-        if constexpr (SPLIT) {
+        if constexpr (CL > 1) {
             for (int s = 0; s < 2; ++s) {
-                mbar_init(&S.x.full[s], 32 * kGroupWarps);    // every thread of the partner's group 0
-                mbar_init(&S.x.empty[s], 32 * kGroupWarps);
+                mbar_init(&S.x.full[s], 32 * kGroupWarps * (CL - 1));   // every group-0 thread of ranks 1..CL-1
+                mbar_init(&S.x.empty[s], 32 * kGroupWarps);             // every group-0 thread of rank 0
             }
         }
         S.abort_flag = 0;
         fence_mbar_init();
     }
     uint32_t rank = 0;
-    if constexpr (SPLIT) {
+    if constexpr (CL > 1) {
         rank = cluster_rank();
         cluster_sync_all();   // the partner's barriers exist before anyone arrives on them
     } else {
         __syncthreads();
     }
     // Programmatic dependent launch: the next kernel on the stream may start
-    // its CTAs as this grid's CTAs leave the SMs, and this grid touches no
-    // global memory before the previous kernel on the stream has completed
-    // (both are no-ops for launches without the attribute).
+    // its CTAs as this grid's CTAs leave the SMs, and this grid reads nothing
+    // into the SM before the previous kernel on the stream has completed
+    // (both are no-ops for launches without the attribute).  Before that
+    // wait the producer only asks L2 for the weight tiles of the CTA's first
+    // ring of stages: L2 is where every SM's writes land, so a tile that the
+    // previous kernel still writes is current by the time this grid reads it.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (warp == kWarpProd && lane == 0) {
+        Walk<CL, SUB> q{};
+        q.start(D, rank);
+        int prob = -1;
+        for (int s = 0; s < RS && q.item >= 0; ++s, q.next(D, rank)) {
+            if (q.prob != prob) prefetch_tensormap(&P.wmap[q.prob]);
+            prob = q.prob;
+            for (int i = 0; i < q.cnt; ++i)
+                tma_prefetch_l2_2d(&P.wmap[q.prob], (q.stage + i) * kStageRowBytes, q.row0);
+        }
+    }
     asm volatile("griddepcontrol.wait;" ::: "memory");
     uint32_t prod_issued = 0;
 
     if (warp == kWarpProd) {
         // ---------------------------------------------------------------- loads
-        Walk<SPLIT, SUB> q{};
+        Walk<CL, SUB> q{};
         q.start(D, rank);
         for (; q.item >= 0; q.next(D, rank)) {
             const GroupProblem &pr = P.p[q.prob];
@@ -386,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
         const int G = warp - kWarpX0;
         const int gx = lane >> 2, tx = lane & 3;
         uint32_t g = 0;
-        Walk<SPLIT, SUB> q{};
+        Walk<CL, SUB> q{};
         q.start(D, rank);
         for (; q.item >= 0; q.next(D, rank), ++g) {
             if ((g & 1) != static_cast<uint32_t>(G)) continue;
@@ -444,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
             #pragma unroll
             for (int j = 0; j < NT; ++j) acc[c][j][0] = acc[c][j][1] = acc[c][j][2] = acc[c][j][3] = 0.f;
         uint32_t g = 0, items_done = 0, split_done = 0, swiglu_done = 0;
-        Walk<SPLIT, SUB> q{};
+        Walk<CL, SUB> q{};
         q.start(D, rank);
         for (; q.item >= 0; q.next(D, rank), ++g) {
             if ((g & 1) == static_cast<uint32_t>(G)) {
@@ -498,26 +517,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
                             sum[j][e] = acc[0][j][e] + acc[1][j][e] + S.comb[tile][j][e][lane];
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S.comb_empty);
-                    if constexpr (SPLIT) {
+                    if constexpr (CL > 1) {
                         if (q.split) {
-                            // rank 1 hands its sums to rank 0 of the cluster
+                            // ranks 1..CL-1 hand their sums to rank 0 of the cluster, which adds
+                            // them in rank order
                             const int xb2 = split_done & 1;
                             const uint32_t xpar = (split_done >> 1) & 1;
                             ++split_done;
-                            if (rank == 1) {
+                            if (rank != 0) {
                                 if (!wait_cluster_or_abort(&S.x.empty[xb2], xpar ^ 1, &S.abort_flag, P.err)) break;
                                 #pragma unroll
                                 for (int j = 0; j < NT; ++j)
                                     #pragma unroll
-                                    for (int e = 0; e < 4; ++e) st_remote(&S.x.v[xb2][tile][j][e][lane], 0, sum[j][e]);
+                                    for (int e = 0; e < 4; ++e)
+                                        st_remote(&S.x.v[xb2][rank - 1][tile][j][e][lane], 0, sum[j][e]);
                                 mbar_arrive_remote(&S.x.full[xb2], 0);
                             } else {
                                 if (!wait_cluster_or_abort(&S.x.full[xb2], xpar, &S.abort_flag, P.err)) break;
                                 #pragma unroll
-                                for (int j = 0; j < NT; ++j)
+                                for (int r = 0; r < CL - 1; ++r)
                                     #pragma unroll
-                                    for (int e = 0; e < 4; ++e) sum[j][e] += S.x.v[xb2][tile][j][e][lane];
-                                mbar_arrive_remote(&S.x.empty[xb2], 1);
+                                    for (int j = 0; j < NT; ++j)
+                                        #pragma unroll
+                                        for (int e = 0; e < 4; ++e) sum[j][e] += S.x.v[xb2][r][tile][j][e][lane];
+                                #pragma unroll
+                                for (int r = 1; r < CL; ++r) mbar_arrive_remote(&S.x.empty[xb2], r);
                             }
                         }
                     }
@@ -583,24 +607,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
             mbar_wait(&S.raw_full[gg % RS], (gg / RS) & 1, P.err);
         }
     }
-    if constexpr (SPLIT) {
+    if constexpr (CL > 1) {
         __syncthreads();
         cluster_sync_all();   // no CTA leaves while its partner may still reach its shared memory
     }
 }
 
-template <int NT, bool SPLIT>
-constexpr size_t smem_bytes() { return sizeof(Smem<NT, SPLIT>) + 1024; }
-static_assert(smem_bytes<4, false>() <= 232448, "shared memory budget");
-static_assert(smem_bytes<1, true>() <= 232448, "shared memory budget");
-static_assert(smem_bytes<2, false>() <= 232448, "shared memory budget");
+template <int NT, int CL>
+constexpr size_t smem_bytes() { return sizeof(Smem<NT, CL>) + 1024; }
+static_assert(smem_bytes<4, 1>() <= 232448, "shared memory budget");
+static_assert(smem_bytes<2, 1>() <= 232448, "shared memory budget");
+static_assert(smem_bytes<1, 2>() <= 232448, "shared memory budget");
+static_assert(smem_bytes<1, 4>() <= 232448, "shared memory budget");
+static_assert(smem_bytes<1, 6>() <= 232448, "shared memory budget");
+static_assert(smem_bytes<1, 8>() <= 232448, "shared memory budget");
 
-template <int NT, int CAP, bool SPLIT>
+template <int NT, int CAP, int CL>
 cudaError_t configure(const q4::DeviceInfo &dev) {
     static int configured_device = -1;
     if (configured_device == dev.device) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<NT, CAP, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem_bytes<NT, SPLIT>()));
+    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<NT, CAP, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem_bytes<NT, CL>()));
     if (e != cudaSuccess) return e;
     configured_device = dev.device;
     return cudaSuccess;
@@ -608,30 +635,31 @@ cudaError_t configure(const q4::DeviceInfo &dev) {
 
 template <int NT, int CAP>
 cudaError_t launch_plain(DecodeParams<CAP> &D, const q4::DeviceInfo &dev, cudaStream_t s) {
-    cudaError_t e = configure<NT, CAP, false>(dev);
+    cudaError_t e = configure<NT, CAP, 1>(dev);
     if (e != cudaSuccess) return e;
     const int grid = std::max(1, std::min(dev.sm_count, D.g.total_items));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem_bytes<NT, false>();
+    cfg.dynamicSmemBytes = smem_bytes<NT, 1>();
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_mma_kernel<NT, CAP, false>, D);
+    return cudaLaunchKernelEx(&cfg, decode_mma_kernel<NT, CAP, 1>, D);
 }
 
+template <int CL>
 cudaLaunchConfig_t cluster_config(int clusters, cudaStream_t s, cudaLaunchAttribute *attr) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * clusters, 1, 1);
+    cfg.gridDim = dim3(CL * clusters, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem_bytes<1, true>();
+    cfg.dynamicSmemBytes = smem_bytes<1, CL>();
     cfg.stream = s;
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.x = CL;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -641,100 +669,188 @@ cudaLaunchConfig_t cluster_config(int clusters, cudaStream_t s, cudaLaunchAttrib
     return cfg;
 }
 
-// Clusters of two that can be resident at once on this device (0 if none).
-template <int CAP>
+// Clusters of CL that can be resident at once on this device (0 if none).
+template <int CAP, int CL>
 int split_clusters(const q4::DeviceInfo &dev) {
     static int cached_device = -1, cached = 0;
     if (cached_device == dev.device) return cached;
     int n = 0;
-    if (configure<1, CAP, true>(dev) == cudaSuccess) {
+    if (configure<1, CAP, CL>(dev) == cudaSuccess) {
         cudaLaunchAttribute attr[2];
-        cudaLaunchConfig_t cfg = cluster_config(std::max(1, dev.sm_count / 2), nullptr, attr);
-        if (cudaOccupancyMaxActiveClusters(&n, decode_mma_kernel<1, CAP, true>, &cfg) != cudaSuccess) n = 0;
+        cudaLaunchConfig_t cfg = cluster_config<CL>(std::max(1, dev.sm_count / CL), nullptr, attr);
+        if (cudaOccupancyMaxActiveClusters(&n, decode_mma_kernel<1, CAP, CL>, &cfg) != cudaSuccess) n = 0;
     }
     (void)cudaGetLastError();
-    cached = std::min(n, kMaxSplitCtas / 2);
+    cached = std::min(n, kMaxSplitCtas / CL);
     cached_device = dev.device;
     return cached;
 }
 
-// The split-mode schedule.  Items longer than the mean load of a CTA are
-// split and dealt to the clusters (cost ceil(n/2) on each CTA of the pair);
-// each CTA's list starts with its cluster's split items, in the same order on
-// both CTAs.  The whole items follow, dealt to single CTAs; every deal puts
-// the next-longest item onto the least loaded cluster or CTA.
 template <int CAP>
-void build_schedule(DecodeParams<CAP> &D, int clusters) {
-    const GroupParams<CAP> &P = D.g;
-    const int ctas = 2 * clusters;
+int split_clusters(const q4::DeviceInfo &dev, int cl) {
+    switch (cl) {
+        case 2: return split_clusters<CAP, 2>(dev);
+        case 4: return split_clusters<CAP, 4>(dev);
+        case 6: return split_clusters<CAP, 6>(dev);
+        case 8: return split_clusters<CAP, 8>(dev);
+        default: return 0;
+    }
+}
+
+// A split-mode schedule.  Items of n >= CL stages that are longer than the
+// mean load of a CTA are split and dealt to the clusters (cost ceil(n/CL) on
+// each CTA of the cluster); each CTA's list starts with its cluster's split
+// items, in the same order on every CTA of the cluster.  The whole items
+// follow, dealt to single CTAs; every deal puts the next-longest item onto
+// the least loaded cluster or CTA.
+struct SplitSchedule {
+    std::vector<std::vector<uint16_t>> split_of, whole_of;
+    long max_load = 0;
+    int entries = 0;
+};
+
+template <int CAP>
+void plan_schedule(const GroupParams<CAP> &P, int clusters, int cl, SplitSchedule &out) {
+    const int ctas = cl * clusters;
     long total = 0;
     for (int i = 0; i < P.count; ++i) {
         const int nitems = (i + 1 < P.count ? P.p[i + 1].item_begin : P.total_items) - P.p[i].item_begin;
         total += static_cast<long>(nitems) * P.p[i].stages;
     }
     const long mean = (total + ctas - 1) / ctas;
+    auto is_split = [&](int n) { return n >= cl && n > mean; };
     using Load = std::pair<long, int>;
-    std::vector<std::vector<uint16_t>> split_of(clusters), whole_of(ctas);
+    out.split_of.assign(clusters, {});
+    out.whole_of.assign(ctas, {});
+    out.entries = 0;
     std::vector<long> load(ctas, 0);
-    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> cl;
-    for (int c = 0; c < clusters; ++c) cl.push({0, c});
+    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> cq;
+    for (int c = 0; c < clusters; ++c) cq.push({0, c});
     for (int i = 0; i < P.count; ++i) {   // problems come sorted by K, largest first
         const int n = P.p[i].stages;
-        if (n < 2 || n <= mean) continue;
+        if (!is_split(n)) continue;
         const int nitems = (i + 1 < P.count ? P.p[i + 1].item_begin : P.total_items) - P.p[i].item_begin;
         for (int k = 0; k < nitems; ++k) {
-            Load l = cl.top();
-            cl.pop();
-            split_of[l.second].push_back(static_cast<uint16_t>(P.p[i].item_begin + k));
-            l.first += (n + 1) / 2;
-            load[2 * l.second] = load[2 * l.second + 1] = l.first;
-            cl.push(l);
+            Load l = cq.top();
+            cq.pop();
+            out.split_of[l.second].push_back(static_cast<uint16_t>(P.p[i].item_begin + k));
+            out.entries += cl;
+            l.first += (n + cl - 1) / cl;
+            for (int r = 0; r < cl; ++r) load[cl * l.second + r] = l.first;
+            cq.push(l);
         }
     }
-    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> ct;
-    for (int b = 0; b < ctas; ++b) ct.push({load[b], b});
+    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> tq;
+    for (int b = 0; b < ctas; ++b) tq.push({load[b], b});
     for (int i = 0; i < P.count; ++i) {
         const int n = P.p[i].stages;
-        if (!(n < 2 || n <= mean)) continue;
+        if (is_split(n)) continue;
         const int nitems = (i + 1 < P.count ? P.p[i + 1].item_begin : P.total_items) - P.p[i].item_begin;
         for (int k = 0; k < nitems; ++k) {
-            Load l = ct.top();
-            ct.pop();
-            whole_of[l.second].push_back(static_cast<uint16_t>(P.p[i].item_begin + k));
+            Load l = tq.top();
+            tq.pop();
+            out.whole_of[l.second].push_back(static_cast<uint16_t>(P.p[i].item_begin + k));
+            ++out.entries;
             l.first += n;
-            ct.push(l);
+            load[l.second] = l.first;
+            tq.push(l);
         }
     }
+    out.max_load = *std::max_element(load.begin(), load.end());
+}
+
+template <int CAP>
+void write_schedule(DecodeParams<CAP> &D, int clusters, int cl, const SplitSchedule &sc) {
+    const int ctas = cl * clusters;
     int pos = 0;
     for (int b = 0; b < ctas; ++b) {
         D.sched_begin[b] = static_cast<uint16_t>(pos);
-        for (uint16_t it : split_of[b >> 1]) D.sched[pos++] = static_cast<uint16_t>(it | kSplitFlag);
-        for (uint16_t it : whole_of[b]) D.sched[pos++] = it;
+        for (uint16_t it : sc.split_of[b / cl]) D.sched[pos++] = static_cast<uint16_t>(it | kSplitFlag);
+        for (uint16_t it : sc.whole_of[b]) D.sched[pos++] = it;
     }
     D.sched_begin[ctas] = static_cast<uint16_t>(pos);
 }
 
-// The schedule depends only on the clusters and on each problem's stages and
-// item count; a call with the same shapes as the previous one on this thread
-// (the usual case: the same layer every token) keeps the schedule that `D`
-// still holds.
+// How an M <= 8 launch runs: plain (cl = 1) or in clusters of cl.
+struct SplitPlan {
+    int cl = 1, clusters = 0;
+};
+
+// Launches with at least one item per SM (up to kMaxItems) run in pairs: the
+// long items of a decoder layer are halved, the rest stay whole.  Launches
+// with fewer items than SMs leave most SMs idle in plain mode; there every
+// item can be cut into CL = 4, 6 or 8 pieces on the CTAs of one cluster,
+// and the cluster size with the least work on the busiest CTA is taken,
+// counting one stage for the hand-over of the partial sums, if that beats
+// one whole item per CTA.
+constexpr long kHandOverStages = 1;
+
 template <int CAP>
-cudaError_t launch_split(DecodeParams<CAP> &D, int clusters, cudaStream_t s) {
+SplitPlan choose_plan(DecodeParams<CAP> &D, const q4::DeviceInfo &dev) {
+    const GroupParams<CAP> &P = D.g;
+    SplitPlan best;
+    if (P.total_items > kMaxItems) return best;
+    static thread_local SplitSchedule sc, best_sc;
+    if (P.total_items >= dev.sm_count) {
+        const int clusters = std::min(split_clusters<CAP>(dev, 2), P.total_items);
+        if (clusters < 1) return best;
+        plan_schedule(P, clusters, 2, sc);
+        if (sc.entries > kMaxSched) return best;
+        best = {2, clusters};
+        write_schedule(D, clusters, 2, sc);
+        return best;
+    }
+    long best_cost = 0;
+    for (int i = 0; i < P.count; ++i) best_cost = std::max<long>(best_cost, P.p[i].stages);
+    for (int cl : {4, 6, 8}) {
+        const int clusters = std::min(split_clusters<CAP>(dev, cl), P.total_items);
+        if (clusters < 1) continue;
+        plan_schedule(P, clusters, cl, sc);
+        if (sc.entries > kMaxSched) continue;
+        const long cost = sc.max_load + kHandOverStages;
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = {cl, clusters};
+            std::swap(best_sc, sc);
+        }
+    }
+    if (best.cl > 1) write_schedule(D, best.clusters, best.cl, best_sc);
+    return best;
+}
+
+template <int CAP, int CL>
+cudaError_t launch_cluster(const DecodeParams<CAP> &D, int clusters, cudaStream_t s) {
+    cudaLaunchAttribute attr[2];
+    cudaLaunchConfig_t cfg = cluster_config<CL>(clusters, s, attr);
+    return cudaLaunchKernelEx(&cfg, decode_mma_kernel<1, CAP, CL>, D);
+}
+
+// The plan and schedule depend only on the device and on each problem's
+// stages and item count; a call with the same shapes as the previous one on
+// this thread (the usual case: the same layer every token) keeps the
+// schedule that `D` still holds.
+template <int CAP>
+cudaError_t launch_m8(DecodeParams<CAP> &D, const q4::DeviceInfo &dev, cudaStream_t s) {
     static thread_local std::vector<int> last;
+    static thread_local SplitPlan plan;
     thread_local std::vector<int> sig;
     const GroupParams<CAP> &P = D.g;
-    sig.assign({clusters, P.count, P.total_items});
+    sig.assign({dev.device, P.count, P.total_items});
     for (int i = 0; i < P.count; ++i) {
         sig.push_back(P.p[i].stages);
         sig.push_back(P.p[i].item_begin);
     }
     if (sig != last) {
-        build_schedule(D, clusters);
+        plan = choose_plan(D, dev);
         last = sig;
     }
-    cudaLaunchAttribute attr[2];
-    cudaLaunchConfig_t cfg = cluster_config(clusters, s, attr);
-    return cudaLaunchKernelEx(&cfg, decode_mma_kernel<1, CAP, true>, D);
+    switch (plan.cl) {
+        case 2: return launch_cluster<CAP, 2>(D, plan.clusters, s);
+        case 4: return launch_cluster<CAP, 4>(D, plan.clusters, s);
+        case 6: return launch_cluster<CAP, 6>(D, plan.clusters, s);
+        case 8: return launch_cluster<CAP, 8>(D, plan.clusters, s);
+        default: return launch_plain<1, CAP>(D, dev, s);
+    }
 }
 
 // problems[order[0..count)] sorted by K (largest first), count <= CAP
@@ -779,16 +895,7 @@ cudaError_t launch_cap(const q4::Problem *probs, const int *order, int count, co
             return cudaErrorInvalidValue;   // the caller sends M > 8 groups in chunks of kXMapCap
         }
     }
-    {
-        // fewer items than SMs: each CTA has at most one item and the launch is
-        // latency-bound, where the hand-over between a pair costs more than it
-        // saves (measured on a single 3072 x 3072 GEMV)
-        if (items >= dev.sm_count && items <= kMaxItems) {
-            const int clusters = std::min(split_clusters<CAP>(dev), items);
-            if (clusters >= 1) return launch_split<CAP>(D, clusters, s);
-        }
-        return launch_plain<1, CAP>(D, dev, s);
-    }
+    return launch_m8<CAP>(D, dev, s);
 }
 
 constexpr int kSmallCap = 8, kLargeCap = 128;

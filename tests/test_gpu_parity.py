@@ -267,6 +267,52 @@ def test_split_mode_mixed_stage_counts(q4):
     no_device_error(q4)
 
 
+@pytest.mark.parametrize("M,N,K", [
+    (1, 100, 8192),    # one 32-stage item: eight pieces of 4 (cluster of 8)
+    (2, 128, 1536),    # one 6-stage item: six pieces of 1 (cluster of 6; 8 would leave it whole)
+    (3, 90, 1024),     # one 4-stage item: four pieces of 1 (cluster of 4)
+    (8, 1000, 1792),   # eight 7-stage items in pieces of 2, 2, 2, 1 (clusters of 4)
+])
+def test_split_mode_few_items(q4, M, N, K):
+    """M <= 8 with fewer items than SMs: each item is cut into pieces on the
+    CTAs of one cluster (4, 6 or 8 of them), whose partial sums meet in rank
+    0 of the cluster.  The second call reuses the schedule of the first."""
+    rng = np.random.default_rng(M * 7 + N + K)
+    codes, scales, X = rand_inputs(rng, M, N, K)
+    W = pack_on_gpu(q4, codes, scales)
+    o = oracle.get()
+    Y_or, B_or = o.gemm(o.pack(codes, scales), X, M, N, K)
+    Y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    for rep in range(2):
+        Y.fill_(float("nan"))
+        q4.q4_0_gemm(W, dev(X), Y, M, N, K)
+        check_gemm(Y.cpu().numpy(), Y_or, B_or, f"few items M={M} N={N} K={K} rep {rep}")
+    no_device_error(q4)
+
+
+def test_split_mode_few_items_grouped(q4):
+    """A grouped launch of 14 items: the 32-, 8- and 7-stage items are cut
+    into pieces (the 7-stage ones unevenly), the 1-stage items stay whole,
+    and every problem's rows land in its own Y."""
+    o = oracle.get()
+    rng = np.random.default_rng(47)
+    shapes = [(2, 1000, 1792), (5, 300, 256), (8, 129, 8192), (1, 1, 2048)]
+    probs, refs, Ys = [], [], []
+    for (M, N, K) in shapes:
+        codes, scales, X = rand_inputs(rng, M, N, K)
+        Y = torch.full((M, N), float("nan"), device="cuda")
+        probs.append((pack_on_gpu(q4, codes, scales), dev(X), Y, M, N, K))
+        refs.append(o.gemm(o.pack(codes, scales), X, M, N, K))
+        Ys.append(Y)
+    for rep in range(2):
+        for Y in Ys:
+            Y.fill_(float("nan"))
+        q4.q4_0_gemm_grouped(probs)
+        for (M, N, K), Y, (Y_or, B_or) in zip(shapes, Ys, refs):
+            check_gemm(Y.cpu().numpy(), Y_or, B_or, f"few items grouped M={M} N={N} K={K} rep {rep}")
+    no_device_error(q4)
+
+
 def test_grouped_call_replays_from_cuda_graph(q4):
     """A grouped decode call captured in a CUDA graph (after one eager call,
     which does the per-device set-up) replays to the eager call's bits."""
