@@ -152,7 +152,10 @@ class ClockSampler:
 class GpuWorkload:
     """A workload resident in HBM: packed Q4_0 weights (packed on the GPU by
     q4_0_pack from seeded codes and scales), activations and outputs, in
-    `copies` independently seeded replicas."""
+    `copies` replicas at distinct addresses; the first SEEDS are seeded
+    independently, later ones repeat their values."""
+
+    SEEDS = 8
 
     def __init__(self, q4, wl: workloads.Workload, copies: int, seed: int):
         import torch
@@ -173,16 +176,22 @@ class GpuWorkload:
             probs = []
             xbuf = torch.zeros(x_total, dtype=torch.int16, device="cuda")
             ybuf = torch.empty(y_total, dtype=torch.float32, device="cuda")
-            for lin, xo, yo in zip(wl.linears, x_off, y_off):
+            for li, (lin, xo, yo) in enumerate(zip(wl.linears, x_off, y_off)):
+                X = xbuf[xo:xo + lin.M * lin.K].view(lin.M, lin.K)
+                Y = ybuf[yo:yo + lin.M * lin.N].view(lin.M, lin.N)
+                if c >= self.SEEDS:   # same values as copy c % SEEDS, in fresh buffers
+                    W0, X0 = self.sets[c % self.SEEDS][0][li][:2]
+                    W = W0.clone()
+                    X.copy_(X0)
+                    probs.append((W, X, Y, lin.M, lin.N, lin.K))
+                    continue
                 s = seed + 7919 * c
                 codes = torch.from_numpy(lin.codes(s)).cuda()
                 scales = torch.from_numpy(lin.scales(s).view(np.int16)).cuda()
                 W = torch.empty(q4.q4_0_bytes(lin.N, lin.K), dtype=torch.uint8, device="cuda")
                 q4.q4_0_pack(codes, scales, W, lin.N, lin.K)
                 del codes, scales
-                X = xbuf[xo:xo + lin.M * lin.K].view(lin.M, lin.K)
                 X.copy_(torch.from_numpy(lin.x(s).view(np.int16)))
-                Y = ybuf[yo:yo + lin.M * lin.N].view(lin.M, lin.N)
                 probs.append((W, X, Y, lin.M, lin.N, lin.K))
             self.sets.append((probs, q4.make_problems(probs)))
             self.xbufs.append(xbuf)
@@ -253,8 +262,9 @@ def run_ours(args, rank: int, world: int):
     tensor = args.workload in TENSOR_WORKLOADS
     step_bytes = wl.hbm_bytes
     step_flops = wl.flops
+    # rotating copies whose operands together exceed twice the L2, so that
+    # every step's operands come from HBM, not L2 (a 3072 x 3072 GEMV needs 48)
     copies = max(1, -(-2 * L2_BYTES // max(1, wl.weight_bytes + sum(l.act_bytes for l in wl.linears))))
-    copies = min(copies, 8)   # rotating copies: every step's operands come from HBM, not L2
     log(f"[rank {rank}] building {wl.name}: {len(wl.linears)} GEMMs x {copies} copies, "
         f"{step_bytes / 1e6:.1f} MB per step")
     G = GpuWorkload(q4, wl, copies, workloads.SEED + 1000 * rank)
