@@ -65,13 +65,12 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
-#include <queue>
-#include <utility>
 #include <vector>
 
 #include "q4_0_convert.cuh"
 #include "q4_0_internal.cuh"
 #include "q4_0_sched.cuh"
+#include "q4_0_split_plan.h"
 #include "q4_0_tcgen05.cuh"
 #include "q4_0_tmap.cuh"
 
@@ -85,10 +84,10 @@ constexpr int kXPitch = kXRow + 16;                 // skews consecutive X rows 
 constexpr int kXBufs = 4;                           // buffer g mod 4 belongs to group g mod 2
 constexpr int kWarpProd = 0, kWarpX0 = 1, kWarp0 = 3, kGroupWarps = 8;
 constexpr int kThreads = 32 * (kWarp0 + 2 * kGroupWarps);  // 608
-constexpr int kMaxItems = 1024;                     // items per launch in split mode
-constexpr int kMaxSplitCtas = 256;
-constexpr int kMaxSched = 2 * kMaxItems;            // schedule entries (a split item has two)
-constexpr uint16_t kSplitFlag = 0x8000;
+using q4split::kMaxItems;
+using q4split::kMaxSched;
+using q4split::kMaxSplitCtas;
+using q4split::kSplitFlag;
 
 // NT = n8 tiles of X rows (M <= 8*NT)
 // X by TMA boxes (M > 8): four boxes of 64 k x 8*NT rows, 128 bytes a row
@@ -185,7 +184,7 @@ struct DecodeParams {
     GroupParams<CAP> g;
     CUtensorMap xmap[CAP <= kXMapCap ? CAP : 1];   // M > 8: X as bf16 [M, K], box 64 x 8*NT, 128-byte swizzle
     // split mode: CTA b runs sched[sched_begin[b] .. sched_begin[b+1]), each
-    // entry an item index, with kSplitFlag set for a half of a split item
+    // entry an item index, with kSplitFlag set for a piece of a split item
     uint16_t sched_begin[kMaxSplitCtas + 1];
     uint16_t sched[kMaxSched];
 };
@@ -226,7 +225,7 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
     return ok != 0;
 }
 
-// wait_or_abort for a barrier that the partner CTA arrives on.
+// wait_or_abort for a barrier that another CTA of the cluster arrives on.
 __device__ __forceinline__ bool wait_cluster_or_abort(uint64_t *bar, uint32_t parity, int *abort_flag,
                                                       unsigned *err) {
     const unsigned long long t0 = global_ns();
@@ -269,8 +268,8 @@ struct Walk {
             split = (e & kSplitFlag) != 0;
             prob = find_problem(P, item);
             const int n = P.p[prob].stages;
-            stage = split ? (n * static_cast<int>(rank) + CL - 1) / CL : 0;
-            end = split ? (n * static_cast<int>(rank + 1) + CL - 1) / CL : n;
+            stage = split ? q4split::piece_begin(n, static_cast<int>(rank), CL) : 0;
+            end = split ? q4split::piece_begin(n, static_cast<int>(rank) + 1, CL) : n;
         }
         row0 = (item - P.p[prob].item_begin) * kItemRows;
         cnt = SUBS == 1 || end - stage >= SUBS ? SUBS : end - stage;   // every item has >= 1 stage here
@@ -330,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
     uint32_t rank = 0;
     if constexpr (CL > 1) {
         rank = cluster_rank();
-        cluster_sync_all();   // the partner's barriers exist before anyone arrives on them
+        cluster_sync_all();   // every CTA's barriers exist before any other CTA arrives on them
     } else {
         __syncthreads();
     }
@@ -609,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
     }
     if constexpr (CL > 1) {
         __syncthreads();
-        cluster_sync_all();   // no CTA leaves while its partner may still reach its shared memory
+        cluster_sync_all();   // no CTA leaves while another CTA of the cluster may still reach its shared memory
     }
 }
 
@@ -697,80 +696,6 @@ int split_clusters(const q4::DeviceInfo &dev, int cl) {
     }
 }
 
-// A split-mode schedule.  Items of n >= CL stages that are longer than the
-// mean load of a CTA are split and dealt to the clusters (cost ceil(n/CL) on
-// each CTA of the cluster); each CTA's list starts with its cluster's split
-// items, in the same order on every CTA of the cluster.  The whole items
-// follow, dealt to single CTAs; every deal puts the next-longest item onto
-// the least loaded cluster or CTA.
-struct SplitSchedule {
-    std::vector<std::vector<uint16_t>> split_of, whole_of;
-    long max_load = 0;
-    int entries = 0;
-};
-
-template <int CAP>
-void plan_schedule(const GroupParams<CAP> &P, int clusters, int cl, SplitSchedule &out) {
-    const int ctas = cl * clusters;
-    long total = 0;
-    for (int i = 0; i < P.count; ++i) {
-        const int nitems = (i + 1 < P.count ? P.p[i + 1].item_begin : P.total_items) - P.p[i].item_begin;
-        total += static_cast<long>(nitems) * P.p[i].stages;
-    }
-    const long mean = (total + ctas - 1) / ctas;
-    auto is_split = [&](int n) { return n >= cl && n > mean; };
-    using Load = std::pair<long, int>;
-    out.split_of.assign(clusters, {});
-    out.whole_of.assign(ctas, {});
-    out.entries = 0;
-    std::vector<long> load(ctas, 0);
-    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> cq;
-    for (int c = 0; c < clusters; ++c) cq.push({0, c});
-    for (int i = 0; i < P.count; ++i) {   // problems come sorted by K, largest first
-        const int n = P.p[i].stages;
-        if (!is_split(n)) continue;
-        const int nitems = (i + 1 < P.count ? P.p[i + 1].item_begin : P.total_items) - P.p[i].item_begin;
-        for (int k = 0; k < nitems; ++k) {
-            Load l = cq.top();
-            cq.pop();
-            out.split_of[l.second].push_back(static_cast<uint16_t>(P.p[i].item_begin + k));
-            out.entries += cl;
-            l.first += (n + cl - 1) / cl;
-            for (int r = 0; r < cl; ++r) load[cl * l.second + r] = l.first;
-            cq.push(l);
-        }
-    }
-    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> tq;
-    for (int b = 0; b < ctas; ++b) tq.push({load[b], b});
-    for (int i = 0; i < P.count; ++i) {
-        const int n = P.p[i].stages;
-        if (is_split(n)) continue;
-        const int nitems = (i + 1 < P.count ? P.p[i + 1].item_begin : P.total_items) - P.p[i].item_begin;
-        for (int k = 0; k < nitems; ++k) {
-            Load l = tq.top();
-            tq.pop();
-            out.whole_of[l.second].push_back(static_cast<uint16_t>(P.p[i].item_begin + k));
-            ++out.entries;
-            l.first += n;
-            load[l.second] = l.first;
-            tq.push(l);
-        }
-    }
-    out.max_load = *std::max_element(load.begin(), load.end());
-}
-
-template <int CAP>
-void write_schedule(DecodeParams<CAP> &D, int clusters, int cl, const SplitSchedule &sc) {
-    const int ctas = cl * clusters;
-    int pos = 0;
-    for (int b = 0; b < ctas; ++b) {
-        D.sched_begin[b] = static_cast<uint16_t>(pos);
-        for (uint16_t it : sc.split_of[b / cl]) D.sched[pos++] = static_cast<uint16_t>(it | kSplitFlag);
-        for (uint16_t it : sc.whole_of[b]) D.sched[pos++] = it;
-    }
-    D.sched_begin[ctas] = static_cast<uint16_t>(pos);
-}
-
 // How an M <= 8 launch runs: plain (cl = 1) or in clusters of cl.
 struct SplitPlan {
     int cl = 1, clusters = 0;
@@ -790,14 +715,19 @@ SplitPlan choose_plan(DecodeParams<CAP> &D, const q4::DeviceInfo &dev) {
     const GroupParams<CAP> &P = D.g;
     SplitPlan best;
     if (P.total_items > kMaxItems) return best;
-    static thread_local SplitSchedule sc, best_sc;
+    static thread_local std::vector<q4split::PlanProblem> pp;
+    static thread_local q4split::Schedule sc, best_sc;
+    pp.resize(P.count);
+    for (int i = 0; i < P.count; ++i)
+        pp[i] = {P.p[i].stages, P.p[i].item_begin,
+                 (i + 1 < P.count ? P.p[i + 1].item_begin : P.total_items) - P.p[i].item_begin};
     if (P.total_items >= dev.sm_count) {
         const int clusters = std::min(split_clusters<CAP>(dev, 2), P.total_items);
         if (clusters < 1) return best;
-        plan_schedule(P, clusters, 2, sc);
+        q4split::plan(pp.data(), P.count, clusters, 2, sc);
         if (sc.entries > kMaxSched) return best;
         best = {2, clusters};
-        write_schedule(D, clusters, 2, sc);
+        q4split::write(sc, clusters, 2, D.sched_begin, D.sched);
         return best;
     }
     long best_cost = 0;
@@ -805,7 +735,7 @@ SplitPlan choose_plan(DecodeParams<CAP> &D, const q4::DeviceInfo &dev) {
     for (int cl : {4, 6, 8}) {
         const int clusters = std::min(split_clusters<CAP>(dev, cl), P.total_items);
         if (clusters < 1) continue;
-        plan_schedule(P, clusters, cl, sc);
+        q4split::plan(pp.data(), P.count, clusters, cl, sc);
         if (sc.entries > kMaxSched) continue;
         const long cost = sc.max_load + kHandOverStages;
         if (cost < best_cost) {
@@ -814,7 +744,7 @@ SplitPlan choose_plan(DecodeParams<CAP> &D, const q4::DeviceInfo &dev) {
             std::swap(best_sc, sc);
         }
     }
-    if (best.cl > 1) write_schedule(D, best.clusters, best.cl, best_sc);
+    if (best.cl > 1) q4split::write(best_sc, best.clusters, best.cl, D.sched_begin, D.sched);
     return best;
 }
 
