@@ -309,13 +309,12 @@ template <int NT, int RT>
 cudaError_t launch_nt(DecodeParams &P, const q4::DeviceInfo &dev, cudaStream_t s) {
     const size_t smem = static_cast<size_t>(kWarps) * kStages * stage_bytes<RT>() +
                         static_cast<size_t>(kWarps) * kStages * sizeof(uint64_t);
-    static int configured_device = -1;   // per process; re-set when the device changes
-    if (configured_device != dev.device) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<NT, RT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-        configured_device = dev.device;
-    }
+    static q4::DeviceOnce configured;
+    cudaError_t e = configured.run(dev.device, [&] {
+        return cudaFuncSetAttribute(decode_kernel<NT, RT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(smem));
+    });
+    if (e != cudaSuccess) return e;
     P.rows_per_item = 16 * RT;
     // item boundaries per problem
     int items = 0;

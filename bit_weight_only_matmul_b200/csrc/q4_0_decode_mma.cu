@@ -623,13 +623,11 @@ static_assert(smem_bytes<1, 8>() <= 232448, "shared memory budget");
 
 template <int NT, int CAP, int CL>
 cudaError_t configure(const q4::DeviceInfo &dev) {
-    static int configured_device = -1;
-    if (configured_device == dev.device) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<NT, CAP, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem_bytes<NT, CL>()));
-    if (e != cudaSuccess) return e;
-    configured_device = dev.device;
-    return cudaSuccess;
+    static q4::DeviceOnce configured;
+    return configured.run(dev.device, [] {
+        return cudaFuncSetAttribute(decode_mma_kernel<NT, CAP, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(smem_bytes<NT, CL>()));
+    });
 }
 
 template <int NT, int CAP>
@@ -671,18 +669,17 @@ cudaLaunchConfig_t cluster_config(int clusters, cudaStream_t s, cudaLaunchAttrib
 // Clusters of CL that can be resident at once on this device (0 if none).
 template <int CAP, int CL>
 int split_clusters(const q4::DeviceInfo &dev) {
-    static int cached_device = -1, cached = 0;
-    if (cached_device == dev.device) return cached;
-    int n = 0;
-    if (configure<1, CAP, CL>(dev) == cudaSuccess) {
-        cudaLaunchAttribute attr[2];
-        cudaLaunchConfig_t cfg = cluster_config<CL>(std::max(1, dev.sm_count / CL), nullptr, attr);
-        if (cudaOccupancyMaxActiveClusters(&n, decode_mma_kernel<1, CAP, CL>, &cfg) != cudaSuccess) n = 0;
-    }
-    (void)cudaGetLastError();
-    cached = std::min(n, kMaxSplitCtas / CL);
-    cached_device = dev.device;
-    return cached;
+    static q4::DeviceValue cached;
+    return cached.get(dev.device, [&] {
+        int n = 0;
+        if (configure<1, CAP, CL>(dev) == cudaSuccess) {
+            cudaLaunchAttribute attr[2];
+            cudaLaunchConfig_t cfg = cluster_config<CL>(std::max(1, dev.sm_count / CL), nullptr, attr);
+            if (cudaOccupancyMaxActiveClusters(&n, decode_mma_kernel<1, CAP, CL>, &cfg) != cudaSuccess) n = 0;
+        }
+        (void)cudaGetLastError();
+        return std::max(0, std::min(n, kMaxSplitCtas / CL));
+    });
 }
 
 template <int CAP>

@@ -398,13 +398,12 @@ constexpr size_t smem_bytes() { return sizeof(Smem<NN>) + 1024; }
 
 template <int NN, int CAP>
 cudaError_t launch_nn(TParams<CAP> &P, const q4::DeviceInfo &dev, cudaStream_t s) {
-    static int configured_device = -1;
-    if (configured_device != dev.device) {
-        cudaError_t e = cudaFuncSetAttribute(decode_tmem_kernel<NN, CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem_bytes<NN>()));
-        if (e != cudaSuccess) return e;
-        configured_device = dev.device;
-    }
+    static q4::DeviceOnce configured;
+    cudaError_t e = configured.run(dev.device, [] {
+        return cudaFuncSetAttribute(decode_tmem_kernel<NN, CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(smem_bytes<NN>()));
+    });
+    if (e != cudaSuccess) return e;
     const int grid = std::max(1, std::min(dev.sm_count, P.total_items));
     decode_tmem_kernel<NN, CAP><<<grid, kThreads, smem_bytes<NN>(), s>>>(P);
     return cudaGetLastError();

@@ -2,6 +2,7 @@
 // and small sm_100a device helpers (mbarrier waits with a bound, bulk copies).
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -26,6 +27,45 @@ struct DeviceInfo {
     int cc_major, cc_minor;
     size_t smem_optin;         // max dynamic shared memory per block (opt-in)
     unsigned *err;             // device address of the error word
+};
+
+// A set-up step done once per device (device indices are below 64, which the
+// API layer checks): one bit per device, set once the step succeeded.  Two
+// threads that come first at the same time may both run it; every step
+// guarded this way is idempotent.
+class DeviceOnce {
+  public:
+    template <class F>
+    cudaError_t run(int device, F &&step) {
+        const uint64_t bit = uint64_t{1} << (device & 63);
+        if (done_.load(std::memory_order_acquire) & bit) return cudaSuccess;
+        const cudaError_t e = step();
+        if (e == cudaSuccess) done_.fetch_or(bit, std::memory_order_release);
+        return e;
+    }
+
+  private:
+    std::atomic<uint64_t> done_{0};
+};
+
+// A non-negative per-device figure computed once (same rules as DeviceOnce).
+class DeviceValue {
+  public:
+    DeviceValue() {
+        for (auto &v : v_) v.store(-1, std::memory_order_relaxed);
+    }
+    template <class F>
+    int get(int device, F &&compute) {
+        std::atomic<int> &slot = v_[device & 63];
+        int v = slot.load(std::memory_order_acquire);
+        if (v >= 0) return v;
+        v = compute();
+        slot.store(v, std::memory_order_release);
+        return v;
+    }
+
+  private:
+    std::atomic<int> v_[64];
 };
 
 // Launchers (host).  Each returns a cudaError_t from the launch.

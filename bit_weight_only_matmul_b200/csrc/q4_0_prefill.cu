@@ -398,22 +398,20 @@ cudaError_t launch_prefill(const Problem &p, const DeviceInfo &dev, cudaStream_t
     const int tiles = local.tiles_n * local.tiles_m;
     const int grid = tiles < dev.sm_count ? tiles : dev.sm_count;
     if (xpre) {
-        static int configured_device = -1;
-        if (configured_device != dev.device) {
-            cudaError_t e = cudaFuncSetAttribute(prefill_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(kSmemBytes));
-            if (e != cudaSuccess) return e;
-            configured_device = dev.device;
-        }
+        static q4::DeviceOnce configured;
+        cudaError_t e = configured.run(dev.device, [] {
+            return cudaFuncSetAttribute(prefill_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(kSmemBytes));
+        });
+        if (e != cudaSuccess) return e;
         prefill_kernel<true><<<grid, threads<true>(), kSmemBytes, s>>>(local);
     } else {
-        static int configured_device = -1;
-        if (configured_device != dev.device) {
-            cudaError_t e = cudaFuncSetAttribute(prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(kSmemBytes));
-            if (e != cudaSuccess) return e;
-            configured_device = dev.device;
-        }
+        static q4::DeviceOnce configured;
+        cudaError_t e = configured.run(dev.device, [] {
+            return cudaFuncSetAttribute(prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(kSmemBytes));
+        });
+        if (e != cudaSuccess) return e;
         prefill_kernel<false><<<grid, threads<false>(), kSmemBytes, s>>>(local);
     }
     return cudaGetLastError();
