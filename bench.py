@@ -253,6 +253,14 @@ class GpuWorkload:
             q4.q4_0_gemm_ws(W, X, Y, M, N, K, self.ws)
 
 
+def rotating_copies(wl: workloads.Workload) -> int:
+    """Copies of a step's operands that together exceed twice the L2, so
+    that every step's operands come from HBM, not L2 (one decoder layer: 5; a
+    3072 x 3072 GEMV: 50)."""
+    step = wl.weight_bytes + sum(l.act_bytes for l in wl.linears)
+    return max(1, -(-2 * L2_BYTES // max(1, step)))
+
+
 def run_ours(args, rank: int, world: int):
     import torch
     import torch.distributed as dist
@@ -262,9 +270,7 @@ def run_ours(args, rank: int, world: int):
     tensor = args.workload in TENSOR_WORKLOADS
     step_bytes = wl.hbm_bytes
     step_flops = wl.flops
-    # rotating copies whose operands together exceed twice the L2, so that
-    # every step's operands come from HBM, not L2 (a 3072 x 3072 GEMV needs 48)
-    copies = max(1, -(-2 * L2_BYTES // max(1, wl.weight_bytes + sum(l.act_bytes for l in wl.linears))))
+    copies = rotating_copies(wl)
     log(f"[rank {rank}] building {wl.name}: {len(wl.linears)} GEMMs x {copies} copies, "
         f"{step_bytes / 1e6:.1f} MB per step")
     G = GpuWorkload(q4, wl, copies, workloads.SEED + 1000 * rank)
@@ -446,16 +452,17 @@ def util_setup(q4, name: str, seed: int):
             codes = torch.from_numpy(workloads.gen_codes(rows, D, seed, layer=r0 // rows)).cuda()
             scales = torch.from_numpy(workloads.gen_scales(rows, D, seed, layer=r0 // rows).view(np.int16)).cuda()
             q4.q4_0_pack(codes, scales, W[r0 * (D // 32) * 18:(r0 + rows) * (D // 32) * 18], rows, D)
-        ids = [torch.from_numpy(workloads.gen_ids(T, V, seed, stream=i)).cuda() for i in range(4)]
+        # 32 id sets: a set's rows come back after 31 other steps (1.8 GB of traffic), not from L2
+        ids = [torch.from_numpy(workloads.gen_ids(T, V, seed, stream=i)).cuda() for i in range(32)]
         outs = [torch.empty((T, D), device="cuda") for _ in range(2)]
         hid = torch.empty(T, dtype=torch.int32, pin_memory=True).copy_(ids[0].cpu())
         hout = torch.empty((T, D), dtype=torch.float32, pin_memory=True)
 
         def launch(k):
-            q4.q4_0_gather(W, ids[k % 4], outs[k % 2], T, V, D)
+            q4.q4_0_gather(W, ids[k % len(ids)], outs[k % 2], T, V, D)
 
         def e2e(k):
-            ids[k % 4].copy_(hid, non_blocking=True)
+            ids[k % len(ids)].copy_(hid, non_blocking=True)
             launch(k)
             hout.copy_(outs[k % 2], non_blocking=True)
 
@@ -570,7 +577,9 @@ def run_util(args, rank: int, world: int):
         "data": "synthetic (seeded Philox)",
         "config": {"workload": f"{args.workload}: {workloads.UTIL_WORKLOADS[args.workload]}",
                    "bytes_per_step": step_bytes,
-                   "l2": "inputs larger than L2 (the 216 MiB table / 201 MB of fp32 weights), rotating buffers",
+                   "l2": ("inputs larger than L2: the 216 MiB table gathered through 32 rotating id sets"
+                          if args.workload == "embed" else
+                          "inputs larger than L2: 2 rotating 201 MB fp32 weight buffers"),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU", "launch": "eager"},
         "roofline": {"bound": "hbm", "kernel": kernel, "achieved": round(value / world, 2),
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(value / world / peaks["hbm_gbs"], 4),

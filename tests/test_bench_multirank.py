@@ -60,3 +60,19 @@ def test_workload_byte_accounting():
     cfg = workloads.workload("cfg_decode")
     assert cfg.hbm_bytes == 1479761920
     assert workloads.workload("adapter").flops == 2 * 4096 * 3072 * 5120
+
+
+def test_rotating_copies_exceed_l2():
+    """Every bench workload rotates enough copies of its step's operands that
+    they come from HBM: more than twice the 126 MiB L2 in all, as the bench
+    line's `l2` field states (a 3072 x 3072 GEMV needs 50 copies)."""
+    import bench
+    import workloads
+    for name in workloads.WORKLOADS:
+        wl = workloads.workload(name)
+        step = wl.weight_bytes + sum(l.act_bytes for l in wl.linears)
+        c = bench.rotating_copies(wl)
+        assert c * step >= 2 * bench.L2_BYTES, name
+        assert c == 1 or (c - 1) * step < 2 * bench.L2_BYTES, name   # no more than needed
+    assert bench.rotating_copies(workloads.workload("gemv")) == 50
+    assert bench.rotating_copies(workloads.workload("layer")) == 5
