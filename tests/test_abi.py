@@ -151,3 +151,33 @@ def test_grouped_ex_argument_checks(q4):
 def test_selftest_argument_checks(q4):
     assert q4.lib.q4_0_selftest_wait_timeout(0, None) == q4.Q4_ERR_INVALID_ARG
     assert q4.lib.q4_0_selftest_wait_timeout(1000001, None) == q4.Q4_ERR_INVALID_ARG
+
+
+def test_header_is_plain_c_and_matches_the_binding(q4, tmp_path):
+    """include/q4_0.h compiles as C99 with no CUDA header, and the problem
+    structs the binding builds with ctypes have the C layout: same size, same
+    field offsets."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("needs gcc")
+    fields = {"q4_0_problem": ["W", "X", "Y", "M", "N", "K"],
+              "q4_0_problem_ex": ["W", "X", "Y", "M", "N", "K", "R", "epilogue"]}
+    lines = ['#include <stddef.h>', '#include <stdio.h>', '#include "q4_0.h"', "int main(void) {"]
+    for st, fs in fields.items():
+        lines.append(f'    printf("{st} size %zu\\n", sizeof({st}));')
+        for f in fs:
+            lines.append(f'    printf("{st} {f} %zu\\n", offsetof({st}, {f}));')
+    lines += ["    return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = str(tmp_path / "layout")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", f"-I{os.path.join(ROOT, 'include')}",
+                    str(src), "-o", exe], check=True)
+    out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split("\n")
+    got = {tuple(l.split()[:2]): int(l.split()[2]) for l in out if l.strip()}
+    for st, fs in fields.items():
+        cls = getattr(q4, st)
+        assert got[(st, "size")] == ctypes.sizeof(cls), st
+        for f in fs:
+            assert got[(st, f)] == getattr(cls, f).offset, (st, f)
