@@ -14,8 +14,8 @@ def pytest_configure(config):
 
 def pytest_collection_modifyitems(config, items):
     # GPU tests must not silently pass on a machine without a GPU: skip them
-    # there (the driver selects them with -m gpu on a GPU machine, where the
-    # library's own loader raises if the CUDA extension is missing).
+    # there (`-m gpu` selects them on a B200, where the library's own loader
+    # raises if the CUDA extension is missing).
     try:
         import torch
         have_gpu = torch.cuda.is_available()
