@@ -76,3 +76,18 @@ def test_rotating_copies_exceed_l2():
         assert c == 1 or (c - 1) * step < 2 * bench.L2_BYTES, name   # no more than needed
     assert bench.rotating_copies(workloads.workload("gemv")) == 50
     assert bench.rotating_copies(workloads.workload("layer")) == 5
+
+
+def test_cpu_baselines_single_and_all_cores():
+    """The bench's two oracle baselines on a GEMV sample: one host core, and
+    the columns dealt to two threads (the oracle call releases the GIL)."""
+    import bench
+    import workloads
+    wl = workloads.workload("gemv")
+    host = bench.pack_on_host(wl, workloads.SEED)
+    one = bench.cpu_baseline(wl, False, 0.5, host=host)
+    two = bench.cpu_baseline_all_cores(wl, False, 0.5, threads=2, host=host)
+    assert one["cores"] == 1 and two["cores"] == 2
+    assert one["unit"] == two["unit"] == "GB/s"
+    assert one["value"] > 0 and two["value"] > 0
+    assert one["kind"] == two["kind"] == "oracle"
