@@ -365,13 +365,20 @@ bool prefill_supports(const Problem &p) {
            (reinterpret_cast<uintptr_t>(p.X) & 15) == 0 && tensor_maps_available();
 }
 
+// Bytes the fp16 conversion of X writes into a workspace: M*K*2, rounded up
+// to 256, whatever M is (a forced tensor-core run of an M <= 32 problem
+// converts too).
+static int64_t x_conversion_bytes(const Problem &p) { return ((p.M * p.K * 2 + 255) / 256) * 256; }
+
 int64_t prefill_workspace_bytes(const Problem &p) {
-    return p.M > 32 ? ((p.M * p.K * 2 + 255) / 256) * 256 : 0;
+    return p.M > 32 ? x_conversion_bytes(p) : 0;
 }
 
 cudaError_t launch_prefill(const Problem &p, const DeviceInfo &dev, cudaStream_t s, void *workspace,
                            int64_t workspace_bytes) {
-    const bool xpre = workspace != nullptr && workspace_bytes >= prefill_workspace_bytes(p) &&
+    // the pre-pass runs only when the workspace holds everything it writes;
+    // otherwise the kernel converts each X tile in shared memory
+    const bool xpre = workspace != nullptr && workspace_bytes >= x_conversion_bytes(p) &&
                       (reinterpret_cast<uintptr_t>(workspace) & 15) == 0;
     PrefillParams local;
     std::memset(&local, 0, sizeof(local));

@@ -137,7 +137,9 @@ Q4_0_API int64_t q4_0_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
  * q4_0_gemm_workspace_size(M, N, K), the tensor-core path (M > 32) first
  * converts X to fp16 once in the workspace (one extra read and write of X)
  * instead of converting every X tile in every CTA that loads it; with a
- * smaller or NULL workspace it behaves exactly as q4_0_gemm.  Same results,
+ * smaller or NULL workspace it behaves exactly as q4_0_gemm.  The library
+ * never writes past workspace_bytes: the conversion runs only when the
+ * workspace holds all M*K*2 bytes (rounded up to 256) that it writes.  Same results,
  * bit for bit, either way.  Calls that share one workspace and overlap on
  * the GPU race.  The pages have no counterpart: this is the B200 path's own
  * trade of one pass over X against per-tile conversion work. */
@@ -151,14 +153,23 @@ Q4_0_API int q4_0_gemm_ws(const void *W, const uint16_t *X, float *Y,
 #define Q4_0_STATIC_WS_BYTES (64LL << 20)
 
 /* q4_0_gemm_ws with the library's own fixed scratch array as the workspace:
- * it allocates nothing, neither device nor host memory, on any call.  For
- * callers that may not allocate when they multiply: a real-time audio thread
- * that must not block in an allocator, a process that budgets device memory
- * once at start-up, code that runs where no allocator is reachable.
+ * it never allocates device memory (no cudaMalloc, no allocating library
+ * routine).  For callers that may not allocate device memory when they
+ * multiply: a real-time audio thread that must not block in an allocator, a
+ * process that budgets device memory once at start-up, code that runs where
+ * no device allocator is reachable.
+ *   * Host memory: the library's small host-side caches (per-thread problem
+ *     lists, the cache of TMA descriptors, guarded by a mutex) grow on a
+ *     thread's first call and on the first call with each new W or X pointer
+ *     or shape.  A caller that must not touch the host allocator either
+ *     makes one call with each of its buffers and shapes first, off the
+ *     real-time thread, or takes the library's host-side growth into account.
  *   * The array (Q4_0_STATIC_WS_BYTES, 256-byte aligned) is a __device__
  *     variable of the library, one copy per device.  A problem whose
  *     workspace size (q4_0_gemm_workspace_size) exceeds it is rejected with
- *     Q4_ERR_TOO_LARGE and nothing is launched; M <= 32 needs none.
+ *     Q4_ERR_TOO_LARGE and nothing is launched; M <= 32 needs none (a
+ *     tensor-core run forced for M <= 32 uses the array only when its fp16
+ *     copy of X fits, and otherwise converts X tile by tile).
  *   * Nothing in the array has to start at zero: each call writes every byte
  *     it reads before reading it, on `stream`.
  *   * Calls whose kernels can overlap on one device (different streams or

@@ -404,6 +404,29 @@ def test_workspace_too_small_falls_back(q4):
     assert q4.q4_0_gemm_workspace_size(8, 64, 512) == 0
 
 
+def test_forced_tensor_path_small_m_small_workspace(q4):
+    """The tensor-core path forced for M <= 32 with a workspace smaller than
+    the fp16 copy of X (M*K*2 bytes): the library must not convert into it
+    (that would write past its end); it converts X tile by tile instead, and
+    the bytes just past the workspace stay untouched."""
+    M, N, K = 24, 200, 1024
+    rng = np.random.default_rng(5)
+    codes, scales, X = rand_inputs(rng, M, N, K, 0.5)
+    W = pack_on_gpu(q4, codes, scales)
+    small = 256                                  # < M*K*2 = 48 KiB
+    guard = torch.full((small + 4096,), 0x5A, dtype=torch.uint8, device="cuda")
+    Y = torch.full((M, N), float("nan"), device="cuda")
+    q4.q4_0_force_path(q4.PATH_TENSOR)
+    try:
+        q4.q4_0_gemm_ws(W, dev(X), Y, M, N, K, guard[:small])
+    finally:
+        q4.q4_0_force_path(0)
+    torch.cuda.synchronize()
+    assert bool((guard[small:] == 0x5A).all()), "bytes past the workspace were written"
+    Y_or, B_or = oracle.get().gemm(oracle.get().pack(codes, scales), X, M, N, K)
+    check_gemm(Y.cpu().numpy(), Y_or, B_or, "forced tensor path, M <= 32, small workspace")
+
+
 @pytest.mark.parametrize("M,N,K", [(1, 100, 1024), (2, 129, 3072), (16, 33, 2048), (32, 70, 512)])
 def test_forced_tmem_decode(q4, M, N, K):
     run_gemm(q4, M, N, K, path=q4.PATH_DECODE_TMEM)
