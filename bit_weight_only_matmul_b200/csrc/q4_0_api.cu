@@ -81,7 +81,18 @@ int check_problem(const q4_0_problem &p) {
     return Q4_OK;
 }
 
-enum Path { kAuto = 0, kGeneric = 1, kDecode = 2, kTensor = 3, kDecodeExact = 4, kDecodeTmem = 5 };
+enum Path { kAuto = 0, kGeneric = 1, kDecode = 2, kTensor = 3, kDecodeExact = 4, kDecodeTmem = 5, kDecodeM8 = 6 };
+
+// The decode problems of one call: M <= 8 on the 512-k-slot kernel, the rest
+// (M <= 32) on the kernel with 1-4 n-tiles of X rows.
+cudaError_t launch_decode_split(std::vector<q4::Problem> &dec, std::vector<q4::Problem> &wide,
+                                const q4::DeviceInfo &dev, cudaStream_t s) {
+    cudaError_t e = cudaSuccess;
+    if (!dec.empty()) e = q4::launch_decode_m8(dec.data(), static_cast<int>(dec.size()), dev, s);
+    if (e == cudaSuccess && !wide.empty())
+        e = q4::launch_decode_mma(wide.data(), static_cast<int>(wide.size()), dev, s);
+    return e;
+}
 
 int run_problems(const q4_0_problem *probs, int count, cudaStream_t s, void *ws = nullptr, int64_t ws_bytes = 0) {
     int st = Q4_OK;
@@ -97,8 +108,9 @@ int run_problems(const q4_0_problem *probs, int count, cudaStream_t s, void *ws 
     if (st != Q4_OK) return st;
     const int force = g_force_path.load(std::memory_order_relaxed);
     // per-thread lists, reused from call to call (no allocation once grown)
-    static thread_local std::vector<q4::Problem> dec, dexact, dtmem, gen, ten;
+    static thread_local std::vector<q4::Problem> dec, dm8, dexact, dtmem, gen, ten;
     dec.clear();
+    dm8.clear();
     dexact.clear();
     dtmem.clear();
     gen.clear();
@@ -113,20 +125,22 @@ int run_problems(const q4_0_problem *probs, int count, cudaStream_t s, void *ws 
         }
         q4::Problem p{static_cast<const uint8_t *>(a.W), a.X, a.Y, a.M, a.N, a.K};
         const bool dec_ok = q4::decode_mma_supports(p);
+        const bool m8_ok = q4::decode_m8_supports(p);
         const bool exact_ok = q4::decode_supports(p);
         const bool tmem_ok = q4::decode_tmem_supports(p);
         const bool ten_ok = q4::prefill_supports(p);
         if (force == kGeneric) gen.push_back(p);
         else if (force == kDecode && dec_ok) dec.push_back(p);
+        else if (force == kDecodeM8 && m8_ok) dm8.push_back(p);
         else if (force == kDecodeExact && exact_ok) dexact.push_back(p);
         else if (force == kDecodeTmem && tmem_ok) dtmem.push_back(p);
         else if (force == kTensor && ten_ok) ten.push_back(p);
+        else if (p.M <= 8 && m8_ok) dm8.push_back(p);
         else if (p.M <= 32 && dec_ok) dec.push_back(p);
         else if (p.M > 32 && ten_ok) ten.push_back(p);
         else gen.push_back(p);
     }
-    cudaError_t e = cudaSuccess;
-    if (!dec.empty()) e = q4::launch_decode_mma(dec.data(), static_cast<int>(dec.size()), *dev, s);
+    cudaError_t e = launch_decode_split(dm8, dec, *dev, s);
     if (e != cudaSuccess) return cuda_fail(e);
     if (!dexact.empty()) e = q4::launch_decode(dexact.data(), static_cast<int>(dexact.size()), *dev, s);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -261,8 +275,9 @@ int q4_0_quantize(const float *X, void *W, int64_t N, int64_t K, q4_0_stream_t s
 int q4_0_gemm_grouped_ex(const q4_0_problem_ex *problems, int count, q4_0_stream_t stream) {
     if (count < 0 || count > Q4_0_MAX_GROUP || (count > 0 && !problems)) return Q4_ERR_INVALID_ARG;
     if (count == 0) return Q4_OK;
-    static thread_local std::vector<q4::Problem> dec;
+    static thread_local std::vector<q4::Problem> dec, dm8;
     dec.clear();
+    dm8.clear();
     for (int i = 0; i < count; ++i) {
         const q4_0_problem_ex &a = problems[i];
         const q4_0_problem base{a.W, a.X, a.Y, a.M, a.N, a.K};
@@ -280,14 +295,15 @@ int q4_0_gemm_grouped_ex(const q4_0_problem_ex *problems, int count, q4_0_stream
         q4::Problem p{static_cast<const uint8_t *>(a.W), a.X, a.Y, a.M, a.N, a.K};
         p.R = a.epilogue == Q4_0_EPI_RESIDUAL ? a.R : nullptr;
         p.epi = a.epilogue;
-        dec.push_back(p);
+        if (!q4::decode_mma_supports(p)) return Q4_ERR_INVALID_ARG;
+        const int force = g_force_path.load(std::memory_order_relaxed);
+        if (p.M <= 8 && force != kDecode && q4::decode_m8_supports(p)) dm8.push_back(p);
+        else dec.push_back(p);
     }
     const q4::DeviceInfo *dev = nullptr;
     int st = current_device(&dev);
     if (st != Q4_OK) return st;
-    for (const q4::Problem &p : dec)
-        if (!q4::decode_mma_supports(p)) return Q4_ERR_INVALID_ARG;
-    const cudaError_t e = q4::launch_decode_mma(dec.data(), count, *dev, reinterpret_cast<cudaStream_t>(stream));
+    const cudaError_t e = launch_decode_split(dm8, dec, *dev, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? Q4_OK : cuda_fail(e);
 }
 
@@ -345,7 +361,7 @@ int q4_0_device_error(uint32_t *flags, int clear) {
 }
 
 int q4_0_force_path(int path) {
-    if (path < 0 || path > 5) return Q4_ERR_INVALID_ARG;
+    if (path < 0 || path > 6) return Q4_ERR_INVALID_ARG;
     g_force_path.store(path, std::memory_order_relaxed);
     return Q4_OK;
 }

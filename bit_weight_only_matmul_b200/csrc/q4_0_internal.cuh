@@ -87,6 +87,10 @@ cudaError_t launch_generic(const Problem *probs, int count, const DeviceInfo &de
 // default decode path: every problem must satisfy decode_mma_supports().
 bool decode_mma_supports(const Problem &p);
 cudaError_t launch_decode_mma(const Problem *probs, int count, const DeviceInfo &dev, cudaStream_t s);
+// Decode kernel for M <= 8 (warp-level mma.sync, fp16 weights, 512-k ring
+// slots): every problem must satisfy decode_m8_supports().
+bool decode_m8_supports(const Problem &p);
+cudaError_t launch_decode_m8(const Problem *probs, int count, const DeviceInfo &dev, cudaStream_t s);
 // Exact-arithmetic decode kernel on warp-level mma.sync (bf16 (q - 8), fp32
 // scale per block; M <= 32): every problem must satisfy decode_supports().
 bool decode_supports(const Problem &p);
@@ -205,6 +209,14 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
     asm volatile(
         "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
             smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// The same with the destination given as a 32-bit shared-space address.
+__device__ __forceinline__ void bulk_g2s_u32(uint32_t dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
         "l"(src), "r"(bytes), "r"(smem_addr(bar))
         : "memory");
 }

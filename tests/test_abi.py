@@ -49,7 +49,8 @@ def test_bytes(q4):
 
 
 def test_force_path_range(q4):
-    assert q4.lib.q4_0_force_path(6) == q4.Q4_ERR_INVALID_ARG
+    assert q4.lib.q4_0_force_path(7) == q4.Q4_ERR_INVALID_ARG
+    assert q4.lib.q4_0_force_path(6) == q4.Q4_OK
     assert q4.lib.q4_0_force_path(-1) == q4.Q4_ERR_INVALID_ARG
     assert q4.lib.q4_0_force_path(0) == q4.Q4_OK
 
