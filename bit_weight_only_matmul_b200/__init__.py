@@ -26,12 +26,13 @@ Q4_ERR_TOO_LARGE = 5
 
 Q4_DEVERR_WAIT_TIMEOUT = 1
 Q4_DEVERR_BAD_INDEX = 2
+Q4_DEVERR_FP16_RANGE = 4
 
 Q4_0_MAX_GROUP = 256
 Q4_0_STATIC_WS_BYTES = 64 << 20
 Q4_0_EPI_NONE, Q4_0_EPI_RESIDUAL, Q4_0_EPI_SWIGLU = 0, 1, 2
 
-PATH_AUTO, PATH_GENERIC, PATH_DECODE, PATH_TENSOR, PATH_DECODE_EXACT, PATH_DECODE_TMEM = 0, 1, 2, 3, 4, 5
+PATH_AUTO, PATH_GENERIC, PATH_DECODE, PATH_TENSOR, PATH_DECODE_EXACT, PATH_DECODE_TMEM, PATH_DECODE_M8 = 0, 1, 2, 3, 4, 5, 6
 
 # every symbol include/q4_0.h declares
 EXPORTS = (

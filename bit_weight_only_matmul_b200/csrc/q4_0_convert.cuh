@@ -56,4 +56,44 @@ __device__ __forceinline__ uint4 x8_to_fp16_permuted(uint4 v) {
     return make_uint4(lo.x, lo.y, hi.x, hi.y);
 }
 
+// Nonzero if any of the 8 bf16 values of v is finite and outside the range in
+// which the fp16 conversion above is exact: |x| >= 65536 (fp16 overflows to
+// inf) or 0 < |x| < 2^-17 (below 2^-17 a bf16 value can need more bits than
+// an fp16 subnormal has).  Per 16-bit half, a = |x| bits: bad iff
+// a - 1 < 0x36FF (1 <= a < 0x3700 = 2^-17) or a - 0x4780 < 0x3800
+// (0x4780 = 65536 <= a < 0x7F80 = inf).
+__device__ __forceinline__ uint32_t x8_fp16_range_bad(uint4 v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t bad = 0;
+    #pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t a = w[i] & 0x7FFF7FFFu;
+        bad |= __vcmpltu2(__vsub2(a, 0x00010001u), 0x36FF36FFu) | __vcmpltu2(__vsub2(a, 0x47804780u), 0x38003800u);
+    }
+    return bad;
+}
+
+// Nonzero if an fp16 scale, given as its bit pattern, is finite and so large
+// that (q - 8) * d overflows fp16 for q = 0: 8188 < |d| < inf.
+__device__ __forceinline__ bool scale_fp16_range_bad(uint32_t dbits) {
+    const uint32_t a = dbits & 0x7FFFu;
+    return a >= 0x7000u && a < 0x7C00u;
+}
+
+// The slow path of the scale check, run only where a fast path produced a
+// non-finite sum: scan the scales of weight rows [n0, n1) of a Q4_0 matrix
+// with K weights per row and flag Q4_DEVERR_FP16_RANGE if one is out of range.
+static __device__ __noinline__ void scan_scales_fp16_range(const uint8_t *W, int64_t n0, int64_t n1, int64_t N, int64_t K,
+                                                    unsigned *err) {
+    const int64_t row_bytes = K / 32 * 18;
+    for (int64_t n = n0; n < n1 && n < N; ++n)
+        for (int64_t b = 0; b < K / 32; ++b) {
+            const uint8_t *p = W + n * row_bytes + 18 * b;
+            if (scale_fp16_range_bad(static_cast<uint32_t>(p[0]) | (static_cast<uint32_t>(p[1]) << 8))) {
+                atomicOr(err, (unsigned)Q4_DEVERR_FP16_RANGE);
+                return;
+            }
+        }
+}
+
 }  // namespace q4dev

@@ -70,7 +70,11 @@ enum {
 /* Device error bits reported by q4_0_device_error. */
 enum {
     Q4_DEVERR_WAIT_TIMEOUT = 1u,   /* a bounded on-chip wait gave up; the output is incomplete */
-    Q4_DEVERR_BAD_INDEX = 2u       /* q4_0_gather met an id outside [0, V) (its row was zeroed) */
+    Q4_DEVERR_BAD_INDEX = 2u,      /* q4_0_gather met an id outside [0, V) (its row was zeroed) */
+    Q4_DEVERR_FP16_RANGE = 4u      /* a fast GEMM path met an operand its fp16 arithmetic does not hold
+                                      exactly: a finite X with |x| > 65504 or 0 < |x| < 2^-17, or a
+                                      scale with 8188 < |d| < inf; its output may hold +-inf or lost
+                                      precision (q4_0_force_path(4) computes such inputs exactly) */
 };
 
 /* Largest N, K and M accepted (each dimension below 2^31). */
@@ -120,10 +124,12 @@ Q4_0_API int q4_0_dequant(const void *W, float *out, int64_t N, int64_t K,
  * tcgen05 tensor-core kernel (weight tiles dequantized into tensor memory,
  * fp32 accumulators in tensor memory).  Both feed the tensor cores fp16
  * operands: each weight (q - 8) * d is rounded once to fp16 (relative error
- * <= 2^-11) and X is exact in fp16 within its normal range, so operands must
- * lie in the fp16 range (|x| <= 65504, |d| <= 8188); beyond it products
- * overflow to +-inf.  q4_0_force_path(4) selects an exact-arithmetic decode
- * kernel without that restriction. */
+ * <= 2^-11) and X is converted to fp16, exactly for 2^-17 <= |x| <= 65504.
+ * An operand outside that (a finite |x| > 65504 or 0 < |x| < 2^-17, a scale
+ * 8188 < |d| < inf) is detected on the GPU and sets Q4_DEVERR_FP16_RANGE in
+ * q4_0_device_error: the output may then hold +-inf or lost precision.
+ * q4_0_force_path(4) selects an exact-arithmetic decode kernel ((q - 8)
+ * exact in bf16, X used as given) without that restriction. */
 Q4_0_API int q4_0_gemm(const void *W, const uint16_t *X, float *Y,
               int64_t M, int64_t N, int64_t K, q4_0_stream_t stream);
 
@@ -292,7 +298,9 @@ Q4_0_API int q4_0_device_error(uint32_t *flags, int clear);
  * q4_0_gemm_grouped.  0 = automatic (default), 1 = portable kernel (any
  * shape), 2 = decode kernel (M <= 32 only), 3 = tensor-core kernel, 4 = the
  * exact-arithmetic decode kernel ((q - 8) exact in bf16, d applied in fp32;
- * M <= 32), 5 = the tcgen05 decode kernel (weights in tensor memory; M <= 32).
+ * M <= 32), 5 = the tcgen05 decode kernel (weights in tensor memory; M <= 32),
+ * 6 = the M <= 8 decode kernel with 512-k ring slots (automatic for M <= 8;
+ * path 2 sends M <= 8 to the kernel with 256-k stages instead).
  * A forced family that cannot run a given shape falls back to automatic.  The
  * pages have no counterpart. */
 Q4_0_API int q4_0_force_path(int path);
