@@ -36,6 +36,7 @@ import subprocess
 import sys
 import threading
 import time
+from typing import Optional
 
 import numpy as np
 
@@ -46,7 +47,7 @@ import workloads  # noqa: E402
 
 METRIC = "Q4_0 dequant-matmul HBM GB/s (M=1,2) and TFLOP/s (M>=64), % of B200 roofline"
 L2_BYTES = 126 * 2**20
-DEFAULT_WORKLOAD = "layer"
+DEFAULT_WORKLOAD = "cfg_decode"
 
 # kernel that dominates each workload, and the source file it lives in
 DOMINANT = {
@@ -157,7 +158,7 @@ class GpuWorkload:
 
     SEEDS = 8
 
-    def __init__(self, q4, wl: workloads.Workload, copies: int, seed: int):
+    def __init__(self, q4, wl: workloads.Workload, copies: int, seed: int, wcache: Optional[dict] = None):
         import torch
         self.wl = wl
         self.sets = []
@@ -171,6 +172,7 @@ class GpuWorkload:
             return out, at
         x_off, x_total = offsets([l.M * l.K for l in wl.linears])
         y_off, y_total = offsets([l.M * l.N for l in wl.linears])
+        self.x_off, self.y_off = x_off, y_off
         self.xbufs, self.ybufs = [], []
         for c in range(copies):
             probs = []
@@ -186,11 +188,16 @@ class GpuWorkload:
                     probs.append((W, X, Y, lin.M, lin.N, lin.K))
                     continue
                 s = seed + 7919 * c
-                codes = torch.from_numpy(lin.codes(s)).cuda()
-                scales = torch.from_numpy(lin.scales(s).view(np.int16)).cuda()
-                W = torch.empty(q4.q4_0_bytes(lin.N, lin.K), dtype=torch.uint8, device="cuda")
-                q4.q4_0_pack(codes, scales, W, lin.N, lin.K)
-                del codes, scales
+                key = (s, lin.layer, lin.linear, lin.N, lin.K)
+                W = wcache.get(key) if wcache is not None else None
+                if W is None:   # weights with the same seed streams are shared between workloads
+                    codes = torch.from_numpy(lin.codes(s)).cuda()
+                    scales = torch.from_numpy(lin.scales(s).view(np.int16)).cuda()
+                    W = torch.empty(q4.q4_0_bytes(lin.N, lin.K), dtype=torch.uint8, device="cuda")
+                    q4.q4_0_pack(codes, scales, W, lin.N, lin.K)
+                    del codes, scales
+                    if wcache is not None:
+                        wcache[key] = W
                 X.copy_(torch.from_numpy(lin.x(s).view(np.int16)))
                 probs.append((W, X, Y, lin.M, lin.N, lin.K))
             self.sets.append((probs, q4.make_problems(probs)))
@@ -235,6 +242,12 @@ class GpuWorkload:
         self.operand_bytes = sum(W.numel() + X.numel() * 2 + Y.numel() * 4 for W, X, Y, *_ in self.sets[0][0])
         torch.cuda.synchronize()
 
+    def views(self, xbuf, ybuf):
+        """The per-GEMM X and Y views of a step-sized pair of buffers."""
+        xs = [xbuf[o:o + l.M * l.K].view(l.M, l.K) for l, o in zip(self.wl.linears, self.x_off)]
+        ys = [ybuf[o:o + l.M * l.N].view(l.M, l.N) for l, o in zip(self.wl.linears, self.y_off)]
+        return xs, ys
+
     def outputs(self, step: int):
         """The Y tensors a step writes."""
         k = step % len(self.sets)
@@ -261,53 +274,60 @@ def rotating_copies(wl: workloads.Workload) -> int:
     return max(1, -(-2 * L2_BYTES // max(1, step)))
 
 
-def run_ours(args, rank: int, world: int):
+# B200 datasheet figures (context for the measured denominators): HBM3e 8 TB/s,
+# dense bf16 tensor 2.25 PFLOP/s
+SPEC = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+# the five configurations of the metric (config 5 as its two GEMMs), measured
+# in one process: the headline workload with its end-to-end and CPU legs,
+# the others as records of the same line
+CONFIG_SET = ("gemv", "layer", "cfg_decode", "concurrent", "adapter", "qkv_prefill")
+# layers of a 26-layer workload whose outputs the oracle samples
+ORACLE_LAYERS = (0, 12, 25)
+
+
+class Timed:
+    """One workload measured on this rank: device time of `steps` back-to-back
+    steps, clocks, and (headline only) the end-to-end time."""
+
+    def __init__(self, **kw):
+        self.__dict__.update(kw)
+
+
+def _barrier(world):
     import torch
-    import torch.distributed as dist
-    import bit_weight_only_matmul_b200 as q4
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
 
-    wl = workloads.workload(args.workload)
-    tensor = args.workload in TENSOR_WORKLOADS
-    step_bytes = wl.hbm_bytes
-    step_flops = wl.flops
-    copies = rotating_copies(wl)
-    log(f"[rank {rank}] building {wl.name}: {len(wl.linears)} GEMMs x {copies} copies, "
-        f"{step_bytes / 1e6:.1f} MB per step")
-    G = GpuWorkload(q4, wl, copies, workloads.SEED + 1000 * rank)
+
+def time_workload(q4, G, tensor: bool, steps: int, warmup: int, soak: float, world: int, no_graphs: bool,
+                  min_ms: float = 0.0):
+    """Warm up, soak for `soak` seconds, then time `steps` steps (at least
+    enough for `min_ms` of device time when min_ms > 0) back to back between
+    one pair of CUDA events on the launching stream.  Returns (ms_total,
+    steps, clocks summary, launch description)."""
+    import torch
     stream = torch.cuda.current_stream()
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    q4.q4_0_device_error(clear=True)
     with ClockSampler(torch.cuda.current_device()) as clocks:
-        # warm-up: W untimed steps, then an untimed soak of about a second so
-        # that the clock sampler sees the GPU under this load
-        for i in range(args.warmup):
+        for i in range(warmup):
             G.launch(q4, i)
-        barrier()
-        t_end = time.time() + args.soak
+        _barrier(world)
+        t_end = time.time() + soak
         i = 0
         while time.time() < t_end:
             for _ in range(16):
                 G.launch(q4, i)
                 i += 1
             torch.cuda.synchronize()
-        barrier()
-        # one CUDA graph holding a whole cycle of steps (one per operand copy,
-        # in order), captured after the warm-up so that the library's one-time
-        # set-up has run: host launch overhead does not gate the device, and
-        # consecutive kernels keep their programmatic-launch overlap
+        _barrier(world)
+        # tensor-core steps (X conversion + GEMM) replay CUDA graphs of a
+        # whole cycle of operand copies; a decode step is one launch that the
+        # host enqueues well ahead of the device, overlapping its
+        # predecessor's tail through programmatic dependent launch
         cycle = len(G.sets)
         graph = None
-        # a decode step is one launch, which the host enqueues well ahead of
-        # the device and which overlaps its predecessor's tail through
-        # programmatic dependent launch; graphs pay off for the tensor-core
-        # steps (two launches each: X conversion, then the GEMM)
-        use_graph = tensor and not args.no_graphs
-        if use_graph:
+        if tensor and not no_graphs:
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph):
                 for k in range(cycle):
@@ -322,122 +342,322 @@ def run_ours(args, rank: int, world: int):
             for j in range(k, n):
                 G.launch(q4, j)
 
-        run_steps(args.warmup)
-        barrier()
-        # timed region: exactly K steps back to back between one pair of
-        # events on the launching stream (events between the steps would put
-        # gaps between the kernels that a real token loop does not have)
+        run_steps(max(warmup, cycle if graph is not None else 0))
+        _barrier(world)
+        if min_ms > 0:
+            # the same step count on every rank: from a short trial, maxed over ranks
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            run_steps(cycle if graph is not None else 8)
+            e1.record(stream)
+            _barrier(world)
+            per = max_over_ranks([e0.elapsed_time(e1) / (cycle if graph is not None else 8)], world, "cuda")[0]
+            steps = max(steps, int(min_ms / max(per, 1e-4)) + 1)
+            if graph is not None:
+                steps = -(-steps // cycle) * cycle
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
-        barrier()
+        _barrier(world)
         t0.record(stream)
-        run_steps(args.steps)
+        run_steps(steps)
         t1.record(stream)
-        barrier()
-    ms_total = t0.elapsed_time(t1)
-    dev_err = q4.q4_0_device_error(clear=True)
-    if dev_err:
-        raise RuntimeError(f"device error word {dev_err:#x} after the timed region")
+        _barrier(world)
+    launch = (f"CUDA graph replay of cycles of {cycle} steps (the library's own launches inside)"
+              if graph is not None else "eager, programmatic dependent launch")
+    del graph
+    return t0.elapsed_time(t1), steps, clocks.summary(), launch
 
-    # end to end through the public API: host X -> device, grouped GEMM, Y -> host
-    # (one pinned copy each way: a step's X and Y live in one buffer each)
-    hx = [torch.empty(G.xbufs[0].shape, dtype=G.xbufs[0].dtype, pin_memory=True).copy_(G.xbufs[0].cpu())]
-    outs0 = [G.ybufs[0]] if not G.fused_arrs else G.outputs(0)
-    hy = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for y in outs0]
-    h2d = sum(t.numel() * t.element_size() for t in hx)
-    d2h = sum(t.numel() * t.element_size() for t in hy)
+
+def e2e_overlapped(q4, G, steps: int, warmup: int, world: int):
+    """End to end through the public API: every step copies its X from pinned
+    host memory to the device, runs the step's grouped / workspace GEMMs and
+    copies its Y back to pinned host memory.  The copies run on two copy
+    streams and the GEMMs on the launching stream, with X and Y double
+    buffered on the device, so that the H2D of step k+1 and the D2H of step
+    k-1 overlap the GEMMs of step k (one cudaMemcpyAsync per buffer and
+    direction).  Returns (ms for `steps` steps, h2d bytes, d2h bytes)."""
+    import torch
+    main = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    xb = [torch.empty_like(G.xbufs[0]) for _ in range(2)]
+    yb = [torch.empty_like(G.ybufs[0]) for _ in range(2)]
+    hx = torch.empty(G.xbufs[0].shape, dtype=G.xbufs[0].dtype, pin_memory=True).copy_(G.xbufs[0].cpu())
+    hy = [torch.empty(G.ybufs[0].shape, dtype=G.ybufs[0].dtype, pin_memory=True) for _ in range(2)]
+    # problem arrays of (operand copy c, buffer slot b): the weights rotate
+    # as in the device-timed steps, X and Y live in the slot's buffers
+    arrays = {}
+    for c, (probs, _) in enumerate(G.sets):
+        for b in range(2):
+            xs, ys = G.views(xb[b], yb[b])
+            arrays[c, b] = [(W, xs[i], ys[i], M, N, K) for i, (W, X, Y, M, N, K) in enumerate(probs)]
+    small_arrs = {key: q4.make_problems([p[i] for i in G.small]) for key, p in arrays.items()}
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    recorded = [False, False]
+
+    def step(k):
+        c, b = k % len(G.sets), k & 1
+        with torch.cuda.stream(s_in):
+            if recorded[b]:
+                s_in.wait_event(ev_done[b])      # step k-2 has read X[b]
+            xb[b].copy_(hx, non_blocking=True)
+            ev_in[b].record(s_in)
+        main.wait_event(ev_in[b])
+        if recorded[b]:
+            main.wait_event(ev_out[b])           # step k-2's Y[b] has reached the host
+        if G.small:
+            q4.q4_0_gemm_grouped(small_arrs[c, b], len(G.small))
+        for i in G.large:
+            W, X, Y, M, N, K = arrays[c, b][i]
+            q4.q4_0_gemm_ws(W, X, Y, M, N, K, G.ws)
+        ev_done[b].record(main)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[b])
+            hy[b].copy_(yb[b], non_blocking=True)
+            ev_out[b].record(s_out)
+        recorded[b] = True
+
+    for k in range(warmup):
+        step(k)
+    _barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(main)
+    s_in.wait_event(e0)
+    for k in range(steps):
+        step(k)
+    for b in range(2):
+        main.wait_event(ev_out[b])
+    e1.record(main)
+    _barrier(world)
+    return e0.elapsed_time(e1), hx.numel() * hx.element_size(), hy[0].numel() * hy[0].element_size()
 
-    def e2e_step(k):
-        c = k % len(G.sets)
-        G.xbufs[c].copy_(hx[0], non_blocking=True)
+
+def e2e_serial(q4, G, steps: int, warmup: int, world: int):
+    """End to end for the fused-epilogue workload (its outputs are not the
+    plain Y buffers): X in, the step, Y out, all on the launching stream."""
+    import torch
+    main = torch.cuda.current_stream()
+    hx = torch.empty(G.xbufs[0].shape, dtype=G.xbufs[0].dtype, pin_memory=True).copy_(G.xbufs[0].cpu())
+    hy = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for y in G.outputs(0)]
+
+    def step(k):
+        G.xbufs[k % len(G.sets)].copy_(hx, non_blocking=True)
         G.launch(q4, k)
-        for Y, h in zip([G.ybufs[c]] if not G.fused_arrs else G.outputs(k), hy):
+        for Y, h in zip(G.outputs(k), hy):
             h.copy_(Y, non_blocking=True)
 
-    for i in range(args.warmup):
-        e2e_step(i)
-    barrier()
-    e0.record(stream)
-    for k in range(args.steps):
-        e2e_step(k)
-    e1.record(stream)
-    barrier()
-    e2e_ms = e0.elapsed_time(e1)
+    for k in range(warmup):
+        step(k)
+    _barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(main)
+    for k in range(steps):
+        step(k)
+    e1.record(main)
+    _barrier(world)
+    return e0.elapsed_time(e1), hx.numel() * hx.element_size(), sum(h.numel() * h.element_size() for h in hy)
 
-    ms_total, e2e_ms = max_over_ranks([ms_total, e2e_ms], world, "cuda")
-    # every step is the dominant kernel's launch (plus, for M > 32, the X
-    # conversion pass before it): its average duration is the step time
-    launch_avg_ms = ms_total / args.steps
-    clock = clocks.summary()
 
-    if rank != 0:
-        return None
-    peaks = measured_peaks()
-    kernel, src = DOMINANT[args.workload]
+def sampled_linears(wl):
+    """Indices of the linears the oracle samples: all of them, or those of
+    layers ORACLE_LAYERS for the 26-layer workloads."""
+    if len(wl.linears) > 16:
+        return [i for i, l in enumerate(wl.linears) if l.layer in ORACLE_LAYERS]
+    return list(range(len(wl.linears)))
+
+
+def pack_on_host(wl, seed, which=None):
+    """The oracle's own packing of the seeded codes and scales of the linears
+    `which` (default all): [(index, W_host, X_host)]."""
+    import oracle
+    o = oracle.get()
+    which = range(len(wl.linears)) if which is None else which
+    return o, [(i, o.pack(wl.linears[i].codes(seed), wl.linears[i].scales(seed)), wl.linears[i].x(seed))
+               for i in which]
+
+
+def oracle_error(q4, G, wl, host, samples: int = 48, seed: int = 7):
+    """max |Y_gpu - Y_oracle| / (1e-3 * sum_k |x w| + 1e-6) over `samples`
+    seeded output positions (the last row and column always among them) of
+    each sampled linear, on operand copy 0 after one more step."""
+    import torch
+    if G.fused_arrs:
+        return None, "fused epilogues: checked by the GPU tests, not here"
+    o, packed = host
+    G.launch(q4, 0)
+    torch.cuda.synchronize()
+    outs = G.outputs(0)
+    rng = np.random.default_rng(seed)
+    worst, n = 0.0, 0
+    for i, W_host, X_host in packed:
+        lin = wl.linears[i]
+        ms = rng.integers(0, lin.M, size=samples)
+        ns = rng.integers(0, lin.N, size=samples)
+        ms[0], ns[0] = lin.M - 1, lin.N - 1
+        Y_or, B_or = o.gemm_sampled(W_host, X_host, lin.M, lin.N, lin.K, ms, ns)
+        got = outs[i].cpu().numpy().astype(np.float64)[ms, ns]
+        worst = max(worst, float(np.max(np.abs(got - Y_or) / (1e-3 * B_or + 1e-6))))
+        n += samples
+    return worst, f"{n} outputs of {len(packed)} GEMM(s) (operand copy 0)"
+
+
+def build_record(name, wl, tensor, ms_total, steps, world, clock, launch, peaks, G):
+    kernel, src = DOMINANT[name]
+    launch_avg_ms = ms_total / steps
     if tensor:
-        unit = "TFLOP/s"
-        value = whole_job_rate(step_flops, args.steps, world, ms_total) / 1e12
-        e2e_value = whole_job_rate(step_flops, args.steps, world, e2e_ms) / 1e12
-        achieved = step_flops / (launch_avg_ms * 1e-3) / 1e12
+        unit, per_step = "TFLOP/s", wl.flops
+        value = whole_job_rate(per_step, steps, world, ms_total) / 1e12
+        achieved = per_step / (launch_avg_ms * 1e-3) / 1e12
         # the steps run back to back after a soak, under the power cap: the
         # sustained GEMM figure is the matching denominator
-        peak = peaks["bf16_tflops_sustained"]
-        bound = "tensor"
+        peak, spec, bound = peaks["bf16_tflops_sustained"], SPEC["bf16_tflops"], "tensor"
+        peak_src = peaks["source"] + " (sustained bf16 GEMM, same rate as fp16)"
     else:
-        unit = "GB/s"
-        value = whole_job_rate(step_bytes, args.steps, world, ms_total) / 1e9
-        e2e_value = whole_job_rate(step_bytes, args.steps, world, e2e_ms) / 1e9
-        achieved = step_bytes / (launch_avg_ms * 1e-3) / 1e9
-        peak = peaks["hbm_gbs"]
-        bound = "hbm"
-    line = {
+        unit, per_step = "GB/s", wl.hbm_bytes
+        value = whole_job_rate(per_step, steps, world, ms_total) / 1e9
+        achieved = per_step / (launch_avg_ms * 1e-3) / 1e9
+        peak, spec, bound = peaks["hbm_gbs"], SPEC["hbm_gbs"], "hbm"
+        peak_src = peaks["source"] + " (STREAM-style copy)"
+    return {
+        "value": round(value, 2), "unit": unit, "ms_per_step": round(launch_avg_ms, 5), "steps": steps,
+        "gpu_launches": steps * launches_per_step(name, wl),
+        "config": {"workload": f"{wl.name}: {wl.description}", "gemms_per_step": len(wl.linears),
+                   "bytes_per_step": wl.hbm_bytes, "flops_per_step": wl.flops,
+                   "l2": (f"inputs larger than L2: {len(G.sets)} rotating copies of the step's operands = "
+                          f"{len(G.sets) * G.operand_bytes / 1e6:.0f} MB > L2 ({L2_BYTES / 2**20:.0f} MiB)"),
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "launch": launch,
+        "roofline": {"bound": bound, "kernel": kernel, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+                     "frac": round(achieved / peak, 4), "peak_source": peak_src,
+                     "spec_peak": spec, "frac_of_spec": round(achieved / spec, 4),
+                     "traffic": recorded_traffic(name), "algorithmic_per_launch": per_step},
+        "clocks": clock,
+    }
+
+
+def stream_ceiling(q4, world: int, reps: int = 10):
+    """The read-only ceiling of the decode kernels' weight stream on this GPU:
+    q4_0_stream_read (the same TMA boxes and per-SM ring, no arithmetic)
+    over a 1 GiB Q4_0 matrix (K = 3072), `reps` reads back to back, timed
+    with CUDA events.  Returns GB/s of weight bytes."""
+    import torch
+    K = 3072
+    row = K // 32 * 18
+    N = ((1 << 30) // row) // 128 * 128
+    W = torch.zeros(N * row, dtype=torch.uint8, device="cuda")
+    cs = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for _ in range(3):
+        q4.q4_0_stream_read(W, N, K, cs)
+    _barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        q4.q4_0_stream_read(W, N, K, cs)
+    e1.record()
+    _barrier(world)
+    ms = max_over_ranks([e0.elapsed_time(e1)], world, "cuda")[0]
+    del W
+    return {"value": round(N * row * reps / (ms * 1e-3) / 1e9, 1), "unit": "GB/s", "bytes_per_read": N * row,
+            "what": f"q4_0_stream_read of a {N} x {K} Q4_0 matrix ({N * row / 2**30:.2f} GiB), {reps} reads "
+                    "back to back: the decode kernels' TMA weight stream with no arithmetic"}
+
+
+def run_ours(args, rank: int, world: int):
+    import torch
+    import bit_weight_only_matmul_b200 as q4
+
+    peaks = measured_peaks()
+    names = [args.workload] + ([n for n in CONFIG_SET if n != args.workload] if not args.only else [])
+    wcache = {}
+    records = {}
+    line = None
+    q4.q4_0_device_error(clear=True)
+    for name in names:
+        headline = name == args.workload
+        wl = workloads.workload(name)
+        tensor = name in TENSOR_WORKLOADS
+        copies = rotating_copies(wl)
+        log(f"[rank {rank}] building {wl.name}: {len(wl.linears)} GEMMs x {copies} copies, "
+            f"{wl.hbm_bytes / 1e6:.1f} MB per step")
+        G = GpuWorkload(q4, wl, copies, workloads.SEED + 1000 * rank, wcache)
+        if headline:
+            ms_total, steps, clock, launch = time_workload(q4, G, tensor, args.steps, args.warmup, args.soak, world,
+                                                           args.no_graphs)
+        else:
+            # enough steps for at least 20 ms of device time (a GEMV step is ~5 us)
+            ms_total, steps, clock, launch = time_workload(q4, G, tensor, args.steps, args.warmup,
+                                                           min(args.soak, 0.5), world, args.no_graphs, min_ms=20.0)
+        dev_err = q4.q4_0_device_error(clear=True)
+        if dev_err:
+            raise RuntimeError(f"device error word {dev_err:#x} after the timed region of {name}")
+        ms_total = max_over_ranks([ms_total], world, "cuda")[0]
+        rec = build_record(name, wl, tensor, ms_total, steps, world, clock, launch, peaks, G)
+        if headline:
+            if G.fused_arrs:
+                e2e_ms, h2d, d2h = e2e_serial(q4, G, args.steps, args.warmup, world)
+            else:
+                e2e_ms, h2d, d2h = e2e_overlapped(q4, G, args.steps, args.warmup, world)
+            e2e_ms = max_over_ranks([e2e_ms], world, "cuda")[0]
+            per = wl.flops if tensor else wl.hbm_bytes
+            e2e_value = whole_job_rate(per, args.steps, world, e2e_ms) / (1e12 if tensor else 1e9)
+            rec["e2e"] = {"value": round(e2e_value, 2), "unit": rec["unit"], "h2d_bytes_per_step": h2d,
+                          "d2h_bytes_per_step": d2h,
+                          "copies": "H2D and D2H on two copy streams, X and Y double-buffered on the device"
+                                    if not G.fused_arrs else "serial on the launching stream"}
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            # the oracle leg: a bounded, timed sample of the same workload on
+            # the host (the CPU baseline), whose values also give the GPU
+            # result's worst error over the method's tolerance
+            host = pack_on_host(wl, workloads.SEED, sampled_linears(wl))
+            rec["max_err_over_bound"], rec["oracle_sample"] = oracle_error(q4, G, wl, host)
+            budget = args.cpu_seconds if headline else args.cpu_seconds / 6
+            rec["cpu_baseline"] = cpu_baseline(wl, tensor, budget_s=budget, host=host)
+            if headline:
+                rec["cpu_baseline_all_cores"] = cpu_baseline_all_cores(wl, tensor, budget_s=budget / 2, host=host)
+        records[name] = rec
+        if headline:
+            line = rec
+        del G
+        torch.cuda.empty_cache()
+    del wcache
+    ceiling = stream_ceiling(q4, world)
+    for r in records.values():
+        if r["roofline"]["bound"] == "hbm":
+            r["roofline"]["frac_of_stream_ceiling"] = round(r["roofline"]["achieved"] / ceiling["value"], 4)
+    if rank != 0:
+        return None
+    out = {
         "metric": METRIC,
-        "value": round(value, 2),
-        "unit": unit,
+        "value": line["value"],
+        "unit": line["unit"],
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(ms_total / args.steps, 5),
+        "ms_per_step": line["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16 x q4_0 -> fp32" if not tensor else "fp16 x fp16(q4_0) -> fp32",
+        "dtype": ("bf16 x q4_0 -> fp32" if args.workload not in TENSOR_WORKLOADS
+                  else "fp16 x fp16(q4_0) -> fp32"),
         "data": "synthetic (seeded Philox; codes U{0..15}, d = fp16(|N(0,1)|*0.002+1e-4), X bf16 N(0,1))",
-        "config": {
-            "workload": f"{wl.name}: {wl.description}",
-            "gemms_per_step": len(wl.linears),
-            "bytes_per_step": step_bytes,
-            "flops_per_step": step_flops,
-            "weight_copies": len(G.sets),
-            "l2": (f"inputs larger than L2: {len(G.sets)} rotating copies of the step's operands = "
-                   f"{len(G.sets) * G.operand_bytes / 1e6:.0f} MB > L2 ({L2_BYTES / 2**20:.0f} MiB)"),
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "launch": (f"CUDA graph replay of cycles of {len(G.sets)} steps (the library's own launches "
-                       "inside)") if (tensor and not args.no_graphs) else "eager, programmatic dependent launch",
-        },
-        "roofline": {
-            "bound": bound,
-            "kernel": kernel,
-            "achieved": round(achieved, 2),
-            "peak": peak,
-            "unit": unit,
-            "frac": round(achieved / peak, 4),
-            "peak_source": peaks["source"] + (" (sustained bf16 GEMM, same rate as fp16)" if tensor else
-                                              " (STREAM-style copy)"),
-            "traffic": recorded_traffic(args.workload),
-            "algorithmic_per_launch": step_flops if tensor else step_bytes,
-        },
-        "e2e": {"value": round(e2e_value, 2), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * launches_per_step(args.workload, wl),
-        "clocks": clock,
+        "config": line["config"],
+        "launch": line["launch"],
+        "roofline": line["roofline"],
+        "e2e": line["e2e"],
+        "gpu_launches": line["gpu_launches"],
+        "clocks": line["clocks"],
+        "stream_ceiling": ceiling,
     }
-    if not args.no_cpu_baseline and world == 1:
-        host = pack_on_host(wl, workloads.SEED)
-        line["cpu_baseline"] = cpu_baseline(wl, tensor, budget_s=args.cpu_seconds, host=host)
-        line["cpu_baseline_all_cores"] = cpu_baseline_all_cores(wl, tensor, budget_s=args.cpu_seconds / 2, host=host)
-    return line
+    for key in ("max_err_over_bound", "oracle_sample", "cpu_baseline", "cpu_baseline_all_cores"):
+        if key in line:
+            out[key] = line[key]
+    if len(records) > 1:
+        out["configs"] = {n: {k: v for k, v in r.items() if k not in ("cpu_baseline_all_cores",)}
+                          for n, r in records.items()}
+    return out
 
 
 # --------------------------------------------------------------------------- the utilities
@@ -644,30 +864,33 @@ def launches_per_step(name, wl) -> int:
 # --------------------------------------------------------------------------- the oracle as a baseline
 
 def oracle_step_sample(o, wl, packed, row_stride: int):
-    """The oracle on every `row_stride`-th output column of every GEMM of
-    the step (all rows of X).  Returns the fraction of the step covered."""
+    """The oracle on every `row_stride`-th output column (all rows of X) of
+    the sampled GEMMs `packed` = [(index, W_host, X_host)].  Returns the
+    fraction of the whole step's multiply-adds covered."""
     covered = 0
-    for lin, (W, X) in zip(wl.linears, packed):
+    for i, W, X in packed:
+        lin = wl.linears[i]
         ns = np.arange(0, lin.N, row_stride)
         ms = np.repeat(np.arange(lin.M), len(ns))
         o.gemm_sampled(W, X, lin.M, lin.N, lin.K, ms, np.tile(ns, lin.M))
         covered += len(ns) * lin.M * lin.K
-    total = sum(l.M * l.N * l.K for l in wl.linears)
-    return covered / total
+    return covered / sum(l.M * l.N * l.K for l in wl.linears)
 
 
-def pack_on_host(wl, seed):
-    import oracle
-    o = oracle.get()
-    return o, [(o.pack(l.codes(seed), l.scales(seed)), l.x(seed)) for l in wl.linears]
+def _sample_macs(wl, packed):
+    return sum(wl.linears[i].M * wl.linears[i].N * wl.linears[i].K for i, _, _ in packed)
+
+
+def _what(wl, packed):
+    if len(packed) == len(wl.linears):
+        return f"all {len(wl.linears)} GEMMs"
+    return f"the {len(packed)} GEMMs of layers {', '.join(map(str, ORACLE_LAYERS))}"
 
 
 def cpu_baseline(wl, tensor: bool, budget_s: float, host=None):
-    o, packed = host or pack_on_host(wl, workloads.SEED)
-    total_macs = sum(l.M * l.N * l.K for l in wl.linears)
+    o, packed = host or pack_on_host(wl, workloads.SEED, sampled_linears(wl))
     # choose a column stride so one sampled pass is about budget/3 seconds (46 M MAC/s measured on one core)
-    est_rate = 4.5e7
-    stride = max(1, int(round(total_macs / (est_rate * budget_s / 3))))
+    stride = max(1, int(round(_sample_macs(wl, packed) / (4.5e7 * budget_s / 3))))
     frac_total, t0 = 0.0, time.perf_counter()
     reps = 0
     while True:
@@ -681,18 +904,19 @@ def cpu_baseline(wl, tensor: bool, budget_s: float, host=None):
     else:
         value, unit = frac_total * wl.hbm_bytes / dt / 1e9, "GB/s"
     return {"value": value, "unit": unit, "cores": 1, "kind": "oracle",
-            "sample": f"{reps} pass(es) over every {stride}th output column of all {len(wl.linears)} GEMMs "
+            "sample": f"{reps} pass(es) over every {stride}th output column of {_what(wl, packed)} "
                       f"({frac_total / reps:.4f} of a step each), {dt:.1f} s, scaled to whole steps"}
 
 
 def oracle_step_sample_threads(o, wl, packed, row_stride: int, pool, threads: int):
     """oracle_step_sample with the sampled columns dealt round-robin to
     `threads` host threads of `pool` (the oracle's C routine releases the
-    GIL).  Returns the fraction of the step covered."""
-    def part(i):
+    GIL).  Returns the fraction of the whole step covered."""
+    def part(t):
         covered = 0
-        for lin, (W, X) in zip(wl.linears, packed):
-            ns = np.arange(0, lin.N, row_stride)[i::threads]
+        for i, W, X in packed:
+            lin = wl.linears[i]
+            ns = np.arange(0, lin.N, row_stride)[t::threads]
             if len(ns):
                 o.gemm_sampled(W, X, lin.M, lin.N, lin.K, np.repeat(np.arange(lin.M), len(ns)), np.tile(ns, lin.M))
             covered += len(ns) * lin.M * lin.K
@@ -706,9 +930,8 @@ def cpu_baseline_all_cores(wl, tensor: bool, budget_s: float, threads: int = 0, 
     cores: one host thread per core."""
     import concurrent.futures
     threads = threads or os.cpu_count() or 1
-    o, packed = host or pack_on_host(wl, workloads.SEED)
-    total_macs = sum(l.M * l.N * l.K for l in wl.linears)
-    stride = max(1, int(round(total_macs / (4.5e7 * threads * budget_s / 3))))
+    o, packed = host or pack_on_host(wl, workloads.SEED, sampled_linears(wl))
+    stride = max(1, int(round(_sample_macs(wl, packed) / (4.5e7 * threads * budget_s / 3))))
     frac_total, reps, t0 = 0.0, 0, time.perf_counter()
     with concurrent.futures.ThreadPoolExecutor(max_workers=threads) as pool:
         while True:
@@ -722,7 +945,7 @@ def cpu_baseline_all_cores(wl, tensor: bool, budget_s: float, threads: int = 0, 
     else:
         value, unit = frac_total * wl.hbm_bytes / dt / 1e9, "GB/s"
     return {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
-            "sample": f"{reps} pass(es) over every {stride}th output column of all {len(wl.linears)} GEMMs, "
+            "sample": f"{reps} pass(es) over every {stride}th output column of {_what(wl, packed)}, "
                       f"columns dealt round-robin to {threads} threads ({frac_total / reps:.4f} of a step "
                       f"each), {dt:.1f} s, scaled to whole steps"}
 
@@ -733,11 +956,10 @@ def run_reference(args, rank: int, world: int):
     wl = workloads.workload(args.workload)
     tensor = args.workload in TENSOR_WORKLOADS
     import concurrent.futures
-    o, packed = pack_on_host(wl, workloads.SEED)
+    o, packed = pack_on_host(wl, workloads.SEED, sampled_linears(wl))
     threads = os.cpu_count() or 1
-    total_macs = sum(l.M * l.N * l.K for l in wl.linears)
     # each step: a sample of about 1 s of oracle work on every host core
-    stride = max(1, int(round(total_macs / (4.5e7 * threads))))
+    stride = max(1, int(round(_sample_macs(wl, packed) / (4.5e7 * threads))))
     with concurrent.futures.ThreadPoolExecutor(max_workers=threads) as pool:
         for _ in range(args.warmup):
             oracle_step_sample_threads(o, wl, packed, stride, pool, threads)
@@ -750,7 +972,7 @@ def run_reference(args, rank: int, world: int):
         value, unit = frac * wl.flops / dt / 1e12, "TFLOP/s"
     else:
         value, unit = frac * wl.hbm_bytes / dt / 1e9, "GB/s"
-    sample = (f"each step = every {stride}th output column of all {len(wl.linears)} GEMMs "
+    sample = (f"each step = every {stride}th output column of {_what(wl, packed)} "
               f"({frac / args.steps:.4f} of a step), columns dealt round-robin to {threads} host threads, "
               f"scaled to whole steps")
     return {
@@ -767,8 +989,11 @@ def run_reference(args, rank: int, world: int):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded Philox, same workload recipe)",
-        "config": {"workload": f"{wl.name}: {wl.description}", "bytes_per_step": wl.hbm_bytes,
-                   "flops_per_step": wl.flops, "parallelism": f"{threads} host threads"},
+        # the same keys as the GPU arm's config; l2 and parallelism say what this arm does
+        "config": {"workload": f"{wl.name}: {wl.description}", "gemms_per_step": len(wl.linears),
+                   "bytes_per_step": wl.hbm_bytes, "flops_per_step": wl.flops,
+                   "l2": "host run: the oracle reads its operands from host memory",
+                   "parallelism": f"{threads} host threads"},
         "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -787,6 +1012,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graphs", action="store_true",
                     help="launch each timed step eagerly instead of replaying its captured CUDA graph")
+    ap.add_argument("--only", action="store_true",
+                    help="measure the named workload alone (no records of the other configurations)")
     ap.add_argument("--soak", type=float, default=1.0,
                     help="seconds of untimed load after warm-up, so the clock sampler sees the GPU busy "
                          "(0 for short profiling runs)")

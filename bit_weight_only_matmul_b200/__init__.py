@@ -51,6 +51,7 @@ EXPORTS = (
     "q4_0_gather",
     "q4_0_quantize",
     "q4_0_selftest_wait_timeout",
+    "q4_0_stream_read",
     "q4_0_device_error",
     "q4_0_force_path",
 )
@@ -98,6 +99,7 @@ def _load() -> ctypes.CDLL:
         "q4_0_quantize": (i32, [vp, vp, i64, i64, vp]),
         "q4_0_device_error": (i32, [ctypes.POINTER(ctypes.c_uint32), i32]),
         "q4_0_selftest_wait_timeout": (i32, [ctypes.c_uint32, vp]),
+        "q4_0_stream_read": (i32, [vp, i64, i64, vp, vp]),
         "q4_0_force_path": (i32, [i32]),
     }
     for name, (res, args) in sig.items():
@@ -153,6 +155,13 @@ def q4_0_dequant(W, out, N: int, K: int, stream=None) -> None:
 def q4_0_gemm(W, X, Y, M: int, N: int, K: int, stream=None) -> None:
     """Y[M,N] = X[M,K] * dequant(W)^T; X bf16 (or int16 bit patterns), Y fp32."""
     _check(_lib.q4_0_gemm(_ptr(W), _ptr(X), _ptr(Y), M, N, K, _stream(stream)), "q4_0_gemm")
+
+
+def q4_0_stream_read(W, N: int, K: int, checksum, stream=None) -> None:
+    """Read the Q4_0 matrix W once with the decode kernels' weight stream and
+    XOR its 32-bit words into `checksum` (a one-element int32/uint32 CUDA
+    tensor the caller initialises): the read-only ceiling of that pattern."""
+    _check(_lib.q4_0_stream_read(_ptr(W), N, K, _ptr(checksum), _stream(stream)), "q4_0_stream_read")
 
 
 def q4_0_gemm_workspace_size(M: int, N: int, K: int) -> int:

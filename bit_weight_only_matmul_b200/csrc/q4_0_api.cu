@@ -323,6 +323,22 @@ int q4_0_interleave_gate_up(const void *W_gate, const void *W_up, void *W_gu, in
     return e == cudaSuccess ? Q4_OK : cuda_fail(e);
 }
 
+int q4_0_stream_read(const void *W, int64_t N, int64_t K, uint32_t *checksum, q4_0_stream_t stream) {
+    int st = check_dims(N, K);
+    if (st != Q4_OK) return st;
+    if (N == 0 || K == 0) return Q4_OK;
+    if (!W || !checksum || K % 256 != 0) return Q4_ERR_INVALID_ARG;
+    if (!aligned16(W)) return Q4_ERR_MISALIGNED;
+    if ((reinterpret_cast<uintptr_t>(checksum) & 3u) != 0) return Q4_ERR_MISALIGNED;
+    const q4::DeviceInfo *dev = nullptr;
+    st = current_device(&dev);
+    if (st != Q4_OK) return st;
+    if (!q4::stream_read_supports(N, K)) return Q4_ERR_INVALID_ARG;
+    const cudaError_t e = q4::launch_stream_read(static_cast<const uint8_t *>(W), N, K, checksum, *dev,
+                                                 reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? Q4_OK : cuda_fail(e);
+}
+
 int q4_0_selftest_wait_timeout(uint32_t limit_us, q4_0_stream_t stream) {
     if (limit_us < 1 || limit_us > 1000000) return Q4_ERR_INVALID_ARG;
     const q4::DeviceInfo *dev = nullptr;

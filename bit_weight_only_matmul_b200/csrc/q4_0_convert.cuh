@@ -56,20 +56,17 @@ __device__ __forceinline__ uint4 x8_to_fp16_permuted(uint4 v) {
     return make_uint4(lo.x, lo.y, hi.x, hi.y);
 }
 
-// Nonzero if any of the 8 bf16 values of v is finite and outside the range in
-// which the fp16 conversion above is exact: |x| >= 65536 (fp16 overflows to
-// inf) or 0 < |x| < 2^-17 (below 2^-17 a bf16 value can need more bits than
-// an fp16 subnormal has).  Per 16-bit half, a = |x| bits: bad iff
-// a - 1 < 0x36FF (1 <= a < 0x3700 = 2^-17) or a - 0x4780 < 0x3800
-// (0x4780 = 65536 <= a < 0x7F80 = inf).
+// Nonzero if any of the 8 bf16 values of v is finite and too large for fp16:
+// |x| >= 65536 (its fp16 conversion overflows to inf).  Per 16-bit half, with
+// a = |x| bits: 0x4780 = 65536 <= a < 0x7F80 = inf, i.e. a - 0x4780 < 0x3800.
+// (Values below the fp16 normal range are not flagged: bf16 values down to
+// 2^-17 convert exactly, and a smaller one is off by at most 2^-25, which
+// moves a product by at most 2^-25 |w|.)
 __device__ __forceinline__ uint32_t x8_fp16_range_bad(uint4 v) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     uint32_t bad = 0;
     #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t a = w[i] & 0x7FFF7FFFu;
-        bad |= __vcmpltu2(__vsub2(a, 0x00010001u), 0x36FF36FFu) | __vcmpltu2(__vsub2(a, 0x47804780u), 0x38003800u);
-    }
+    for (int i = 0; i < 4; ++i) bad |= __vcmpltu2(__vsub2(w[i] & 0x7FFF7FFFu, 0x47804780u), 0x38003800u);
     return bad;
 }
 

@@ -29,12 +29,18 @@
 //    (q - 8) * d pairs and feeds them as A fragments of 16 mma.sync per stage:
 //    with the scale folded into each weight, one MMA may mix blocks, so every
 //    byte a thread loads is its own;
-//  * an X warp per group converts the slot's X rows to fp16 straight into the
-//    MMA's B fragments, stored as pairs so that a compute thread fetches the
-//    two fragments of a code word with one 16-byte load;
+//  * the compute warps also convert the slot's X rows to fp16, straight into
+//    the MMA's B fragments: each takes a share of the (stage, X row) pairs,
+//    only the M real rows, one 16-byte chunk per lane, and arrives on the
+//    group's fragment barrier before it computes (a separate conversion warp
+//    got only a fair share of its scheduler's issue slots and could never run
+//    ahead, so compute warps waited on it); the fragments are stored as pairs
+//    so that a compute thread fetches the two fragments of a code word with
+//    one 16-byte load;
 //  * the accumulators (two chains) live across the whole item; at its end the
-//    group-1 warp hands its sums through shared memory to the group-0 warp of
-//    the same rows, which stores Y (optionally + R, or silu(gate) * up).
+//    group that worked the item's last slot stores Y (optionally + R, or
+//    silu(gate) * up), the other group's warps handing their sums over
+//    through a double-buffered exchange without waiting.
 // Split mode (up to q4split::kMaxItems items): launches of few items leave a
 // tail or idle SMs, so the CTAs run in clusters of CL (2 when there is at
 // least one item per SM, else 4, 6 or 8); items longer than the mean load of
@@ -65,13 +71,13 @@ using namespace q4dev;
 
 constexpr int kSub = 2;                               // 256-k stages per ring slot
 constexpr int kRawW = kItemRows * kStageRowBytes;     // 18432: one stage of 128 weight rows
-constexpr int kXPitch = 544;                          // X row pitch: 512 bytes + 32 (rows 8 banks apart)
-constexpr int kSubBytes = kRawW + 8 * kXPitch;        // 22784 (a multiple of 128)
-constexpr int kSlotBytes = kSub * kSubBytes;          // 45568
+constexpr int kXPitch = 512;                          // X row pitch: lanes read 16-byte chunks of one row at a time
+constexpr int kSubBytes = kRawW + 8 * kXPitch;        // 22528 (a multiple of 128)
+constexpr int kSlotBytes = kSub * kSubBytes;          // 45056
 constexpr int kXBufs = 4;                             // fragment buffers: group G uses G and G + 2
 
-constexpr int kWarpProd = 0, kWarpX0 = 1, kWarp0 = 3, kGroupWarps = 8;
-constexpr int kThreads = 32 * (kWarp0 + 2 * kGroupWarps);   // 608
+constexpr int kWarpProd = 0, kWarp0 = 1, kGroupWarps = 8;
+constexpr int kThreads = 32 * (kWarp0 + 2 * kGroupWarps);   // 544
 static_assert(kSubBytes % 128 == 0 && kXPitch % 16 == 0, "TMA and bulk-copy destinations stay aligned");
 
 using q4split::kMaxItems;
@@ -95,13 +101,13 @@ struct PartnerSums<1> {};
 
 template <int CL>
 struct Smem {
-    uint8_t raw[ring<CL>()][kSub][kSubBytes];   // per stage: W rows (pitch 144), then X rows (pitch 544)
+    uint8_t raw[ring<CL>()][kSub][kSubBytes];   // per stage: W rows (pitch 144), then X rows (pitch 512)
     uint4 frag[kXBufs][kSub][8][32];            // B fragment pairs: [buffer][stage][pair][lane]
-    float comb[8][4][32];                       // group-1 sums handed to group 0 at an item's end
+    float comb[2][8][4][32];                    // an item's sums handed to the group that stores it (by item parity)
     float epi[4][4][32];                        // SwiGLU: up-row sums handed to the gate rows
     uint64_t raw_full[ring<CL>()], raw_empty[ring<CL>()];
-    uint64_t frag_full[kXBufs], frag_empty[kXBufs];
-    uint64_t comb_full, comb_empty, epi_full, epi_empty;
+    uint64_t frag_full[kXBufs];
+    uint64_t comb_full[2], comb_empty[2], epi_full, epi_empty;
     PartnerSums<CL> x;
     int abort_flag;
 };
@@ -137,9 +143,8 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
     return v;
 }
 
-__device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                 : "memory");
+__device__ __forceinline__ void sts64(uint32_t a, uint32_t x, uint32_t y) {
+    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(a), "r"(x), "r"(y) : "memory");
 }
 
 __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -328,14 +333,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_m8_kernel(const __grid_con
     if (threadIdx.x == 0) {
         for (int s = 0; s < RS; ++s) {
             mbar_init(&S.raw_full[s], 1);
-            mbar_init(&S.raw_empty[s], kGroupWarps + 1);   // the group's compute warps and its X warp
+            mbar_init(&S.raw_empty[s], kGroupWarps);
         }
-        for (int s = 0; s < kXBufs; ++s) {
-            mbar_init(&S.frag_full[s], 1);
-            mbar_init(&S.frag_empty[s], kGroupWarps);
+        for (int s = 0; s < kXBufs; ++s) mbar_init(&S.frag_full[s], kGroupWarps);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&S.comb_full[s], kGroupWarps);
+            mbar_init(&S.comb_empty[s], kGroupWarps);
         }
-        mbar_init(&S.comb_full, kGroupWarps);
-        mbar_init(&S.comb_empty, kGroupWarps);
         mbar_init(&S.epi_full, kGroupWarps / 2);
         mbar_init(&S.epi_empty, kGroupWarps / 2);
         if constexpr (CL > 1) {
@@ -405,74 +409,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_m8_kernel(const __grid_con
                 ++prod_issued;
             }
         }
-    } else if (warp < kWarp0) {
-        // ---------------------------------------------------------------- X rows -> fp16 B fragments
-        // X warp G fills the fragments of its group's slots.  Lane (gx, tx):
-        // X row gx, blocks 2tx and 2tx+1 of each stage (its 128 bytes, read
-        // as 16-byte chunks: chunk c = 4B + 2h + W/2 holds the elements of
-        // code words W, W+1 of block 2tx+B, low (h = 0) or high (h = 1)
-        // nibble half).  Chunks c and c + 2 make fragment pairs 4B + W and
-        // 4B + W + 1; lane tx starts at a rotated chunk, so that with the
-        // 544-byte pitch each 8-lane phase of a 16-byte load hits 32 banks.
-        const int G = warp - kWarpX0;
-        const int gx = lane >> 2, tx = lane & 3;
-        RingPos<RS> rp{G, 0};
-        int k = 0;   // slots of this group so far
-        uint32_t g = 0;
-        Items<CL> it;
-        bool ok = true;
-        while (ok && it.next(D, rank)) {
-            const GroupProblem &pr = P.p[it.prob];
-            const bool active = gx < pr.M;
-            // every problem's X is range-checked once, by the CTA (or cluster)
-            // that works its first item
-            const bool check = it.row0 == 0;
-            uint32_t xbad = 0;
-            const int n = (it.s1 - it.s0 + kSub - 1) / kSub;
-            for (int j = (G - static_cast<int>(g)) & 1; j < n; j += 2, ++k, rp.advance(2)) {
-                const int cnt = min(kSub, it.s1 - (it.s0 + kSub * j));
-                const int xb = G + 2 * (k & 1);
-                if (lane == 0) {
-                    ok = wait_or_abort(&S.raw_full[rp.slot], rp.phase, &S.abort_flag, P.err);
-                    if (ok) ok = wait_or_abort(&S.frag_empty[xb], ((k >> 1) & 1) ^ 1, &S.abort_flag, P.err);
-                }
-                if (!__shfl_sync(0xffffffffu, ok, 0)) { ok = false; break; }
-                #pragma unroll
-                for (int i = 0; i < kSub; ++i) {
-                    if (i >= cnt) break;
-                    const uint32_t xr = raw0 + rp.slot * kSlotBytes + i * kSubBytes + kRawW + gx * kXPitch + 128 * tx;
-                    const uint32_t fo = frag0 + (xb * kSub + i) * 4096 + lane * 16;
-                    #pragma unroll
-                    for (int pp = 0; pp < 4; ++pp) {
-                        const int v = (pp + tx) & 3;
-                        const int c = (v & 1) | ((v & 2) << 1);          // 0, 1, 4, 5
-                        uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
-                        if (active) {
-                            const uint4 rl = lds128(xr + 16 * c), rh = lds128(xr + 16 * (c + 2));
-                            if (check) xbad |= x8_fp16_range_bad(rl) | x8_fp16_range_bad(rh);
-                            lo = x8_to_fp16_permuted(rl);
-                            hi = x8_to_fp16_permuted(rh);
-                        }
-                        const int p = 4 * (c >> 2) + 2 * (c & 1);       // pair of code word W = 2 (c & 1)
-                        sts128(fo + p * 512, make_uint4(lo.x, lo.y, hi.x, hi.y));
-                        sts128(fo + (p + 1) * 512, make_uint4(lo.z, lo.w, hi.z, hi.w));
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&S.frag_full[xb]);
-                    mbar_arrive(&S.raw_empty[rp.slot]);
-                }
-            }
-            if (xbad) atomicOr(P.err, (unsigned)Q4_DEVERR_FP16_RANGE);
-            g += n;
-        }
     } else {
         // ---------------------------------------------------------------- compute
         const int cw = warp - kWarp0;
         const int G = cw >> 3, tile = cw & 7;   // slot parity, rows 16*tile .. 16*tile+15
         const int gq = lane >> 2, t = lane & 3;
         const uint32_t wbase = raw0 + (16 * tile + gq) * kStageRowBytes + 36 * t;
+        // X conversion: lane L takes elements 8L .. 8L+7 of a stage row, i.e.
+        // chunk c = L & 7 of window tx = L >> 3 (blocks 2tx and 2tx+1); chunk
+        // c = 4B + 2h + W/2 holds code words W, W+1 of block 2tx+B, low (h = 0)
+        // or high (h = 1) nibble half, which become half h of fragment pairs
+        // 4B + W and 4B + W + 1 of B-fragment lane 4m + tx.  Only the M real
+        // rows are converted: fragment columns past M feed accumulator columns
+        // that are never stored, so whatever they hold is harmless.
+        const int cx = lane & 7;
+        const uint32_t fl = (4 * (cx >> 2) + 2 * (cx & 1)) * 512 + (lane >> 3) * 16 + ((cx >> 1) & 1) * 8;
+        uint32_t xbad = 0;
         float acc[2][4];
         #pragma unroll
         for (int c = 0; c < 2; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.f;
@@ -482,14 +434,37 @@ __global__ void __launch_bounds__(kThreads, 1) decode_m8_kernel(const __grid_con
         Items<CL> it;
         while (it.next(D, rank)) {
             const int n = (it.s1 - it.s0 + kSub - 1) / kSub;
+            const int M = P.p[it.prob].M;
+            // every problem's X is range-checked once, by the CTA (or cluster)
+            // that works its first item
+            const bool check = it.row0 == 0;
             bool ok = true;
             for (int j = (G - static_cast<int>(g)) & 1; j < n; j += 2, ++k, rp.advance(2)) {
                 const int cnt = min(kSub, it.s1 - (it.s0 + kSub * j));
                 const int xb = G + 2 * (k & 1);
-                // the slot's words into registers, then the slot goes back to the
-                // producer at once (a stage that is not part of the item -- cnt = 1
-                // -- is read but not used)
                 if (!(ok = wait_or_abort(&S.raw_full[rp.slot], rp.phase, &S.abort_flag, P.err))) break;
+                // this warp's share of the slot's X rows -> fp16 B fragments:
+                // (stage, row) pairs tile and tile + 8 of the cnt * M pairs.
+                // Buffer xb was last read by the group's slot k - 2; every warp
+                // finished that before it arrived on the fragment barrier of
+                // slot k - 1, which this warp has passed.
+                {
+                    const uint32_t xr = raw0 + rp.slot * kSlotBytes + kRawW + lane * 16;
+                    const uint32_t fo = frag0 + xb * kSub * 4096 + fl;
+                    for (int pi = tile; pi < cnt * M; pi += kGroupWarps) {
+                        const int i = pi >= M ? 1 : 0, m = pi - i * M;
+                        const uint4 v = lds128(xr + i * kSubBytes + m * kXPitch);
+                        if (check) xbad |= x8_fp16_range_bad(v);
+                        const uint4 o = x8_to_fp16_permuted(v);
+                        sts64(fo + i * 4096 + m * 64, o.x, o.y);
+                        sts64(fo + i * 4096 + 512 + m * 64, o.z, o.w);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.frag_full[xb]);
+                // the slot's words into registers, then the slot goes back to the
+                // producer (a stage that is not part of the item -- cnt = 1 -- is
+                // read but not used)
                 const uint32_t w = wbase + rp.slot * kSlotBytes;
                 uint32_t r[kSub][9], r8[kSub][9];
                 #pragma unroll
@@ -500,35 +475,40 @@ __global__ void __launch_bounds__(kThreads, 1) decode_m8_kernel(const __grid_con
                 const uint32_t fa = frag0 + xb * kSub * 4096 + lane * 16;
                 stage_mma(r[0], r8[0], fa, acc);
                 if (cnt > 1) stage_mma(r[1], r8[1], fa + 4096, acc);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&S.frag_empty[xb]);
             }
             if (!ok) break;
-            g += n;
             // ------------------------------------------------------------ end of the item
+            // The group that worked the item's last slot stores it; the other
+            // group hands its sums over (buffer by item parity) and goes on.
             const GroupProblem &pr = P.p[it.prob];
-            const uint32_t par = items_done & 1;
+            const int last = static_cast<int>((g + n - 1) & 1);
+            g += n;
+            const int cb = items_done & 1;
+            const uint32_t cpar = (items_done >> 1) & 1;
             ++items_done;
-            if (G == 1) {
-                if (!wait_or_abort(&S.comb_empty, par ^ 1, &S.abort_flag, P.err)) break;
+            // every warp counts the split and SwiGLU items, whichever group stores them
+            const uint32_t split_k = split_done, swiglu_k = swiglu_done;
+            if (it.split) ++split_done;
+            if (pr.epi == kEpiSwiGLU && (!it.split || rank == 0)) ++swiglu_done;
+            if (G != last) {
+                if (!wait_or_abort(&S.comb_empty[cb], cpar ^ 1, &S.abort_flag, P.err)) break;
                 #pragma unroll
-                for (int e = 0; e < 4; ++e) S.comb[tile][e][lane] = acc[0][e] + acc[1][e];
+                for (int e = 0; e < 4; ++e) S.comb[cb][tile][e][lane] = acc[0][e] + acc[1][e];
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&S.comb_full);
+                if (lane == 0) mbar_arrive(&S.comb_full[cb]);
             } else {
-                if (!wait_or_abort(&S.comb_full, par, &S.abort_flag, P.err)) break;
+                if (!wait_or_abort(&S.comb_full[cb], cpar, &S.abort_flag, P.err)) break;
                 float sum[4];
                 #pragma unroll
-                for (int e = 0; e < 4; ++e) sum[e] = acc[0][e] + acc[1][e] + S.comb[tile][e][lane];
+                for (int e = 0; e < 4; ++e) sum[e] = acc[0][e] + acc[1][e] + S.comb[cb][tile][e][lane];
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&S.comb_empty);
+                if (lane == 0) mbar_arrive(&S.comb_empty[cb]);
                 if constexpr (CL > 1) {
                     if (it.split) {
                         // ranks 1..CL-1 hand their sums to rank 0 of the cluster, which adds
                         // them in rank order
-                        const int xb2 = split_done & 1;
-                        const uint32_t xpar = (split_done >> 1) & 1;
-                        ++split_done;
+                        const int xb2 = split_k & 1;
+                        const uint32_t xpar = (split_k >> 1) & 1;
                         if (rank != 0) {
                             if (!wait_cluster_or_abort(&S.x.empty[xb2], xpar ^ 1, &S.abort_flag, P.err)) break;
                             #pragma unroll
@@ -564,8 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_m8_kernel(const __grid_con
                     // rows 0-63 of the item are gate rows of features row0/2 .. row0/2+63,
                     // rows 64-127 the up rows of the same features: tiles 4-7 hand their
                     // sums to tiles 0-3, which store silu(gate) * up into Y[M, N/2]
-                    const uint32_t epar = swiglu_done & 1;
-                    ++swiglu_done;
+                    const uint32_t epar = swiglu_k & 1;
                     if (tile >= 4) {
                         if (!wait_or_abort(&S.epi_empty, epar ^ 1, &S.abort_flag, P.err)) break;
                         #pragma unroll
@@ -600,6 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_m8_kernel(const __grid_con
             #pragma unroll
             for (int c = 0; c < 2; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.f;
         }
+        if (xbad) atomicOr(P.err, (unsigned)Q4_DEVERR_FP16_RANGE);
     }
 
     __syncthreads();

@@ -403,12 +403,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
         // 8-byte stores in sixteen bank pairs.
         const int G = warp - kWarpX0;
         const int gx = lane >> 2, tx = lane & 3;
-        uint32_t g = 0;
+        uint32_t g = 0, xbad = 0;
         Walk<CL, SUB> q{};
         q.start(D, rank);
         for (; q.item >= 0; q.next(D, rank), ++g) {
             if ((g & 1) != static_cast<uint32_t>(G)) continue;
             const GroupProblem &pr = P.p[q.prob];
+            // every problem's X is range-checked once, by the CTA (or cluster)
+            // that works its first item
+            const bool check = q.row0 == 0;
             const int slot = g % RS, xb = g % kXBufs;
             bool ok = true;
             if (lane == 0) {
@@ -416,6 +419,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
                 if (ok) ok = wait_or_abort(&S.xf_empty[xb], ((g / kXBufs) & 1) ^ 1, &S.abort_flag, P.err);
             }
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            if (check) {
+                // a separate pass, so that the conversion below stays as it is
+                // for every other item: this lane's 16-byte pieces of its rows
+                for (int i = 0; i < q.cnt && i < SUB; ++i) {
+                    const uint8_t *xr = S.raw[slot][i] + kRawW;
+                    for (int j = 0; j < NT; ++j) {
+                        const int m = 8 * j + gx;
+                        if (m >= pr.M) continue;
+                        for (int piece = 0; piece < 8; ++piece) {
+                            const int k = 64 * tx + 8 * piece;
+                            const uint8_t *src = xmap<NT>() ? xr + tx * xbox_bytes<NT>() + m * 128 +
+                                                                  ((((k & 63) >> 3) ^ (m & 7)) << 4)
+                                                            : xr + m * kXPitch + 2 * k;
+                            xbad |= x8_fp16_range_bad(*reinterpret_cast<const uint4 *>(src));
+                        }
+                    }
+                }
+            }
             #pragma unroll
             for (int i = 0; i < SUB; ++i) {
                 if (i >= q.cnt) break;
@@ -430,7 +451,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
                             #pragma unroll
                             for (int wp = 0; wp < 2; ++wp) {
                                 uint4 o = make_uint4(0u, 0u, 0u, 0u);
-                                if (m < pr.M) {
+                                // TMA boxes (M > 8) zero-fill the rows past M, so every row
+                                // converts unconditionally (straight-line loads); 1-D copies
+                                // (M <= 8) leave those rows stale
+                                if (xmap<NT>() || m < pr.M) {
                                     const int k = 32 * (2 * tx + xw) + 16 * h + 8 * wp;
                                     // box tx holds k 64tx..64tx+63; its 16-byte chunk c of row m
                                     // sits at chunk c ^ (m & 7) (128-byte swizzle)
@@ -451,6 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
                 mbar_arrive(&S.raw_empty[slot]);
             }
         }
+        if (xbad) atomicOr(P.err, (unsigned)Q4_DEVERR_FP16_RANGE);
     } else {
         // ---------------------------------------------------------------- compute
         const int cw = warp - kWarp0;
@@ -545,6 +570,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
                         }
                     }
                     // thread holds rows gq / gq+8 of the tile x columns 8j+2t, 8j+2t+1
+                    if (!q.split || rank == 0) {
+                        // a non-finite sum from finite inputs means an fp16 weight
+                        // overflowed: look at the rows' scales (slow path, rare)
+                        bool bad_row[2] = {false, false};
+                        #pragma unroll
+                        for (int j = 0; j < NT; ++j)
+                            #pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                if (8 * j + 2 * t + (e & 1) < pr.M && !(fabsf(sum[j][e]) <= 3.402823466e38f))
+                                    bad_row[e >> 1] = true;
+                        #pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            if (bad_row[h]) {
+                                const int64_t nn = q.row0 + 16 * tile + gq + 8 * h;
+                                scan_scales_fp16_range(pr.W, nn, nn + 1, pr.N, pr.K, P.err);
+                            }
+                    }
                     if ((!q.split || rank == 0) && pr.epi == kEpiSwiGLU) {
                         // rows 0-63 of the item are gate rows of features row0/2 .. row0/2+63,
                         // rows 64-127 the up rows of the same features: tiles 4-7 hand their

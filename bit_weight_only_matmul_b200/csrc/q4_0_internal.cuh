@@ -99,6 +99,11 @@ cudaError_t launch_decode(const Problem *probs, int count, const DeviceInfo &dev
 // problem must satisfy decode_tmem_supports().
 bool decode_tmem_supports(const Problem &p);
 cudaError_t launch_decode_tmem(const Problem *probs, int count, const DeviceInfo &dev, cudaStream_t s);
+// Read-only stream of a Q4_0 matrix with the decode kernels' TMA boxes (the
+// measurement behind q4_0_stream_read).
+bool stream_read_supports(int64_t N, int64_t K);
+cudaError_t launch_stream_read(const uint8_t *W, int64_t N, int64_t K, uint32_t *checksum, const DeviceInfo &dev,
+                               cudaStream_t s);
 // Tensor-core kernel: every problem must satisfy prefill_supports().  With a
 // workspace of at least prefill_workspace_bytes() X is converted to fp16 once
 // by a pre-pass; without one the kernel converts each X tile it loads.

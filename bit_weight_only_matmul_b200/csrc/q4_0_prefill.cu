@@ -71,6 +71,7 @@ struct alignas(64) PrefillParams {
     CUtensorMap tmap_x;    // bf16 [M, K], box 64 x 256, 128-byte swizzle
     CUtensorMap tmap_w;    // uint8 [N, K/32*18], box 144 x 128
     float *Y;
+    const uint8_t *W;      // the Q4_0 weights (read directly only by the rare scale check)
     unsigned *err;
     int M, N, K;
     int tiles_n, tiles_m;
@@ -287,9 +288,12 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
         // 8 consecutive lanes take the 8 16-byte chunks of one row (the
         // conversion is chunk-local, so the swizzled order does not matter)
         const int cw = warp - kWarpCvt0;
-        uint32_t xc = 0;
+        uint32_t xc = 0, xbad = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            // the tiles of the first weight-row tile range-check X: every
+            // activation row once
+            const bool check = t % P.tiles_n == 0;
             for (int ks = 0; ks < ksteps; ++ks) {
                 const int s = xc % kXStages;
                 if (!(ok = wait_or_abort(&S.x_full[s], (xc / kXStages) & 1, S, P.err))) break;
@@ -297,8 +301,10 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
                 for (int it = 0; it < 8; ++it) {
                     const int row = 32 * cw + 4 * it + (lane >> 3);
                     uint4 *p = reinterpret_cast<uint4 *>(S.x[s] + row * 128 + 16 * (lane & 7));
-                    const uint4 o = x8_to_fp16_permuted(*p);
-                    *p = o;
+                    const uint4 v = *p;
+                    // rows past M are zero-filled by the load
+                    if (check) xbad |= x8_fp16_range_bad(v);
+                    *p = x8_to_fp16_permuted(v);
                 }
                 // make the generic-proxy writes visible to the tensor core (async proxy)
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -307,6 +313,7 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
                 ++xc;
             }
         }
+        if (xbad) atomicOr(P.err, (unsigned)Q4_DEVERR_FP16_RANGE);
     } else {   // epilogue warps
         const int quad = warp & 3;
         uint32_t dc = 0;
@@ -315,6 +322,8 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
             tc_fence_after();
             const int n0 = (t % P.tiles_n) * kTileN, m0 = (t / P.tiles_n) * kTileM;
             const int n = n0 + 32 * quad + lane;
+            // a non-finite sum shows in the running value sum_j v[j] * 0
+            float nonfinite = 0.f;
             #pragma unroll 1
             for (int c = 0; c < kTileM / 32; ++c) {
                 float v[32];
@@ -323,13 +332,19 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
                 if (n < P.N) {
                     #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        // streaming store: Y is not read again here, X and W tiles are
-                        if (mb + j < P.M) __stcs(P.Y + static_cast<int64_t>(mb + j) * P.N + n, v[j]);
+                        if (mb + j < P.M) {
+                            nonfinite = fmaf(v[j], 0.f, nonfinite);
+                            // streaming store: Y is not read again here, X and W tiles are
+                            __stcs(P.Y + static_cast<int64_t>(mb + j) * P.N + n, v[j]);
+                        }
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.d_empty);
+            // a non-finite sum from finite inputs means an fp16 weight
+            // overflowed: look at this row's scales (slow path, rare)
+            if (nonfinite != 0.f) scan_scales_fp16_range(P.W, n, n + 1, P.N, P.K, P.err);
         }
     }
 
@@ -348,11 +363,15 @@ constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 // bf16 X -> fp16 X' in the permuted k order of the A operand (positions 1 and
 // 2 of every 4 swapped), 8 elements per thread.  Exact for |x| in the fp16
 // normal range.
-__global__ void x_to_fp16_kernel(const uint4 *__restrict__ X, uint4 *__restrict__ Xh, int64_t n8) {
+// Also flags Q4_DEVERR_FP16_RANGE for values too large for fp16.
+__global__ void x_to_fp16_kernel(const uint4 *__restrict__ X, uint4 *__restrict__ Xh, int64_t n8, unsigned *err) {
+    uint32_t bad = 0;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
-        const uint4 o = x8_to_fp16_permuted(__ldg(X + i));
-        Xh[i] = o;
+        const uint4 v = __ldg(X + i);
+        bad |= x8_fp16_range_bad(v);
+        Xh[i] = x8_to_fp16_permuted(v);
     }
+    if (bad) atomicOr(err, (unsigned)Q4_DEVERR_FP16_RANGE);
 }
 
 }  // namespace
@@ -387,7 +406,7 @@ cudaError_t launch_prefill(const Problem &p, const DeviceInfo &dev, cudaStream_t
         const int64_t blocks = (n8 + 255) / 256;
         const int grid = static_cast<int>(blocks < dev.sm_count * 8 ? blocks : dev.sm_count * 8);
         x_to_fp16_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const uint4 *>(p.X), static_cast<uint4 *>(workspace),
-                                              n8);
+                                              n8, dev.err);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -396,6 +415,7 @@ cudaError_t launch_prefill(const Problem &p, const DeviceInfo &dev, cudaStream_t
         !get_tensor_map(&local.tmap_w, p.W, p.N, p.K / 32 * 18, kMapWeights128Prefill))
         return cudaErrorInvalidValue;
     local.Y = p.Y;
+    local.W = p.W;
     local.err = dev.err;
     local.M = static_cast<int>(p.M);
     local.N = static_cast<int>(p.N);

@@ -71,10 +71,10 @@ enum {
 enum {
     Q4_DEVERR_WAIT_TIMEOUT = 1u,   /* a bounded on-chip wait gave up; the output is incomplete */
     Q4_DEVERR_BAD_INDEX = 2u,      /* q4_0_gather met an id outside [0, V) (its row was zeroed) */
-    Q4_DEVERR_FP16_RANGE = 4u      /* a fast GEMM path met an operand its fp16 arithmetic does not hold
-                                      exactly: a finite X with |x| > 65504 or 0 < |x| < 2^-17, or a
-                                      scale with 8188 < |d| < inf; its output may hold +-inf or lost
-                                      precision (q4_0_force_path(4) computes such inputs exactly) */
+    Q4_DEVERR_FP16_RANGE = 4u      /* a fast GEMM path met an operand too large for its fp16
+                                      arithmetic: a finite X with |x| > 65504, or a scale with
+                                      8188 < |d| < inf; its output may hold +-inf (q4_0_force_path(4)
+                                      computes such inputs exactly) */
 };
 
 /* Largest N, K and M accepted (each dimension below 2^31). */
@@ -124,12 +124,12 @@ Q4_0_API int q4_0_dequant(const void *W, float *out, int64_t N, int64_t K,
  * tcgen05 tensor-core kernel (weight tiles dequantized into tensor memory,
  * fp32 accumulators in tensor memory).  Both feed the tensor cores fp16
  * operands: each weight (q - 8) * d is rounded once to fp16 (relative error
- * <= 2^-11) and X is converted to fp16, exactly for 2^-17 <= |x| <= 65504.
- * An operand outside that (a finite |x| > 65504 or 0 < |x| < 2^-17, a scale
- * 8188 < |d| < inf) is detected on the GPU and sets Q4_DEVERR_FP16_RANGE in
- * q4_0_device_error: the output may then hold +-inf or lost precision.
- * q4_0_force_path(4) selects an exact-arithmetic decode kernel ((q - 8)
- * exact in bf16, X used as given) without that restriction. */
+ * <= 2^-11) and X is converted to fp16: exactly for 2^-17 <= |x| <= 65504,
+ * with an absolute error below 2^-25 for smaller |x|.  An operand too large
+ * for fp16 (a finite |x| > 65504, a scale 8188 < |d| < inf) is detected on
+ * the GPU and sets Q4_DEVERR_FP16_RANGE in q4_0_device_error: the output may
+ * then hold +-inf.  q4_0_force_path(4) selects an exact-arithmetic decode
+ * kernel ((q - 8) exact in bf16, X used as given) without that restriction. */
 Q4_0_API int q4_0_gemm(const void *W, const uint16_t *X, float *Y,
               int64_t M, int64_t N, int64_t K, q4_0_stream_t stream);
 
@@ -238,6 +238,18 @@ Q4_0_API int q4_0_interleave_gate_up(const void *W_gate, const void *W_up, void 
  * lets a test show that a bounded wait ends and reports, without any fault.
  * Asynchronous on `stream` like every call. */
 Q4_0_API int q4_0_selftest_wait_timeout(uint32_t limit_us, q4_0_stream_t stream);
+
+/* A measurement instrument (no counterpart on the pages): read the Q4_0
+ * matrix W (N rows, K weights each) once from device memory with the same
+ * weight stream the decode kernels use -- TMA boxes of 128 rows x 144 bytes
+ * (256 k) into a ring of shared-memory slots, one persistent CTA per SM,
+ * each CTA walking along K of one 128-row item and then the next -- and do
+ * nothing with the bytes but XOR their 32-bit words into *checksum (a device
+ * word the caller initialises; rows past N read as zero).  The bandwidth this
+ * reaches is the ceiling of the decode kernels' access pattern: what they
+ * would stream if their arithmetic were free.  W 16-byte aligned, checksum
+ * 4-byte aligned, K % 256 == 0; N == 0 or K == 0 is a no-op. */
+Q4_0_API int q4_0_stream_read(const void *W, int64_t N, int64_t K, uint32_t *checksum, q4_0_stream_t stream);
 
 /* Row gather (a Q4 embedding lookup): out[t, :] = dequant(W)[ids[t], :] for
  * t < T, W a Q4_0 matrix of V rows by D weights, out float32 [T, D] row-major

@@ -154,6 +154,17 @@ def test_selftest_argument_checks(q4):
     assert q4.lib.q4_0_selftest_wait_timeout(1000001, None) == q4.Q4_ERR_INVALID_ARG
 
 
+def test_stream_read_argument_checks(q4):
+    f = q4.lib.q4_0_stream_read
+    assert f(A, 0, 256, A, None) == q4.Q4_OK               # nothing to read
+    assert f(None, 4, 256, A, None) == q4.Q4_ERR_INVALID_ARG
+    assert f(A, 4, 256, None, None) == q4.Q4_ERR_INVALID_ARG
+    assert f(A, 4, 96, A, None) == q4.Q4_ERR_INVALID_ARG   # K % 256 != 0
+    assert f(A, 4, 250, A, None) == q4.Q4_ERR_INVALID_ARG  # K % 32 != 0
+    assert f(A + 8, 4, 256, A, None) == q4.Q4_ERR_MISALIGNED
+    assert f(A, 4, 256, A + 2, None) == q4.Q4_ERR_MISALIGNED
+
+
 def test_header_is_plain_c_and_matches_the_binding(q4, tmp_path):
     """include/q4_0.h compiles as C99 with no CUDA header, and the problem
     structs the binding builds with ctypes have the C layout: same size, same

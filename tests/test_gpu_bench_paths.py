@@ -1,0 +1,165 @@
+"""The launch patterns the bench and a token loop use, against the float64
+oracle: the workspace path (X converted to fp16 once, the bench's M > 32
+path) at the full adapter and QKV sizes, decode launches back to back with
+programmatic dependent launch where the second consumes the first's output,
+and grouped calls running concurrently on two streams (the library's
+per-thread and per-device host state under concurrent use)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests.gpu_helpers import build_workload, check_built, check_gemm, dev, no_device_error, pack_on_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def q4():
+    import bit_weight_only_matmul_b200 as q4
+    q4.q4_0_force_path(q4.PATH_AUTO)
+    yield q4
+    q4.q4_0_force_path(q4.PATH_AUTO)
+
+
+@pytest.fixture(autouse=True)
+def _clean_error_word(q4):
+    q4.q4_0_device_error(clear=True)
+    yield
+    no_device_error(q4)
+
+
+def _weights(rng, N, K):
+    codes = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
+    scales = (np.abs(rng.standard_normal((N, K // 32))) * 0.002 + 1e-4).astype(np.float16).view(np.uint16)
+    return codes, scales
+
+
+def _x(rng, M, K):
+    return workloads.fp32_to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+
+
+@pytest.mark.parametrize("name", ["adapter", "qkv_prefill"])
+def test_workspace_path_full_size_sampled(q4, name):
+    """q4_0_gemm_ws with a full workspace, the path the bench times for
+    M = 4096, at the configuration's full size: 2000 sampled outputs against
+    the oracle, and bit-equal to the path that converts X tile by tile."""
+    b = build_workload(q4, workloads.workload(name), samples=2000)
+    (W, X, Y, M, N, K), = b.problems()
+    ws = torch.empty(q4.q4_0_gemm_workspace_size(M, N, K), dtype=torch.uint8, device="cuda")
+    q4.q4_0_gemm_ws(W, X, Y, M, N, K, ws)
+    check_built(b, f"{name} through the workspace")
+    Y2 = torch.full_like(Y, float("nan"))
+    q4.q4_0_gemm(W, X, Y2, M, N, K)
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y2)
+
+
+@pytest.mark.parametrize("M", [1, 2, 16])
+def test_back_to_back_residual_chain(q4, M):
+    """Two fused decode launches queued back to back on one stream: the
+    second's residual R is the first's output Y1 (Y2 = X2 W2^T + Y1).  With
+    programmatic dependent launch the second grid starts while the first
+    drains and must still read the finished Y1."""
+    rng = np.random.default_rng(40 + M)
+    o = oracle.get()
+    N, K = 3072, 3072
+    (c1, s1), (c2, s2) = _weights(rng, N, K), _weights(rng, N, K)
+    X1, X2 = _x(rng, M, K), _x(rng, M, K)
+    R0 = rng.standard_normal((M, N)).astype(np.float32)
+    W1, W2 = pack_on_gpu(q4, c1, s1), pack_on_gpu(q4, c2, s2)
+    R0d = dev(R0)
+    for rep in range(3):
+        Y1 = torch.full((M, N), float("nan"), device="cuda")
+        Y2 = torch.full((M, N), float("nan"), device="cuda")
+        q4.q4_0_gemm_grouped_ex([(W1, dev(X1), Y1, M, N, K, R0d, q4.Q4_0_EPI_RESIDUAL)])
+        q4.q4_0_gemm_grouped_ex([(W2, dev(X2), Y2, M, N, K, Y1, q4.Q4_0_EPI_RESIDUAL)])
+        torch.cuda.synchronize()
+        ya, ba = o.gemm(o.pack(c1, s1), X1, M, N, K)
+        yb, bb = o.gemm(o.pack(c2, s2), X2, M, N, K)
+        ref1 = ya + R0
+        ref2 = yb + ref1
+        t1 = 1e-3 * ba + 1e-6 + 2.0**-22 * np.abs(ref1)
+        err1 = np.abs(Y1.cpu().numpy().astype(np.float64) - ref1)
+        assert (err1 <= t1).all(), f"first launch: worst {float((err1 / t1).max())}"
+        # the second inherits the first's error through R
+        err2 = np.abs(Y2.cpu().numpy().astype(np.float64) - ref2)
+        t2 = 1e-3 * bb + 1e-6 + t1 + 2.0**-22 * np.abs(ref2)
+        assert (err2 <= t2).all(), f"chained launch: worst {float((err2 / t2).max())}"
+
+
+def test_two_streams_concurrently(q4):
+    """Two grouped calls with different shape sets on two streams, issued
+    alternately so that their kernels can overlap on the device: a decode
+    layer at M=2 and a set of M=1 / M=32 GEMMs; each result against the
+    oracle."""
+    rng = np.random.default_rng(11)
+    o = oracle.get()
+    sets = {
+        "a": [(2, 5120, 3072), (2, 3072, 3072), (2, 3072, 8192)],
+        "b": [(1, 1000, 1024), (32, 640, 2048), (7, 129, 768)],
+    }
+    built = {}
+    for key, shapes in sets.items():
+        items = []
+        for (M, N, K) in shapes:
+            codes, scales = _weights(rng, N, K)
+            X = _x(rng, M, K)
+            items.append((codes, scales, X, pack_on_gpu(q4, codes, scales), dev(X),
+                          torch.full((M, N), float("nan"), device="cuda"), M, N, K))
+        built[key] = items
+    sa, sb = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    for rep in range(4):
+        for key, s in (("a", sa), ("b", sb)):
+            with torch.cuda.stream(s):
+                q4.q4_0_gemm_grouped([(W, X, Y, M, N, K) for (_, _, _, W, X, Y, M, N, K) in built[key]])
+    sa.synchronize()
+    sb.synchronize()
+    for key, items in built.items():
+        for codes, scales, X, W, Xd, Y, M, N, K in items:
+            Y_or, B_or = o.gemm(o.pack(codes, scales), X, M, N, K)
+            check_gemm(Y.cpu().numpy(), Y_or, B_or, f"stream {key} {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("N,K", [(1, 256), (129, 3072), (3072, 8192), (1000, 5120)])
+def test_stream_read_checksum(q4, N, K):
+    """The streaming-ceiling instrument reads every byte of W once: its XOR of
+    W's 32-bit words equals the same XOR on the host (rows past N count as
+    zero)."""
+    rng = np.random.default_rng(N + K)
+    W = rng.integers(0, 256, size=q4.q4_0_bytes(N, K), dtype=np.uint8)
+    cs = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q4.q4_0_stream_read(dev(W), N, K, cs)
+    torch.cuda.synchronize()
+    want = int(np.bitwise_xor.reduce(W.view(np.uint32)))
+    assert int(cs.cpu().numpy().view(np.uint32)[0]) == want
+
+
+@pytest.mark.parametrize("M,N,K", [(512, 18944, 256), (176, 300, 512), (177, 128, 1024), (4096, 256, 768)])
+def test_tensor_core_tiles_sampled(q4, M, N, K):
+    """The tensor-core kernel on one and several activation tiles (ragged last
+    tiles included, a grid of two tiles per SM): sampled outputs against the
+    oracle, through both the in-kernel and the workspace conversion of X,
+    which must agree bit for bit."""
+    rng = np.random.default_rng(M + N + K)
+    codes, scales = _weights(rng, N, K)
+    X = _x(rng, M, K)
+    W = pack_on_gpu(q4, codes, scales)
+    Xd = dev(X)
+    o = oracle.get()
+    W_host = o.pack(codes, scales)
+    ms = rng.integers(0, M, size=1500)
+    ns = rng.integers(0, N, size=1500)
+    ms[:4] = [0, M - 1, M - 1, min(M - 1, 175)]
+    ns[:4] = [0, N - 1, 0, N - 1]
+    Y_or, B_or = o.gemm_sampled(W_host, X, M, N, K, ms, ns)
+    Y1 = torch.full((M, N), float("nan"), device="cuda")
+    q4.q4_0_gemm(W, Xd, Y1, M, N, K)
+    ws = torch.empty(q4.q4_0_gemm_workspace_size(M, N, K), dtype=torch.uint8, device="cuda")
+    Y2 = torch.full((M, N), float("nan"), device="cuda")
+    q4.q4_0_gemm_ws(W, Xd, Y2, M, N, K, ws)
+    torch.cuda.synchronize()
+    check_gemm(Y1.cpu().numpy()[ms, ns], Y_or, B_or, f"tensor core {M}x{N}x{K}")
+    assert torch.equal(Y1, Y2)
