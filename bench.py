@@ -51,12 +51,12 @@ DEFAULT_WORKLOAD = "cfg_decode"
 
 # kernel that dominates each workload, and the source file it lives in
 DOMINANT = {
-    "gemv": ("decode_mma_kernel", "q4_0_decode_mma.cu"),
-    "layer": ("decode_mma_kernel", "q4_0_decode_mma.cu"),
-    "cfg_decode": ("decode_mma_kernel", "q4_0_decode_mma.cu"),
+    "gemv": ("decode_m8_kernel", "q4_0_decode_m8.cu"),
+    "layer": ("decode_m8_kernel", "q4_0_decode_m8.cu"),
+    "cfg_decode": ("decode_m8_kernel", "q4_0_decode_m8.cu"),
     "concurrent": ("decode_mma_kernel", "q4_0_decode_mma.cu"),
-    "flow_head": ("decode_mma_kernel", "q4_0_decode_mma.cu"),
-    "layer_fused": ("decode_mma_kernel", "q4_0_decode_mma.cu"),
+    "flow_head": ("decode_m8_kernel", "q4_0_decode_m8.cu"),
+    "layer_fused": ("decode_m8_kernel", "q4_0_decode_m8.cu"),
     "adapter": ("prefill_kernel", "q4_0_prefill.cu"),
     "qkv_prefill": ("prefill_kernel", "q4_0_prefill.cu"),
 }

@@ -27,6 +27,7 @@ Q4_ERR_TOO_LARGE = 5
 Q4_DEVERR_WAIT_TIMEOUT = 1
 Q4_DEVERR_BAD_INDEX = 2
 Q4_DEVERR_FP16_RANGE = 4
+Q4_DEVERR_DEBUG_CHECK = 8
 
 Q4_0_MAX_GROUP = 256
 Q4_0_STATIC_WS_BYTES = 64 << 20

@@ -1,12 +1,15 @@
 """Build libq4_0_b200.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python bit_weight_only_matmul_b200/build.py [--force] [--verbose] [--ptxas-info]
+    python bit_weight_only_matmul_b200/build.py [--force] [--verbose] [--ptxas-info] [--debug]
 
 (run it as a script: importing the package needs the library it builds).
 
 Each .cu under csrc/ is compiled to an object in _build/ (only when it or a
 header changed) and the objects are linked into
-bit_weight_only_matmul_b200/libq4_0_b200.so.
+bit_weight_only_matmul_b200/libq4_0_b200.so.  --debug builds the same sources
+with Q4_DEBUG defined (index checks in the decode and tensor-core kernels that
+report Q4_DEVERR_DEBUG_CHECK instead of touching memory outside a buffer)
+into _build_debug/ and libq4_0_b200_debug.so.
 """
 from __future__ import annotations
 
@@ -21,6 +24,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libq4_0_b200.so")
+BUILD_DEBUG = os.path.join(PKG, "_build_debug")
+LIB_DEBUG = os.path.join(PKG, "libq4_0_b200_debug.so")
 INCLUDE = os.path.join(ROOT, "include")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -38,33 +43,34 @@ def _headers():
             + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False, debug: bool = False) -> str:
+    build_dir, lib = (BUILD_DEBUG, LIB_DEBUG) if debug else (BUILD, LIB)
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     newest_header = max((os.path.getmtime(h) for h in _headers()), default=0.0)
-    objs, relink = [], force or not os.path.exists(LIB)
+    objs, relink = [], force or not os.path.exists(lib)
     for src in srcs:
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         stale = (force or ptxas_info or not os.path.exists(obj)
                  or os.path.getmtime(obj) < max(os.path.getmtime(src), newest_header))
         if not stale:
             continue
-        cmd = [_nvcc(), *ARCH, *FLAGS, "-c", src, "-o", obj]
+        cmd = [_nvcc(), *ARCH, *FLAGS, *(["-DQ4_DEBUG"] if debug else []), "-c", src, "-o", obj]
         if ptxas_info:
             cmd += ["-Xptxas", "-v"]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)
         relink = True
-    if relink or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if relink or any(os.path.getmtime(o) > os.path.getmtime(lib) for o in objs):
+        tmp = lib + f".tmp{os.getpid()}"
         cmd = [_nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", *objs, "-o", tmp]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 def main(argv=None) -> int:
@@ -72,8 +78,9 @@ def main(argv=None) -> int:
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-info", action="store_true", help="recompile everything with -Xptxas -v")
+    ap.add_argument("--debug", action="store_true", help="build libq4_0_b200_debug.so with Q4_DEBUG index checks")
     a = ap.parse_args(argv)
-    print(build(a.force, a.verbose, a.ptxas_info))
+    print(build(a.force, a.verbose, a.ptxas_info, a.debug))
     return 0
 
 

@@ -391,6 +391,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_m8_kernel(const __grid_con
                 const int cnt = min(kSub, it.s1 - s);
                 if (lane == 0) ok = wait_or_abort(&S.raw_empty[rp.slot], rp.phase ^ 1u, &S.abort_flag, P.err);
                 if (!__shfl_sync(0xffffffffu, ok, 0)) { ok = false; break; }
+                if (Q4_DEBUG_BAD(rp.slot >= 0 && rp.slot < RS && cnt >= 1 && cnt <= kSub && pr.M >= 1 && pr.M <= 8,
+                                 P.err, &S.abort_flag)) {
+                    ok = false;
+                    break;
+                }
                 const uint32_t dst = raw0 + rp.slot * kSlotBytes;
                 if (lane == 0) {
                     // full boxes are counted, zero-filled rows past N included
@@ -442,6 +447,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_m8_kernel(const __grid_con
             for (int j = (G - static_cast<int>(g)) & 1; j < n; j += 2, ++k, rp.advance(2)) {
                 const int cnt = min(kSub, it.s1 - (it.s0 + kSub * j));
                 const int xb = G + 2 * (k & 1);
+                // the slot, buffer and byte ranges this slot touches stay inside their arrays
+                if (Q4_DEBUG_BAD(rp.slot >= 0 && rp.slot < RS && xb >= 0 && xb < kXBufs && cnt >= 1 &&
+                                     cnt <= kSub && M >= 1 && M <= 8 &&
+                                     wbase + rp.slot * kSlotBytes + (kSub - 1) * kSubBytes + 8 * kStageRowBytes + 36 <=
+                                         raw0 + RS * kSlotBytes &&
+                                     frag0 + (xb * kSub + kSub - 1) * 4096 + 7 * 512 + lane * 16 + 16 <=
+                                         frag0 + kXBufs * kSub * 4096,
+                                 P.err, &S.abort_flag)) {
+                    ok = false;
+                    break;
+                }
                 if (!(ok = wait_or_abort(&S.raw_full[rp.slot], rp.phase, &S.abort_flag, P.err))) break;
                 // this warp's share of the slot's X rows -> fp16 B fragments:
                 // (stage, row) pairs tile and tile + 8 of the cnt * M pairs.
@@ -469,6 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_m8_kernel(const __grid_con
                 uint32_t r[kSub][9], r8[kSub][9];
                 #pragma unroll
                 for (int i = 0; i < kSub; ++i) stage_words(w + i * kSubBytes, r[i], r8[i]);
+                fence_proxy_async_smem();   // the producer's next copies may land in this slot
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.raw_empty[rp.slot]);
                 if (!(ok = wait_or_abort(&S.frag_full[xb], (k >> 1) & 1, &S.abort_flag, P.err))) break;

@@ -469,6 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
                             }
                 }
             }
+            fence_proxy_async_smem();   // the producer's next copies may land in this slot
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&S.xf_full[xb]);
@@ -501,6 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
                     load_blocks(rowg, t, rg[i]);
                     load_blocks(rowg + 8 * kStageRowBytes, t, rg8[i]);
                 }
+                fence_proxy_async_smem();   // the producer's next copies may land in this slot
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.raw_empty[slot]);
                 if (!wait_or_abort(&S.xf_full[xb], (g / kXBufs) & 1, &S.abort_flag, P.err)) break;

@@ -325,6 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tmem_kernel(const __grid_c
                     w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
                 }
             }
+            fence_proxy_async_smem();   // the producer's next copies may land in this slot
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.raw_empty[slot]);
             uint32_t cols[64];

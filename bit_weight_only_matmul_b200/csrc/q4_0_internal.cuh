@@ -155,6 +155,15 @@ __device__ __forceinline__ void fence_mbar_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
+// Orders this thread's generic-proxy shared-memory accesses before later
+// async-proxy ones (TMA and bulk copies).  A consumer that read a slot with
+// ordinary loads runs it before releasing the slot to the copy engine: the
+// mbarrier release alone does not keep the next copy from landing before
+// those loads have read the slot.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile(
         "{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}" ::"r"(smem_addr(bar))
@@ -207,6 +216,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsign
     }
     return true;
 }
+
+// Index checks of a debug build (compiled with Q4_DEBUG defined): a failed
+// check ORs Q4_DEVERR_DEBUG_CHECK into the error word, sets the CTA's abort
+// flag so that the other roles stop at their next wait, and yields true, so
+// that the caller skips the access and leaves its loop.  Nothing traps.  In
+// the product build the check is the constant false and costs nothing.
+__device__ __forceinline__ bool debug_bad(bool bad, unsigned *err, int *abort_flag) {
+    if (bad) {
+        atomicOr(err, (unsigned)Q4_DEVERR_DEBUG_CHECK);
+        *reinterpret_cast<volatile int *>(abort_flag) = 1;
+    }
+    return bad;
+}
+#ifdef Q4_DEBUG
+#define Q4_DEBUG_BAD(ok_cond, err, abort_flag) (::q4dev::debug_bad(!(ok_cond), (err), (abort_flag)))
+#else
+#define Q4_DEBUG_BAD(ok_cond, err, abort_flag) false
+#endif
 
 // 1-D bulk copy global -> shared, completion counted on an mbarrier.
 // dst, src 16-byte aligned, bytes a multiple of 16.

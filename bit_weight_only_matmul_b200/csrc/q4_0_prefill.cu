@@ -182,12 +182,20 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
                 for (int ks = 0; ks < ksteps && ok; ++ks) {
                     if ((ks & 3) == 0) {
                         const int s = rc % kRawStages;
+                        if (Q4_DEBUG_BAD(s < kRawStages && n0 < P.tiles_n * kTileN, P.err, &S.abort_flag)) {
+                            ok = false;
+                            break;
+                        }
                         if (!(ok = wait_or_abort(&S.raw_empty[s], ((rc / kRawStages) & 1) ^ 1, S, P.err))) break;
                         mbar_arrive_expect_tx(&S.raw_full[s], kRawStageBytes);
                         tma_load_2d(S.raw[s], &P.tmap_w, (ks >> 2) * kRawRowBytes, n0, &S.raw_full[s]);
                         ++rc;
                     }
                     const int s = xc % kXStages;
+                    if (Q4_DEBUG_BAD(s < kXStages && m0 < P.tiles_m * kTileM, P.err, &S.abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     if (!(ok = wait_or_abort(&S.x_empty[s], ((xc / kXStages) & 1) ^ 1, S, P.err))) break;
                     mbar_arrive_expect_tx(&S.x_full[s], kXStageBytes);
                     tma_load_2d(S.x[s], &P.tmap_x, ks * kStageK, m0, &S.x_full[s]);
@@ -214,6 +222,13 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
                 tc_fence_after();
                 for (int ks = 0; ks < ksteps; ++ks) {
                     const int sx = xc % kXStages, sa = ac % kAStages;
+                    // A buffers and the accumulator stay inside the 512 tensor-memory columns
+                    if (Q4_DEBUG_BAD(sx < kXStages && sa < kAStages && kACol + 32 * sa + 32 <= kTmemCols &&
+                                         kDCol + kTileM <= kACol,
+                                     P.err, &S.abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     if (!(ok = wait_or_abort(XPRE ? &S.x_full[sx] : &S.x_conv[sx], (xc / kXStages) & 1, S, P.err)))
                         break;
                     if (!(ok = wait_or_abort(&S.a_full[sa], (ac / kAStages) & 1, S, P.err))) break;
@@ -242,6 +257,10 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
         for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
             for (int ks = 0; ks < ksteps && ok; ks += 4) {
                 const int s = rc % kRawStages;
+                if (Q4_DEBUG_BAD(s < kRawStages && row < kTileN, P.err, &S.abort_flag)) {
+                    ok = false;
+                    break;
+                }
                 if (!(ok = wait_or_abort(&S.raw_full[s], (rc / kRawStages) & 1, S, P.err))) break;
                 uint32_t raw[36];
                 const uint4 *src = reinterpret_cast<const uint4 *>(S.raw[s] + row * kRawRowBytes);
@@ -250,12 +269,17 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
                     const uint4 v = src[i];
                     raw[4 * i] = v.x; raw[4 * i + 1] = v.y; raw[4 * i + 2] = v.z; raw[4 * i + 3] = v.w;
                 }
+                fence_proxy_async_smem();   // the next weight tile may land here
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.raw_empty[s]);
                 ++rc;
                 #pragma unroll
                 for (int sub = 0; sub < 4; ++sub) {      // 64 k = blocks 2*sub, 2*sub+1
                     const int sa = ac % kAStages;
+                    if (Q4_DEBUG_BAD(sa < kAStages && kACol + 32 * sa + 32 <= kTmemCols, P.err, &S.abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     if (!(ok = wait_or_abort(&S.a_empty[sa], ((ac / kAStages) & 1) ^ 1, S, P.err))) break;
                     tc_fence_after();
                     uint32_t cols[32];
@@ -296,6 +320,10 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
             const bool check = t % P.tiles_n == 0;
             for (int ks = 0; ks < ksteps; ++ks) {
                 const int s = xc % kXStages;
+                if (Q4_DEBUG_BAD(s < kXStages && 32 * cw + 32 <= kTileM, P.err, &S.abort_flag)) {
+                    ok = false;
+                    break;
+                }
                 if (!(ok = wait_or_abort(&S.x_full[s], (xc / kXStages) & 1, S, P.err))) break;
                 #pragma unroll
                 for (int it = 0; it < 8; ++it) {
@@ -322,6 +350,7 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
             tc_fence_after();
             const int n0 = (t % P.tiles_n) * kTileN, m0 = (t / P.tiles_n) * kTileM;
             const int n = n0 + 32 * quad + lane;
+            if (Q4_DEBUG_BAD(quad < 4 && kDCol + kTileM <= kACol, P.err, &S.abort_flag)) break;
             // a non-finite sum shows in the running value sum_j v[j] * 0
             float nonfinite = 0.f;
             #pragma unroll 1
@@ -359,6 +388,7 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
 // ---------------------------------------------------------------- host side
 
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 // bf16 X -> fp16 X' in the permuted k order of the A operand (positions 1 and
 // 2 of every 4 swapped), 8 elements per thread.  Exact for |x| in the fp16

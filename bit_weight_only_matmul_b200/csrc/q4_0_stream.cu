@@ -78,6 +78,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_kernel(const __grid_consta
                 const uint4 v = p[i];
                 x ^= v.x ^ v.y ^ v.z ^ v.w;
             }
+            fence_proxy_async_smem();   // the next box may land in this slot
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.empty[s]);
         }

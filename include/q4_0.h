@@ -71,10 +71,13 @@ enum {
 enum {
     Q4_DEVERR_WAIT_TIMEOUT = 1u,   /* a bounded on-chip wait gave up; the output is incomplete */
     Q4_DEVERR_BAD_INDEX = 2u,      /* q4_0_gather met an id outside [0, V) (its row was zeroed) */
-    Q4_DEVERR_FP16_RANGE = 4u      /* a fast GEMM path met an operand too large for its fp16
+    Q4_DEVERR_FP16_RANGE = 4u,     /* a fast GEMM path met an operand too large for its fp16
                                       arithmetic: a finite X with |x| > 65504, or a scale with
                                       8188 < |d| < inf; its output may hold +-inf (q4_0_force_path(4)
                                       computes such inputs exactly) */
+    Q4_DEVERR_DEBUG_CHECK = 8u     /* only in a library built with Q4_DEBUG defined: an index check
+                                      found a shared- or tensor-memory index outside its buffer; the
+                                      access was skipped and the kernel stopped early */
 };
 
 /* Largest N, K and M accepted (each dimension below 2^31). */
