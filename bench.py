@@ -321,13 +321,14 @@ def time_workload(q4, G, tensor: bool, steps: int, warmup: int, soak: float, wor
                 i += 1
             torch.cuda.synchronize()
         _barrier(world)
-        # tensor-core steps (X conversion + GEMM) replay CUDA graphs of a
-        # whole cycle of operand copies; a decode step is one launch that the
-        # host enqueues well ahead of the device, overlapping its
-        # predecessor's tail through programmatic dependent launch
+        # the steps replay CUDA graphs of a whole cycle of operand copies (the
+        # library's own launches captured: the X conversion and GEMM of a
+        # tensor-core step, the one grouped launch of a decode step, whose
+        # programmatic dependent launch edges the graph keeps), so that the
+        # host's enqueue cost stays off the device's critical path
         cycle = len(G.sets)
         graph = None
-        if tensor and not no_graphs:
+        if not no_graphs:
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph):
                 for k in range(cycle):

@@ -275,15 +275,16 @@ int q4_0_quantize(const float *X, void *W, int64_t N, int64_t K, q4_0_stream_t s
 int q4_0_gemm_grouped_ex(const q4_0_problem_ex *problems, int count, q4_0_stream_t stream) {
     if (count < 0 || count > Q4_0_MAX_GROUP || (count > 0 && !problems)) return Q4_ERR_INVALID_ARG;
     if (count == 0) return Q4_OK;
-    static thread_local std::vector<q4::Problem> dec, dm8;
+    static thread_local std::vector<q4::Problem> dec, dm8, big;
     dec.clear();
     dm8.clear();
+    big.clear();
     for (int i = 0; i < count; ++i) {
         const q4_0_problem_ex &a = problems[i];
         const q4_0_problem base{a.W, a.X, a.Y, a.M, a.N, a.K};
         int st = check_problem(base);
         if (st != Q4_OK) return st;
-        if (a.M < 1 || a.M > 32 || a.N < 1 || a.K < 256 || a.K % 256 != 0) return Q4_ERR_INVALID_ARG;
+        if (a.M < 1 || a.N < 1 || a.K < 256 || a.K % 256 != 0) return Q4_ERR_INVALID_ARG;
         if (a.epilogue == Q4_0_EPI_RESIDUAL) {
             if (!a.R) return Q4_ERR_INVALID_ARG;
             if (!aligned16(a.R)) return Q4_ERR_MISALIGNED;
@@ -295,6 +296,11 @@ int q4_0_gemm_grouped_ex(const q4_0_problem_ex *problems, int count, q4_0_stream
         q4::Problem p{static_cast<const uint8_t *>(a.W), a.X, a.Y, a.M, a.N, a.K};
         p.R = a.epilogue == Q4_0_EPI_RESIDUAL ? a.R : nullptr;
         p.epi = a.epilogue;
+        if (p.M > 32) {   // the tensor-core kernel, its epilogue warps applying the epilogue
+            if (!q4::prefill_supports(p)) return Q4_ERR_INVALID_ARG;
+            big.push_back(p);
+            continue;
+        }
         if (!q4::decode_mma_supports(p)) return Q4_ERR_INVALID_ARG;
         const int force = g_force_path.load(std::memory_order_relaxed);
         if (p.M <= 8 && force != kDecode && q4::decode_m8_supports(p)) dm8.push_back(p);
@@ -303,7 +309,9 @@ int q4_0_gemm_grouped_ex(const q4_0_problem_ex *problems, int count, q4_0_stream
     const q4::DeviceInfo *dev = nullptr;
     int st = current_device(&dev);
     if (st != Q4_OK) return st;
-    const cudaError_t e = launch_decode_split(dm8, dec, *dev, reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_decode_split(dm8, dec, *dev, reinterpret_cast<cudaStream_t>(stream));
+    for (size_t i = 0; i < big.size() && e == cudaSuccess; ++i)
+        e = q4::launch_prefill(big[i], *dev, reinterpret_cast<cudaStream_t>(stream), nullptr, 0);
     return e == cudaSuccess ? Q4_OK : cuda_fail(e);
 }
 

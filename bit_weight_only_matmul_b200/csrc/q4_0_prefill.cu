@@ -72,9 +72,11 @@ struct alignas(64) PrefillParams {
     CUtensorMap tmap_w;    // uint8 [N, K/32*18], box 144 x 128
     float *Y;
     const uint8_t *W;      // the Q4_0 weights (read directly only by the rare scale check)
+    const float *R;        // residual [M, N] (Q4_0_EPI_RESIDUAL; may be Y itself)
     unsigned *err;
     int M, N, K;
     int tiles_n, tiles_m;
+    int epi;               // Q4_0_EPI_* (one per launch)
 };
 
 struct Smem {
@@ -84,6 +86,10 @@ struct Smem {
     uint64_t raw_full[kRawStages], raw_empty[kRawStages];
     uint64_t a_full[kAStages], a_empty[kAStages];
     uint64_t d_full, d_empty, mma_done;
+    // SwiGLU epilogue: the up rows' sums of one 32-column chunk, handed from
+    // the warps of tensor-memory lanes 64-127 to those of lanes 0-63
+    float up[32][64];
+    uint64_t up_full, up_empty;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -159,6 +165,8 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
         mbar_init(&S.d_full, 1);
         mbar_init(&S.d_empty, kNumEpi);
         mbar_init(&S.mma_done, 1);
+        mbar_init(&S.up_full, kNumEpi / 2);
+        mbar_init(&S.up_empty, kNumEpi / 2);
         S.abort_flag = 0;
         fence_mbar_init();
     }
@@ -343,9 +351,13 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
         }
         if (xbad) atomicOr(P.err, (unsigned)Q4_DEVERR_FP16_RANGE);
     } else {   // epilogue warps
+        // lane l of warp quad holds weight row n0 + 32*quad + l of the tile,
+        // for the 256 activation rows in 8 chunks of 32 tensor-memory columns
         const int quad = warp & 3;
-        uint32_t dc = 0;
-        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++dc) {
+        const bool swiglu = P.epi == Q4_0_EPI_SWIGLU, residual = P.epi == Q4_0_EPI_RESIDUAL;
+        uint32_t dc = 0, uc = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++dc) {
             if (!wait_or_abort(&S.d_full, dc & 1, S, P.err)) break;
             tc_fence_after();
             const int n0 = (t % P.tiles_n) * kTileN, m0 = (t / P.tiles_n) * kTileM;
@@ -361,19 +373,55 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
                 if (n < P.N) {
                     #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        if (mb + j < P.M) {
-                            nonfinite = fmaf(v[j], 0.f, nonfinite);
-                            // streaming store: Y is not read again here, X and W tiles are
+                        if (mb + j < P.M) nonfinite = fmaf(v[j], 0.f, nonfinite);
+                }
+                if (swiglu) {
+                    // rows 0-63 of the tile are the gate rows of features
+                    // n0/2 .. n0/2+63 and rows 64-127 their up rows (N % 128 == 0)
+                    if (quad >= 2) {
+                        if (!(ok = wait_or_abort(&S.up_empty, (uc & 1) ^ 1, S, P.err))) break;
+                        #pragma unroll
+                        for (int j = 0; j < 32; ++j) S.up[j][32 * (quad - 2) + lane] = v[j];
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&S.up_full);
+                    } else {
+                        if (!(ok = wait_or_abort(&S.up_full, uc & 1, S, P.err))) break;
+                        const int F = P.N >> 1, f = (n0 >> 1) + 32 * quad + lane;
+                        #pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (mb + j < P.M) {
+                                const float g = v[j], u = S.up[j][32 * quad + lane];
+                                __stcs(P.Y + static_cast<int64_t>(mb + j) * F + f, g / (1.0f + expf(-g)) * u);
+                            }
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&S.up_empty);
+                    }
+                    ++uc;
+                } else if (n < P.N && residual) {
+                    // all 32 residual loads before any store: R may be Y itself,
+                    // and loads interleaved with stores to a possible alias
+                    // would each wait for the one before
+                    float r[32];
+                    #pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        r[j] = mb + j < P.M ? __ldcs(P.R + static_cast<int64_t>(mb + j) * P.N + n) : 0.f;
+                    #pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (mb + j < P.M) __stcs(P.Y + static_cast<int64_t>(mb + j) * P.N + n, v[j] + r[j]);
+                } else if (n < P.N) {
+                    #pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (mb + j < P.M)   // streaming store: Y is not read again here, X and W tiles are
                             __stcs(P.Y + static_cast<int64_t>(mb + j) * P.N + n, v[j]);
-                        }
                 }
             }
+            if (!ok) break;
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.d_empty);
             // a non-finite sum from finite inputs means an fp16 weight
             // overflowed: look at this row's scales (slow path, rare)
-            if (nonfinite != 0.f) scan_scales_fp16_range(P.W, n, n + 1, P.N, P.K, P.err);
+            if (nonfinite != 0.f && n < P.N) scan_scales_fp16_range(P.W, n, n + 1, P.N, P.K, P.err);
         }
     }
 
@@ -446,6 +494,8 @@ cudaError_t launch_prefill(const Problem &p, const DeviceInfo &dev, cudaStream_t
         return cudaErrorInvalidValue;
     local.Y = p.Y;
     local.W = p.W;
+    local.R = p.R;
+    local.epi = p.epi;
     local.err = dev.err;
     local.M = static_cast<int>(p.M);
     local.N = static_cast<int>(p.N);

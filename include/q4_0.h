@@ -195,7 +195,7 @@ Q4_0_API int q4_0_gemm_ws(const void *W, const uint16_t *X, float *Y,
 Q4_0_API int q4_0_gemm_static_ws(const void *W, const uint16_t *X, float *Y,
                                  int64_t M, int64_t N, int64_t K, q4_0_stream_t stream);
 
-/* Fused epilogues of the decode path (q4_0_gemm_grouped_ex). */
+/* Fused epilogues (q4_0_gemm_grouped_ex). */
 #define Q4_0_EPI_NONE 0      /* Y = X * dequant(W)^T */
 #define Q4_0_EPI_RESIDUAL 1  /* Y = X * dequant(W)^T + R (R [M,N] fp32; R == Y allowed) */
 #define Q4_0_EPI_SWIGLU 2    /* Y[M, N/2] = silu(gate) * up of a row-interleaved gate/up W */
@@ -219,8 +219,11 @@ typedef struct q4_0_problem_ex {
  * trip through HBM: the residual add after the O and down projections, and
  * the SwiGLU activation silu(g) * u (silu(g) = g / (1 + exp(-g)), fp32)
  * between the fused gate/up projection (voxtral-mini-realtime-rs README, TTS
- * section, optimizations) and the down projection.  The epilogues run on the
- * decode path: every problem needs 1 <= M <= 32, K a positive multiple of 256
+ * section, optimizations) and the down projection.  Problems with M <= 32
+ * run on the decode path (all of them in one launch); each problem with
+ * M > 32 runs on the tensor-core kernel, whose epilogue warps apply its
+ * epilogue as they drain the accumulator (X converted to fp16 tile by tile,
+ * no workspace).  Every problem needs M >= 1, K a positive multiple of 256
  * and 16-byte aligned W, X, Y, R, else Q4_ERR_INVALID_ARG and nothing is
  * launched.  Tolerance: the GEMM bound of each input of the epilogue, carried
  * through it (silu' <= 1.1), plus fp32 rounding of the epilogue. */

@@ -136,7 +136,13 @@ def test_grouped_ex_argument_checks(q4):
         arr = (q4.q4_0_problem_ex * 1)()
         arr[0] = q4.q4_0_problem_ex(A, A, A, M, N, K, R, epi)
         return q4.lib.q4_0_gemm_grouped_ex(arr, 1, None)
-    assert ex(33, 128, 256) == q4.Q4_ERR_INVALID_ARG                      # decode path only: M <= 32
+    assert ex(0, 128, 256) == q4.Q4_ERR_INVALID_ARG                       # M >= 1
+    for M in (4, 300):                                                    # decode and tensor-core paths
+        assert ex(M, 128, 288) == q4.Q4_ERR_INVALID_ARG                   # K % 256
+        assert ex(M, 128, 256, R=None) == q4.Q4_ERR_INVALID_ARG           # residual needs R
+        assert ex(M, 128, 256, R=A + 4) == q4.Q4_ERR_MISALIGNED
+        assert ex(M, 192, 256, epi=q4.Q4_0_EPI_SWIGLU) == q4.Q4_ERR_INVALID_ARG   # 2F with F % 64
+        assert ex(M, 128, 256, epi=7) == q4.Q4_ERR_INVALID_ARG
     assert ex(4, 128, 288) == q4.Q4_ERR_INVALID_ARG                       # K % 256
     assert ex(4, 128, 256, R=None) == q4.Q4_ERR_INVALID_ARG               # residual needs R
     assert ex(4, 128, 256, R=A + 4) == q4.Q4_ERR_MISALIGNED

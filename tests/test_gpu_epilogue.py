@@ -1,5 +1,7 @@
-"""Fused decode epilogues (residual add, SwiGLU of a row-interleaved gate/up
-weight) through q4_0_gemm_grouped_ex, against the float64 oracle."""
+"""Fused epilogues (residual add, SwiGLU of a row-interleaved gate/up weight)
+through q4_0_gemm_grouped_ex, against the float64 oracle: on the decode path
+(M <= 32) and on the tensor-core kernel (M > 32, ragged activation tiles
+included)."""
 import numpy as np
 import pytest
 import torch
@@ -49,7 +51,8 @@ def test_interleave_bit_exact(q4):
     assert np.array_equal(out.cpu().numpy(), want.reshape(-1))
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 3072, 3072), (2, 200, 1024), (32, 300, 512), (7, 129, 768)])
+@pytest.mark.parametrize("M,N,K", [(1, 3072, 3072), (2, 200, 1024), (32, 300, 512), (7, 129, 768),
+                                   (33, 200, 512), (300, 129, 768), (600, 512, 1024)])
 @pytest.mark.parametrize("inplace", [False, True])
 def test_residual_epilogue(q4, M, N, K, inplace):
     rng = np.random.default_rng(M + N + K + inplace)
@@ -82,7 +85,8 @@ def _swiglu_case(q4, rng, M, F, K):
     return Wgu, X, ref, tol
 
 
-@pytest.mark.parametrize("M,F,K", [(1, 64, 256), (2, 512, 1024), (32, 256, 512), (1, 8192, 3072)])
+@pytest.mark.parametrize("M,F,K", [(1, 64, 256), (2, 512, 1024), (32, 256, 512), (1, 8192, 3072),
+                                   (33, 64, 256), (300, 320, 512), (513, 1024, 1024)])
 def test_swiglu_epilogue(q4, M, F, K):
     rng = np.random.default_rng(M * 3 + F + K)
     Wgu, X, ref, tol = _swiglu_case(q4, rng, M, F, K)
@@ -126,4 +130,31 @@ def test_fused_decoder_layer_one_launch(q4):
         _check(Yg.cpu().numpy(), ref_g, tol_g, "gate/up swiglu")
         y, b = o.gemm(o.pack(cd, sd), Xd, M, 3072, 8192)
         _check(Yd.cpu().numpy(), y + Rd, _bound(b) + 2.0**-22 * np.abs(y + Rd), "down + residual")
+    no_device_error(q4)
+
+
+def test_mixed_paths_one_call(q4):
+    """One grouped_ex call holding M <= 32 problems (one decode launch) and
+    M > 32 problems (one tensor-core launch each), every epilogue kind."""
+    rng = np.random.default_rng(9)
+    o = oracle.get()
+    cases = []
+    for M, N, K, epi in [(2, 384, 512, q4.Q4_0_EPI_RESIDUAL), (100, 384, 512, q4.Q4_0_EPI_RESIDUAL),
+                         (64, 256, 768, q4.Q4_0_EPI_NONE), (4, 256, 768, q4.Q4_0_EPI_NONE)]:
+        codes, scales = _weights(rng, N, K)
+        X = _x(rng, M, K)
+        R = rng.standard_normal((M, N)).astype(np.float32)
+        Y = torch.full((M, N), float("nan"), device="cuda")
+        cases.append((codes, scales, X, R, Y, M, N, K, epi))
+    Wgu, Xg, ref_g, tol_g = _swiglu_case(q4, rng, 70, 128, 512)
+    Yg = torch.full((70, 128), float("nan"), device="cuda")
+    probs = [(pack_on_gpu(q4, c, s), dev(X), Y, M, N, K, dev(R) if epi == q4.Q4_0_EPI_RESIDUAL else None, epi)
+             for (c, s, X, R, Y, M, N, K, epi) in cases]
+    probs.append((Wgu, dev(Xg), Yg, 70, 256, 512, None, q4.Q4_0_EPI_SWIGLU))
+    q4.q4_0_gemm_grouped_ex(probs)
+    for (c, s, X, R, Y, M, N, K, epi) in cases:
+        y, b = o.gemm(o.pack(c, s), X, M, N, K)
+        ref = y + R if epi == q4.Q4_0_EPI_RESIDUAL else y
+        _check(Y.cpu().numpy(), ref, _bound(b) + 2.0**-22 * np.abs(ref), f"M={M} epilogue {epi}")
+    _check(Yg.cpu().numpy(), ref_g, tol_g, "swiglu M=70")
     no_device_error(q4)
