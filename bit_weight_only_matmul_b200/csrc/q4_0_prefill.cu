@@ -86,10 +86,11 @@ struct Smem {
     uint64_t raw_full[kRawStages], raw_empty[kRawStages];
     uint64_t a_full[kAStages], a_empty[kAStages];
     uint64_t d_full, d_empty, mma_done;
-    // SwiGLU epilogue: the up rows' sums of one 32-column chunk, handed from
-    // the warps of tensor-memory lanes 64-127 to those of lanes 0-63
-    float up[32][64];
-    uint64_t up_full, up_empty;
+    // SwiGLU epilogue, per 32-column chunk (double-buffered): the up rows'
+    // sums of columns 0-15 for the gate rows' warps and the gate rows' sums
+    // of columns 16-31 for the up rows' warps, [column][feature of the tile]
+    float xch[2][32][64];
+    uint64_t xch_full[2], xch_empty[2];
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -165,8 +166,10 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
         mbar_init(&S.d_full, 1);
         mbar_init(&S.d_empty, kNumEpi);
         mbar_init(&S.mma_done, 1);
-        mbar_init(&S.up_full, kNumEpi / 2);
-        mbar_init(&S.up_empty, kNumEpi / 2);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&S.xch_full[b], kNumEpi);
+            mbar_init(&S.xch_empty[b], kNumEpi);
+        }
         S.abort_flag = 0;
         fence_mbar_init();
     }
@@ -355,6 +358,16 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
         // for the 256 activation rows in 8 chunks of 32 tensor-memory columns
         const int quad = warp & 3;
         const bool swiglu = P.epi == Q4_0_EPI_SWIGLU, residual = P.epi == Q4_0_EPI_RESIDUAL;
+        // the residual rows of a tile are asked into L2 while its MMAs run: one
+        // 128-byte line (32 weight rows) per activation row and warp
+        auto prefetch_r = [&](int t) {
+            if (!residual || t >= tiles) return;
+            const int n0 = (t % P.tiles_n) * kTileN + 32 * quad, m0 = (t / P.tiles_n) * kTileM;
+            if (n0 >= P.N) return;
+            for (int m = m0 + lane; m < m0 + kTileM && m < P.M; m += 32)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(P.R + static_cast<int64_t>(m) * P.N + n0));
+        };
+        prefetch_r(blockIdx.x);
         uint32_t dc = 0, uc = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++dc) {
@@ -377,37 +390,61 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
                 }
                 if (swiglu) {
                     // rows 0-63 of the tile are the gate rows of features
-                    // n0/2 .. n0/2+63 and rows 64-127 their up rows (N % 128 == 0)
-                    if (quad >= 2) {
-                        if (!(ok = wait_or_abort(&S.up_empty, (uc & 1) ^ 1, S, P.err))) break;
+                    // n0/2 .. n0/2+63 and rows 64-127 their up rows (N % 128 == 0):
+                    // warps 0/1 (gate) pair with warps 2/3 (up) on the same 32
+                    // features; the gate warp finishes columns 0-15 of the chunk,
+                    // the up warp columns 16-31
+                    const int xb = uc & 1;
+                    const uint32_t xpar = (uc >> 1) & 1;
+                    const bool up = quad >= 2;
+                    const int fl = 32 * (quad & 1) + lane;
+                    if (!(ok = wait_or_abort(&S.xch_empty[xb], xpar ^ 1, S, P.err))) break;
+                    // (constant indices into v on both sides: v stays in registers)
+                    if (up) {
                         #pragma unroll
-                        for (int j = 0; j < 32; ++j) S.up[j][32 * (quad - 2) + lane] = v[j];
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&S.up_full);
+                        for (int j = 0; j < 16; ++j) S.xch[xb][j][fl] = v[j];
                     } else {
-                        if (!(ok = wait_or_abort(&S.up_full, uc & 1, S, P.err))) break;
-                        const int F = P.N >> 1, f = (n0 >> 1) + 32 * quad + lane;
                         #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (mb + j < P.M) {
-                                const float g = v[j], u = S.up[j][32 * quad + lane];
-                                __stcs(P.Y + static_cast<int64_t>(mb + j) * F + f, g / (1.0f + expf(-g)) * u);
-                            }
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&S.up_empty);
+                        for (int j = 16; j < 32; ++j) S.xch[xb][j][fl] = v[j];
                     }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.xch_full[xb]);
+                    if (!(ok = wait_or_abort(&S.xch_full[xb], xpar, S, P.err))) break;
+                    float* const yf = P.Y + (static_cast<int64_t>(mb) * (P.N >> 1) + (n0 >> 1) + fl);
+                    const int64_t F = P.N >> 1;
+                    if (up) {
+                        #pragma unroll
+                        for (int j = 16; j < 32; ++j)
+                            if (mb + j < P.M) {
+                                const float g = S.xch[xb][j][fl];
+                                __stcs(yf + j * F, __fdividef(g, 1.0f + __expf(-g)) * v[j]);
+                            }
+                    } else {
+                        #pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (mb + j < P.M) {
+                                const float g = v[j];
+                                __stcs(yf + j * F, __fdividef(g, 1.0f + __expf(-g)) * S.xch[xb][j][fl]);
+                            }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.xch_empty[xb]);
                     ++uc;
                 } else if (n < P.N && residual) {
-                    // all 32 residual loads before any store: R may be Y itself,
-                    // and loads interleaved with stores to a possible alias
-                    // would each wait for the one before
-                    float r[32];
+                    // the residual loads of 16 columns before their stores: R may
+                    // be Y itself, and loads interleaved with stores to a possible
+                    // alias would each wait for the one before
                     #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        r[j] = mb + j < P.M ? __ldcs(P.R + static_cast<int64_t>(mb + j) * P.N + n) : 0.f;
-                    #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (mb + j < P.M) __stcs(P.Y + static_cast<int64_t>(mb + j) * P.N + n, v[j] + r[j]);
+                    for (int h = 0; h < 32; h += 16) {
+                        float r[16];
+                        #pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            r[j] = mb + h + j < P.M ? __ldcs(P.R + static_cast<int64_t>(mb + h + j) * P.N + n) : 0.f;
+                        #pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (mb + h + j < P.M)
+                                __stcs(P.Y + static_cast<int64_t>(mb + h + j) * P.N + n, v[h + j] + r[j]);
+                    }
                 } else if (n < P.N) {
                     #pragma unroll
                     for (int j = 0; j < 32; ++j)
@@ -419,6 +456,7 @@ __global__ void __launch_bounds__(threads<XPRE>(), 1) prefill_kernel(const __gri
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.d_empty);
+            prefetch_r(t + gridDim.x);
             // a non-finite sum from finite inputs means an fp16 weight
             // overflowed: look at this row's scales (slow path, rare)
             if (nonfinite != 0.f && n < P.N) scan_scales_fp16_range(P.W, n, n + 1, P.N, P.K, P.err);

@@ -137,11 +137,13 @@ def test_stream_read_checksum(q4, N, K):
     assert int(cs.cpu().numpy().view(np.uint32)[0]) == want
 
 
-@pytest.mark.parametrize("M,N,K", [(512, 18944, 256), (176, 300, 512), (177, 128, 1024), (4096, 256, 768)])
+@pytest.mark.parametrize("M,N,K", [(512, 18944, 256), (176, 300, 512), (177, 128, 1024), (4096, 256, 768),
+                                   (300, 19000, 768), (4096, 2368, 5120), (1000, 5000, 256)])
 def test_tensor_core_tiles_sampled(q4, M, N, K):
     """The tensor-core kernel on one and several activation tiles (ragged last
-    tiles included, a grid of two tiles per SM): sampled outputs against the
-    oracle, through both the in-kernel and the workspace conversion of X,
+    tiles included, a grid of two tiles per SM, tile counts that leave a
+    part-filled last wave: 298, 304 and 160 tiles): sampled outputs against
+    the oracle, through both the in-kernel and the workspace conversion of X,
     which must agree bit for bit."""
     rng = np.random.default_rng(M + N + K)
     codes, scales = _weights(rng, N, K)
