@@ -209,6 +209,18 @@ class GpuWorkload:
         self.large = [i for i, l in enumerate(wl.linears) if l.M > 32]
         ws = max([q4.q4_0_gemm_workspace_size(l.M, l.N, l.K) for l in wl.linears] + [0])
         self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device="cuda")
+        # pipelined tensor-core steps: each M > 32 GEMM's X is converted on a
+        # side stream (q4_0_prepare_x) into one of two buffers while the
+        # previous step's GEMM (q4_0_gemm_prepared) runs on the launching stream
+        self.pipelined = bool(self.large) and not wl.fused
+        if self.pipelined:
+            self.side = torch.cuda.Stream()
+            self.xh = [[torch.empty(q4.q4_0_prepared_x_bytes(wl.linears[i].M, wl.linears[i].K), dtype=torch.uint8,
+                                    device="cuda") for i in self.large] for _ in range(2)]
+            self.prep_done = [torch.cuda.Event(), torch.cuda.Event()]
+            self.gemm_done = [torch.cuda.Event(), torch.cuda.Event()]
+            self.fork = torch.cuda.Event()
+            self.begun = [False, False]
         self.small_arrs = [q4.make_problems([probs[i] for i in self.small]) for probs, _ in self.sets]
         self.fused_arrs = []
         if wl.fused:
@@ -264,6 +276,40 @@ class GpuWorkload:
         for i in self.large:
             W, X, Y, M, N, K = probs[i]
             q4.q4_0_gemm_ws(W, X, Y, M, N, K, self.ws)
+
+    def begin_pipeline(self):
+        """Start a sequence of pipelined steps (a graph capture or an eager
+        run): the side stream joins the launching stream here."""
+        import torch
+        main = torch.cuda.current_stream()
+        self.fork.record(main)
+        self.side.wait_event(self.fork)
+        self.begun = [False, False]
+
+    def launch_pipelined(self, q4, step: int):
+        """One step with its X conversion on the side stream: buffer step % 2,
+        free once the GEMM two steps back (which read it) is done; the GEMM
+        waits for its conversion.  The conversion of step k+1 thus overlaps
+        the GEMM of step k."""
+        import torch
+        k, b = step % len(self.sets), step % 2
+        probs, _ = self.sets[k]
+        main = torch.cuda.current_stream()
+        if self.begun[b]:
+            self.side.wait_event(self.gemm_done[b])
+        with torch.cuda.stream(self.side):
+            for j, i in enumerate(self.large):
+                W, X, Y, M, N, K = probs[i]
+                q4.q4_0_prepare_x(X, M, K, self.xh[b][j])
+            self.prep_done[b].record(self.side)
+        if self.small:
+            q4.q4_0_gemm_grouped(self.small_arrs[k], len(self.small))
+        main.wait_event(self.prep_done[b])
+        for j, i in enumerate(self.large):
+            W, X, Y, M, N, K = probs[i]
+            q4.q4_0_gemm_prepared(W, self.xh[b][j], Y, M, N, K)
+        self.gemm_done[b].record(main)
+        self.begun[b] = True
 
 
 def rotating_copies(wl: workloads.Workload) -> int:
@@ -326,13 +372,19 @@ def time_workload(q4, G, tensor: bool, steps: int, warmup: int, soak: float, wor
         # tensor-core step, the one grouped launch of a decode step, whose
         # programmatic dependent launch edges the graph keeps), so that the
         # host's enqueue cost stays off the device's critical path
-        cycle = len(G.sets)
+        # tensor-core steps run pipelined (each step's X conversion on a side
+        # stream beside the previous step's GEMM), captured at least 12 steps
+        # to a graph so that few conversions fall on a replay boundary
+        cycle = len(G.sets) * (max(1, -(-12 // len(G.sets))) if G.pipelined else 1)
+        step_fn = G.launch_pipelined if G.pipelined else G.launch
         graph = None
         if not no_graphs:
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph):
+                if G.pipelined:
+                    G.begin_pipeline()
                 for k in range(cycle):
-                    G.launch(q4, k)
+                    step_fn(q4, k)
             torch.cuda.synchronize()
 
         def run_steps(n):
@@ -340,8 +392,10 @@ def time_workload(q4, G, tensor: bool, steps: int, warmup: int, soak: float, wor
             while graph is not None and k + cycle <= n:
                 graph.replay()
                 k += cycle
+            if k < n and G.pipelined:
+                G.begin_pipeline()
             for j in range(k, n):
-                G.launch(q4, j)
+                step_fn(q4, j)
 
         run_steps(max(warmup, cycle if graph is not None else 0))
         _barrier(world)
@@ -365,6 +419,9 @@ def time_workload(q4, G, tensor: bool, steps: int, warmup: int, soak: float, wor
         _barrier(world)
     launch = (f"CUDA graph replay of cycles of {cycle} steps (the library's own launches inside)"
               if graph is not None else "eager, programmatic dependent launch")
+    if G.pipelined:
+        launch += ("; each step's X converted to fp16 (q4_0_prepare_x) on a second stream while the previous "
+                   "step's tensor-core GEMM (q4_0_gemm_prepared) runs, two conversion buffers")
     del graph
     return t0.elapsed_time(t1), steps, clocks.summary(), launch
 
@@ -488,7 +545,11 @@ def oracle_error(q4, G, wl, host, samples: int = 48, seed: int = 7):
     if G.fused_arrs:
         return None, "fused epilogues: checked by the GPU tests, not here"
     o, packed = host
-    G.launch(q4, 0)
+    if G.pipelined:   # the path the timed steps take
+        G.begin_pipeline()
+        G.launch_pipelined(q4, 0)
+    else:
+        G.launch(q4, 0)
     torch.cuda.synchronize()
     outs = G.outputs(0)
     rng = np.random.default_rng(seed)

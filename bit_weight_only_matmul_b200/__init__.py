@@ -46,6 +46,9 @@ EXPORTS = (
     "q4_0_gemm_workspace_size",
     "q4_0_gemm_ws",
     "q4_0_gemm_static_ws",
+    "q4_0_prepared_x_bytes",
+    "q4_0_prepare_x",
+    "q4_0_gemm_prepared",
     "q4_0_gemm_grouped",
     "q4_0_gemm_grouped_ex",
     "q4_0_interleave_gate_up",
@@ -93,6 +96,9 @@ def _load() -> ctypes.CDLL:
         "q4_0_gemm_workspace_size": (i64, [i64, i64, i64]),
         "q4_0_gemm_ws": (i32, [vp, vp, vp, i64, i64, i64, vp, i64, vp]),
         "q4_0_gemm_static_ws": (i32, [vp, vp, vp, i64, i64, i64, vp]),
+        "q4_0_prepared_x_bytes": (i64, [i64, i64]),
+        "q4_0_prepare_x": (i32, [vp, i64, i64, vp, i64, vp]),
+        "q4_0_gemm_prepared": (i32, [vp, vp, vp, i64, i64, i64, vp]),
         "q4_0_gemm_grouped": (i32, [ctypes.POINTER(q4_0_problem), i32, vp]),
         "q4_0_gemm_grouped_ex": (i32, [ctypes.POINTER(q4_0_problem_ex), i32, vp]),
         "q4_0_interleave_gate_up": (i32, [vp, vp, vp, i64, i64, vp]),
@@ -184,6 +190,23 @@ def q4_0_gemm_static_ws(W, X, Y, M: int, N: int, K: int, stream=None) -> None:
     allocates nothing (Q4Error Q4_ERR_TOO_LARGE when M*K*2 exceeds
     Q4_0_STATIC_WS_BYTES for M > 32)."""
     _check(_lib.q4_0_gemm_static_ws(_ptr(W), _ptr(X), _ptr(Y), M, N, K, _stream(stream)), "q4_0_gemm_static_ws")
+
+
+def q4_0_prepared_x_bytes(M: int, K: int) -> int:
+    return int(_lib.q4_0_prepared_x_bytes(M, K))
+
+
+def q4_0_prepare_x(X, M: int, K: int, xh, xh_bytes: Optional[int] = None, stream=None) -> None:
+    """X (bf16 [M, K]) into `xh` in the tensor-core kernel's fp16 layout (its
+    byte size taken from the tensor unless given)."""
+    if xh_bytes is None:
+        xh_bytes = xh.numel() * xh.element_size()
+    _check(_lib.q4_0_prepare_x(_ptr(X), M, K, _ptr(xh), xh_bytes, _stream(stream)), "q4_0_prepare_x")
+
+
+def q4_0_gemm_prepared(W, xh, Y, M: int, N: int, K: int, stream=None) -> None:
+    """The tensor-core GEMM on an X prepared by q4_0_prepare_x."""
+    _check(_lib.q4_0_gemm_prepared(_ptr(W), _ptr(xh), _ptr(Y), M, N, K, _stream(stream)), "q4_0_gemm_prepared")
 
 
 def make_problems(problems: Sequence) -> ctypes.Array:

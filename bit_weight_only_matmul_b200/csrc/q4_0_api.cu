@@ -229,6 +229,40 @@ int q4_0_gemm_ws(const void *W, const uint16_t *X, float *Y, int64_t M, int64_t 
     return run_problems(&p, 1, reinterpret_cast<cudaStream_t>(stream), workspace, workspace_bytes);
 }
 
+int64_t q4_0_prepared_x_bytes(int64_t M, int64_t K) {
+    if (M < 0 || M > Q4_0_MAX_DIM || K < 0 || K > Q4_0_MAX_DIM || K % 256 != 0) return -1;
+    return q4::prepared_x_bytes(M, K);
+}
+
+int q4_0_prepare_x(const uint16_t *X, int64_t M, int64_t K, void *xh, int64_t xh_bytes, q4_0_stream_t stream) {
+    const int64_t need = q4_0_prepared_x_bytes(M, K);
+    if (need < 0 || xh_bytes < 0) return Q4_ERR_INVALID_ARG;
+    if (M == 0 || K == 0) return Q4_OK;
+    if (!X || !xh || xh_bytes < need) return Q4_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(xh)) return Q4_ERR_MISALIGNED;
+    const q4::DeviceInfo *dev = nullptr;
+    int st = current_device(&dev);
+    if (st != Q4_OK) return st;
+    const cudaError_t e = q4::launch_prepare_x(X, M, K, xh, *dev, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? Q4_OK : cuda_fail(e);
+}
+
+int q4_0_gemm_prepared(const void *W, const void *xh, float *Y, int64_t M, int64_t N, int64_t K,
+                       q4_0_stream_t stream) {
+    const q4_0_problem base{W, static_cast<const uint16_t *>(xh), Y, M, N, K};
+    int st = check_problem(base);
+    if (st != Q4_OK) return st;
+    if (M == 0 || N == 0) return Q4_OK;
+    if (K < 256 || K % 256 != 0) return Q4_ERR_INVALID_ARG;
+    q4::Problem p{static_cast<const uint8_t *>(W), static_cast<const uint16_t *>(xh), Y, M, N, K};
+    const q4::DeviceInfo *dev = nullptr;
+    st = current_device(&dev);
+    if (st != Q4_OK) return st;
+    if (!q4::prefill_supports(p)) return Q4_ERR_INVALID_ARG;
+    const cudaError_t e = q4::launch_prefill_prepared(p, xh, *dev, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? Q4_OK : cuda_fail(e);
+}
+
 int q4_0_gemm_static_ws(const void *W, const uint16_t *X, float *Y, int64_t M, int64_t N, int64_t K,
                         q4_0_stream_t stream) {
     const int64_t need = q4_0_gemm_workspace_size(M, N, K);

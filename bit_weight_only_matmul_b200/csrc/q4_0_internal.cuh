@@ -115,6 +115,12 @@ int64_t prefill_workspace_bytes(const Problem &p);
 cudaError_t static_workspace(int dev, void **out);
 cudaError_t launch_prefill(const Problem &p, const DeviceInfo &dev, cudaStream_t s, void *workspace,
                            int64_t workspace_bytes);
+// The two phases of the workspace path as separate launches: X (bf16) to the
+// fp16 layout the tensor-core kernel reads, and the kernel on it.
+int64_t prepared_x_bytes(int64_t M, int64_t K);
+cudaError_t launch_prepare_x(const uint16_t *X, int64_t M, int64_t K, void *xh, const DeviceInfo &dev,
+                             cudaStream_t s);
+cudaError_t launch_prefill_prepared(const Problem &p, const void *xh, const DeviceInfo &dev, cudaStream_t s);
 
 }  // namespace q4
 

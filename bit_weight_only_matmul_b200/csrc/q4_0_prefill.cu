@@ -509,24 +509,25 @@ int64_t prefill_workspace_bytes(const Problem &p) {
     return p.M > 32 ? x_conversion_bytes(p) : 0;
 }
 
-cudaError_t launch_prefill(const Problem &p, const DeviceInfo &dev, cudaStream_t s, void *workspace,
-                           int64_t workspace_bytes) {
-    // the pre-pass runs only when the workspace holds everything it writes;
-    // otherwise the kernel converts each X tile in shared memory
-    const bool xpre = workspace != nullptr && workspace_bytes >= x_conversion_bytes(p) &&
-                      (reinterpret_cast<uintptr_t>(workspace) & 15) == 0;
+int64_t prepared_x_bytes(int64_t M, int64_t K) { return ((M * K * 2 + 255) / 256) * 256; }
+
+cudaError_t launch_prepare_x(const uint16_t *X, int64_t M, int64_t K, void *xh, const DeviceInfo &dev,
+                             cudaStream_t s) {
+    const int64_t n8 = M * K / 8;
+    const int64_t blocks = (n8 + 255) / 256;
+    const int grid = static_cast<int>(blocks < dev.sm_count * 8 ? blocks : dev.sm_count * 8);
+    if (grid < 1) return cudaSuccess;
+    x_to_fp16_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const uint4 *>(X), static_cast<uint4 *>(xh), n8, dev.err);
+    return cudaGetLastError();
+}
+
+// The tensor-core kernel on X already in fp16 (xh != nullptr: the pre-pass's
+// layout) or on bf16 X converted tile by tile (xh == nullptr).
+static cudaError_t launch_prefill_kernel(const Problem &p, const void *xh, const DeviceInfo &dev, cudaStream_t s) {
+    const bool xpre = xh != nullptr;
     PrefillParams local;
     std::memset(&local, 0, sizeof(local));
-    if (xpre) {
-        const int64_t n8 = p.M * p.K / 8;
-        const int64_t blocks = (n8 + 255) / 256;
-        const int grid = static_cast<int>(blocks < dev.sm_count * 8 ? blocks : dev.sm_count * 8);
-        x_to_fp16_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const uint4 *>(p.X), static_cast<uint4 *>(workspace),
-                                              n8, dev.err);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
-    if (!get_tensor_map(&local.tmap_x, xpre ? workspace : p.X, p.M, p.K,
+    if (!get_tensor_map(&local.tmap_x, xpre ? xh : p.X, p.M, p.K,
                         xpre ? kMapActivationsF16Sw128 : kMapActivationsSw128) ||
         !get_tensor_map(&local.tmap_w, p.W, p.N, p.K / 32 * 18, kMapWeights128Prefill))
         return cudaErrorInvalidValue;
@@ -560,6 +561,23 @@ cudaError_t launch_prefill(const Problem &p, const DeviceInfo &dev, cudaStream_t
         prefill_kernel<false><<<grid, threads<false>(), kSmemBytes, s>>>(local);
     }
     return cudaGetLastError();
+}
+
+cudaError_t launch_prefill(const Problem &p, const DeviceInfo &dev, cudaStream_t s, void *workspace,
+                           int64_t workspace_bytes) {
+    // the pre-pass runs only when the workspace holds everything it writes;
+    // otherwise the kernel converts each X tile in shared memory
+    const bool xpre = workspace != nullptr && workspace_bytes >= x_conversion_bytes(p) &&
+                      (reinterpret_cast<uintptr_t>(workspace) & 15) == 0;
+    if (xpre) {
+        cudaError_t e = launch_prepare_x(p.X, p.M, p.K, workspace, dev, s);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_prefill_kernel(p, xpre ? workspace : nullptr, dev, s);
+}
+
+cudaError_t launch_prefill_prepared(const Problem &p, const void *xh, const DeviceInfo &dev, cudaStream_t s) {
+    return launch_prefill_kernel(p, xh, dev, s);
 }
 
 }  // namespace q4

@@ -156,6 +156,34 @@ Q4_0_API int q4_0_gemm_ws(const void *W, const uint16_t *X, float *Y,
                           int64_t M, int64_t N, int64_t K, void *workspace,
                           int64_t workspace_bytes, q4_0_stream_t stream);
 
+/* The two phases of q4_0_gemm_ws's tensor-core path as separate calls, so
+ * that a caller can convert the X of the next GEMM while the current one runs
+ * (on another stream: the conversion reads and writes HBM while the GEMM
+ * keeps the tensor cores busy), or convert an X once for several GEMMs that
+ * share it.  No counterpart on the pages: the same trade as q4_0_gemm_ws.
+ *
+ * q4_0_prepared_x_bytes: bytes of the prepared copy of an [M, K] X:
+ * M*K*2 rounded up to 256; -1 for a negative or too large M or K, or K not a
+ * multiple of 256.
+ *
+ * q4_0_prepare_x: writes bf16 X [M, K] (device, 16-byte aligned, row-major)
+ * into `xh` (device, 16-byte aligned, owned by the caller, at least
+ * q4_0_prepared_x_bytes(M, K) bytes, else Q4_ERR_INVALID_ARG) as fp16 in the
+ * order the tensor-core kernel reads (within every 4 consecutive k, positions
+ * 1 and 2 swapped).  A finite |x| > 65504 sets Q4_DEVERR_FP16_RANGE.
+ *
+ * q4_0_gemm_prepared: Y[M,N] = X * dequant(W)^T on the tensor-core kernel
+ * whatever M is, reading X from `xh` as written by q4_0_prepare_x for the
+ * same M and K (device pointers, 16-byte aligned; K a positive multiple of
+ * 256, else Q4_ERR_INVALID_ARG).  For M > 32 the result is that of
+ * q4_0_gemm_ws (and so q4_0_gemm) bit for bit.  The order between the two
+ * calls is the caller's: the same stream, or an event. */
+Q4_0_API int64_t q4_0_prepared_x_bytes(int64_t M, int64_t K);
+Q4_0_API int q4_0_prepare_x(const uint16_t *X, int64_t M, int64_t K, void *xh, int64_t xh_bytes,
+                            q4_0_stream_t stream);
+Q4_0_API int q4_0_gemm_prepared(const void *W, const void *xh, float *Y, int64_t M, int64_t N, int64_t K,
+                                q4_0_stream_t stream);
+
 /* Size of the library's fixed device scratch array used by
  * q4_0_gemm_static_ws: 64 MiB on each device (an fp16 copy of X up to
  * M*K = 32 Mi elements, e.g. M = 4096 rows at K = 8192). */

@@ -199,3 +199,22 @@ def test_header_is_plain_c_and_matches_the_binding(q4, tmp_path):
         assert got[(st, "size")] == ctypes.sizeof(cls), st
         for f in fs:
             assert got[(st, f)] == getattr(cls, f).offset, (st, f)
+
+
+def test_prepared_path_argument_checks(q4):
+    pb = q4.lib.q4_0_prepared_x_bytes
+    assert pb(4096, 5120) == 4096 * 5120 * 2
+    assert pb(3, 256) == 1536 and pb(1, 256) == 512
+    assert pb(5, 512) == 5120 and pb(3, 768) == 4608
+    assert pb(4, 288) == -1 and pb(-1, 256) == -1
+    px = q4.lib.q4_0_prepare_x
+    assert px(A, 4, 256, A, 2047, None) == q4.Q4_ERR_INVALID_ARG          # buffer too small
+    assert px(A, 4, 288, A, 4096, None) == q4.Q4_ERR_INVALID_ARG          # K % 256
+    assert px(A + 8, 4, 256, A, 2048, None) == q4.Q4_ERR_MISALIGNED
+    assert px(A, 4, 256, A + 8, 2048, None) == q4.Q4_ERR_MISALIGNED
+    assert px(None, 0, 256, None, 0, None) == q4.Q4_OK                    # nothing to convert
+    gp = q4.lib.q4_0_gemm_prepared
+    assert gp(A, A, A, 64, 128, 288, None) == q4.Q4_ERR_INVALID_ARG       # K % 256
+    assert gp(A, A, A, 64, 128, 224, None) == q4.Q4_ERR_INVALID_ARG
+    assert gp(A, A + 8, A, 64, 128, 256, None) == q4.Q4_ERR_MISALIGNED
+    assert gp(None, None, None, 0, 128, 256, None) == q4.Q4_OK

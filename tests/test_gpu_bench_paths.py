@@ -209,3 +209,38 @@ def test_repeated_runs_bit_identical(q4):
             torch.cuda.synchronize()
             for i, (p, r) in enumerate(zip(probs, refs)):
                 assert torch.equal(p[2], r), f"decode M={Md} problem {i}, run {rep}"
+
+
+@pytest.mark.parametrize("M,N,K", [(4096, 3072, 5120), (300, 19000, 768), (33, 200, 512), (8, 256, 1024)])
+def test_prepared_path(q4, M, N, K):
+    """q4_0_prepare_x then q4_0_gemm_prepared, the conversion on a second
+    stream ordered by an event: for M > 32 bit-equal to q4_0_gemm_ws, for any
+    M within the oracle's bound on sampled outputs (M <= 32 runs the
+    tensor-core kernel too)."""
+    rng = np.random.default_rng(M + 3 * N + K)
+    codes, scales = _weights(rng, N, K)
+    Xh = _x(rng, M, K)
+    W, X = pack_on_gpu(q4, codes, scales), dev(Xh)
+    xh = torch.empty(q4.q4_0_prepared_x_bytes(M, K), dtype=torch.uint8, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        q4.q4_0_prepare_x(X, M, K, xh)
+        done = torch.cuda.Event()
+        done.record()
+    torch.cuda.current_stream().wait_event(done)
+    Y = torch.full((M, N), float("nan"), device="cuda")
+    q4.q4_0_gemm_prepared(W, xh, Y, M, N, K)
+    torch.cuda.synchronize()
+    if M > 32:
+        ws = torch.empty(q4.q4_0_gemm_workspace_size(M, N, K), dtype=torch.uint8, device="cuda")
+        Y2 = torch.full((M, N), float("nan"), device="cuda")
+        q4.q4_0_gemm_ws(W, X, Y2, M, N, K, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(Y, Y2)
+    o = oracle.get()
+    ms = rng.integers(0, M, size=800)
+    ns = rng.integers(0, N, size=800)
+    ms[0], ns[0] = M - 1, N - 1
+    Y_or, B_or = o.gemm_sampled(o.pack(codes, scales), Xh, M, N, K, ms, ns)
+    check_gemm(Y.cpu().numpy()[ms, ns], Y_or, B_or, f"prepared {M}x{N}x{K}")
