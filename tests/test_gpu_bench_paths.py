@@ -244,3 +244,44 @@ def test_prepared_path(q4, M, N, K):
     ms[0], ns[0] = M - 1, N - 1
     Y_or, B_or = o.gemm_sampled(o.pack(codes, scales), Xh, M, N, K, ms, ns)
     check_gemm(Y.cpu().numpy()[ms, ns], Y_or, B_or, f"prepared {M}x{N}x{K}")
+
+
+def test_prepared_pipeline_over_steps(q4):
+    """The bench's pipeline for tensor-core steps: step k's X converted on a
+    side stream into buffer k % 2 once the GEMM of step k - 2 (the buffer's
+    last reader) is done, the GEMM of step k on the launching stream after
+    its conversion; six steps over three operand sets, each output bit-equal
+    to q4_0_gemm_ws on the same operands."""
+    rng = np.random.default_rng(21)
+    M, N, K = 600, 1536, 1024
+    sets = []
+    for _ in range(3):
+        codes, scales = _weights(rng, N, K)
+        sets.append((pack_on_gpu(q4, codes, scales), dev(_x(rng, M, K))))
+    ws = torch.empty(q4.q4_0_gemm_workspace_size(M, N, K), dtype=torch.uint8, device="cuda")
+    refs = []
+    for W, X in sets:
+        Y = torch.empty((M, N), device="cuda")
+        q4.q4_0_gemm_ws(W, X, Y, M, N, K, ws)
+        refs.append(Y)
+    torch.cuda.synchronize()
+    xh = [torch.empty(q4.q4_0_prepared_x_bytes(M, K), dtype=torch.uint8, device="cuda") for _ in range(2)]
+    ys = [torch.full((M, N), float("nan"), device="cuda") for _ in range(6)]
+    side, main = torch.cuda.Stream(), torch.cuda.current_stream()
+    side.wait_stream(main)
+    prep_done = [torch.cuda.Event(), torch.cuda.Event()]
+    gemm_done = [torch.cuda.Event(), torch.cuda.Event()]
+    for k in range(6):
+        b = k % 2
+        W, X = sets[k % 3]
+        if k >= 2:
+            side.wait_event(gemm_done[b])
+        with torch.cuda.stream(side):
+            q4.q4_0_prepare_x(X, M, K, xh[b])
+            prep_done[b].record(side)
+        main.wait_event(prep_done[b])
+        q4.q4_0_gemm_prepared(W, xh[b], ys[k], M, N, K)
+        gemm_done[b].record(main)
+    torch.cuda.synchronize()
+    for k in range(6):
+        assert torch.equal(ys[k], refs[k % 3]), f"step {k}"
