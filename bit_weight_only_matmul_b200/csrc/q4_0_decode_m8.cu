@@ -52,7 +52,11 @@
 // previous grid before it reads anything into the SM.
 // Numerics: each weight is rounded once to fp16 (relative error <= 2^-11,
 // inside the 1e-3 tolerance of the method); X is exact in fp16 within its
-// normal range; products are exact and accumulation is fp32.
+// normal range; products are exact and accumulation is fp32.  An X too large
+// for fp16 (checked once per problem) or a scale that makes a weight overflow
+// (looked for when a row's sum is not finite) sets Q4_DEVERR_FP16_RANGE.
+// A slot read with ordinary loads is released with a proxy fence first, so
+// the next TMA copy into it cannot land before those loads have read it.
 #include <cuda_fp16.h>
 
 #include <algorithm>

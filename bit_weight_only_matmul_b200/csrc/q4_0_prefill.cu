@@ -13,14 +13,16 @@
 //     tensor memory as fp16 (q - 8) * d: the raw Q4_0 bytes arrive by TMA
 //     (128 rows x 144 bytes = 256 k per load), each thread turns its row's
 //     blocks into fp16 pairs and writes them with tcgen05.st;
-//   * B operand = the activation tile, loaded by TMA as bf16 into the
-//     128-byte-swizzled K-major layout the MMA reads, then converted to fp16
-//     in place by eight warps;
+//   * B operand = the activation tile, loaded by TMA into the
+//     128-byte-swizzled K-major layout the MMA reads: as fp16 written once by
+//     the pre-pass (x_to_fp16_kernel: q4_0_gemm_ws, or q4_0_prepare_x on its
+//     own) or as bf16, converted to fp16 in place by eight warps;
 //   * one thread issues tcgen05.mma (kind::f16, M=128, N=256, K=16), four per
 //     64-k stage, and signals stage release with tcgen05.commit;
 //   * four epilogue warps drain the accumulator with tcgen05.ld; lane = weight
 //     row, column = activation row, so each store of a column is one
-//     contiguous 128-byte run of Y[m, n0..n0+31].
+//     contiguous 128-byte run of Y[m, n0..n0+31]; they add a residual or
+//     apply SwiGLU on the way (q4_0_gemm_grouped_ex).
 // fp16 operands: a weight (q - 8) * d is rounded once to fp16 (relative error
 // <= 2^-11, inside the 1e-3 tolerance of the method); X is exact in fp16 in
 // the normal range.  Both must lie within the fp16 range (|x| <= 65504,
