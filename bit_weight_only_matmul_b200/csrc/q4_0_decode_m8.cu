@@ -618,6 +618,147 @@ __global__ void __launch_bounds__(kThreads, 1) decode_m8_kernel(const __grid_con
     }
 }
 
+// ---------------------------------------------------------------- one small problem
+
+// A launch of one problem with few rows (a lone GEMV at M <= 8) is short:
+// its time is latency, not bandwidth.  Here each CTA takes 16*NR weight rows
+// over all of K, requests all of its weights at once (one TMA box of
+// 16*NR rows x 144 bytes per 256-k stage, each on its own barrier), and its
+// 16 warps split the work into NR row tiles x 16/NR k-groups (k-group j takes
+// stages j, j + 16/NR, ...).  X is converted once per CTA into the B
+// fragments of every stage.  The k-groups' partial sums meet in shared memory
+// and are added in k-group order by the first k-group's warps, which store
+// Y.  No clusters, no ring, no hand-over between CTAs.
+struct NarrowParams {
+    CUtensorMap wmap;     // Q4_0 bytes [N, K/32*18], box 144 x 16*NR
+    const uint8_t *W;     // the same bytes (read directly only by the rare scale check)
+    const uint16_t *X;
+    float *Y;
+    const float *R;       // residual (Q4_0_EPI_RESIDUAL)
+    unsigned *err;
+    int M, N, K, S, epi;  // S = K / 256 stages
+};
+
+constexpr int kNarrowWarps = 16;
+constexpr int kNarrowThreads = 32 * kNarrowWarps;
+
+template <int NR>
+constexpr int narrow_rows() { return 16 * NR; }
+
+// dynamic shared memory of a CTA: weights, fragments, partial sums, barriers
+template <int NR>
+constexpr size_t narrow_smem(int S) {
+    return static_cast<size_t>(S) * narrow_rows<NR>() * kStageRowBytes   // weight boxes
+           + static_cast<size_t>(S) * 4096                               // B fragment pairs per stage
+           + static_cast<size_t>(kNarrowWarps) * 4 * 32 * 4               // partial sums
+           + static_cast<size_t>(S) * 8 + 16 + 128;                      // barriers, abort flag, alignment
+}
+
+template <int NR>
+__global__ void __launch_bounds__(kNarrowThreads, 1) narrow_kernel(const __grid_constant__ NarrowParams P) {
+    constexpr int KG = kNarrowWarps / NR, ROWS = narrow_rows<NR>();
+    constexpr int kBox = ROWS * kStageRowBytes;
+    const int S = P.S;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *const wsm = align_smem<128>(smem_raw);
+    uint8_t *const fsm = wsm + S * kBox;                                    // kBox is a multiple of 16
+    float *const red = reinterpret_cast<float *>(fsm + S * 4096);
+    uint64_t *const bar = reinterpret_cast<uint64_t *>(red + kNarrowWarps * 4 * 32);
+    int *const abort_flag = reinterpret_cast<int *>(bar + S);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row0 = blockIdx.x * ROWS;
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < S; ++st) mbar_init(&bar[st], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    // programmatic dependent launch: the weights are asked into L2 before the
+    // previous grid is waited for, everything is read after it
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (threadIdx.x == 0) {
+        prefetch_tensormap(&P.wmap);
+        for (int st = 0; st < S; ++st) tma_prefetch_l2_2d(&P.wmap, st * kStageRowBytes, row0);
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < S; ++st) {
+            mbar_arrive_expect_tx(&bar[st], kBox);   // full boxes counted, rows past N zero-filled
+            tma_load_2d_u32(smem_addr(wsm + st * kBox), &P.wmap, st * kStageRowBytes, row0, &bar[st]);
+        }
+    }
+    // X -> fp16 B fragments of every stage: the (stage, row) pairs dealt over
+    // the warps, one 16-byte chunk (8 values) per lane, in the layout the
+    // decode kernel's stage_mma reads
+    const uint32_t f0 = smem_addr(fsm);
+    uint32_t xbad = 0;
+    {
+        const int cx = lane & 7;
+        const uint32_t fl = (4 * (cx >> 2) + 2 * (cx & 1)) * 512 + (lane >> 3) * 16 + ((cx >> 1) & 1) * 8;
+        for (int pi = warp; pi < S * P.M; pi += kNarrowWarps) {
+            const int st = pi / P.M, m = pi - st * P.M;
+            if (Q4_DEBUG_BAD(st < S && m < P.M, P.err, abort_flag)) break;
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(P.X + static_cast<int64_t>(m) * P.K + st * kStageK) +
+                                  lane);
+            if (blockIdx.x == 0) xbad |= x8_fp16_range_bad(v);   // every row of X checked once
+            const uint4 o = x8_to_fp16_permuted(v);
+            sts64(f0 + st * 4096 + fl + m * 64, o.x, o.y);
+            sts64(f0 + st * 4096 + fl + 512 + m * 64, o.z, o.w);
+        }
+    }
+    __syncthreads();
+    // this warp's row tile and k-group
+    const int rt = warp % NR, kg = warp / NR;
+    const int gq = lane >> 2, t = lane & 3;
+    float acc[2][4];
+    #pragma unroll
+    for (int c = 0; c < 2; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.f;
+    const uint32_t w0 = smem_addr(wsm) + (16 * rt + gq) * kStageRowBytes + 36 * t;
+    bool ok = true;
+    for (int st = kg; st < S; st += KG) {
+        if (!(ok = wait_or_abort(&bar[st], 0, abort_flag, P.err))) break;
+        uint32_t r[9], r8[9];
+        stage_words(w0 + st * kBox, r, r8);
+        stage_mma(r, r8, f0 + st * 4096 + lane * 16, acc);
+    }
+    {
+        float *const mine = red + ((rt * KG + kg) * 4) * 32;
+        #pragma unroll
+        for (int e = 0; e < 4; ++e) mine[e * 32 + lane] = acc[0][e] + acc[1][e];
+    }
+    __syncthreads();
+    if (kg == 0 && ok && !*reinterpret_cast<volatile int *>(abort_flag)) {
+        float sum[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int j = 0; j < KG; ++j) {
+            const float *part = red + ((rt * KG + j) * 4) * 32;
+            #pragma unroll
+            for (int e = 0; e < 4; ++e) sum[e] += part[e * 32 + lane];
+        }
+        // thread holds rows gq / gq+8 of the row tile x X rows 2t, 2t+1
+        bool bad_row[2] = {false, false};
+        #pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int m = 2 * t + (e & 1);
+            const int n = row0 + 16 * rt + gq + ((e & 2) ? 8 : 0);
+            if (m < P.M && n < P.N) {
+                if (!(fabsf(sum[e]) <= 3.402823466e38f)) bad_row[e >> 1] = true;
+                const int64_t o = static_cast<int64_t>(m) * P.N + n;
+                P.Y[o] = P.epi == kEpiResidual ? sum[e] + P.R[o] : sum[e];
+            }
+        }
+        #pragma unroll
+        for (int h = 0; h < 2; ++h)
+            if (bad_row[h]) {
+                const int64_t n = row0 + 16 * rt + gq + 8 * h;
+                scan_scales_fp16_range(P.W, n, n + 1, P.N, P.K, P.err);
+            }
+    }
+    if (xbad) atomicOr(P.err, (unsigned)Q4_DEVERR_FP16_RANGE);
+    // a wait that gave up: let every box land (bounded) before the CTA exits
+    if (threadIdx.x == 0 && *reinterpret_cast<volatile int *>(abort_flag))
+        for (int st = 0; st < S; ++st) mbar_wait(&bar[st], 0, P.err);
+}
+
 // ---------------------------------------------------------------- host side
 
 template <int CAP, int CL>
@@ -794,6 +935,54 @@ cudaError_t launch_cap(const q4::Problem *probs, const int *order, int count, co
 
 constexpr int kSmallCap = 8, kLargeCap = 128;
 
+// The one-problem kernel: 16 or 32 rows per CTA, as many CTAs as that takes,
+// when they fit on the SMs at once and the CTA's weights, fragments and sums
+// fit in shared memory.  Returns the row tiles per CTA (1 or 2), 0 if not.
+int narrow_rows_per_cta(const q4::Problem &p, const q4::DeviceInfo &dev) {
+    if (p.M < 1 || p.M > 8 || p.K < kStageK || p.K % kStageK != 0 || p.N < 1) return 0;
+    if (p.epi != kEpiNone && p.epi != kEpiResidual) return 0;
+    const int S = static_cast<int>(p.K / kStageK);
+    const int nr = p.N <= 16LL * dev.sm_count ? 1 : p.N <= 32LL * dev.sm_count ? 2 : 0;
+    if (nr == 0) return 0;
+    const size_t smem = nr == 1 ? narrow_smem<1>(S) : narrow_smem<2>(S);
+    return smem <= dev.smem_optin ? nr : 0;
+}
+
+template <int NR>
+cudaError_t launch_narrow(const q4::Problem &p, const q4::DeviceInfo &dev, cudaStream_t s) {
+    NarrowParams P;
+    if (!q4::get_tensor_map(&P.wmap, p.W, p.N, p.K / 32 * 18, NR == 1 ? q4::kMapWeights16 : q4::kMapWeights32))
+        return cudaErrorInvalidValue;
+    P.W = p.W;
+    P.X = p.X;
+    P.Y = p.Y;
+    P.R = p.R;
+    P.err = dev.err;
+    P.M = static_cast<int>(p.M);
+    P.N = static_cast<int>(p.N);
+    P.K = static_cast<int>(p.K);
+    P.S = static_cast<int>(p.K / kStageK);
+    P.epi = p.epi;
+    const size_t smem = narrow_smem<NR>(P.S);
+    static q4::DeviceOnce configured;
+    cudaError_t e = configured.run(dev.device, [&] {
+        return cudaFuncSetAttribute(narrow_kernel<NR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(dev.smem_optin));
+    });
+    if (e != cudaSuccess) return e;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((p.N + narrow_rows<NR>() - 1) / narrow_rows<NR>()), 1, 1);
+    cfg.blockDim = dim3(kNarrowThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, narrow_kernel<NR>, P);
+}
+
 }  // namespace
 
 namespace q4 {
@@ -806,6 +995,11 @@ bool decode_m8_supports(const Problem &p) {
 
 cudaError_t launch_decode_m8(const Problem *probs, int count, const DeviceInfo &dev, cudaStream_t s) {
     if (count <= 0) return cudaSuccess;
+    if (count == 1) {   // a lone small problem: the one-problem kernel
+        const int nr = narrow_rows_per_cta(probs[0], dev);
+        if (nr == 1) return launch_narrow<1>(probs[0], dev, s);
+        if (nr == 2) return launch_narrow<2>(probs[0], dev, s);
+    }
     static thread_local std::vector<int> order;
     order.resize(count);
     for (int i = 0; i < count; ++i) order[i] = i;

@@ -50,11 +50,13 @@ bool encode(CUtensorMap *out, const Key &k) {
     EncodeTiled enc = encoder();
     if (!enc) return false;
     const cuuint32_t estr[2] = {1, 1};
-    if (k.kind == q4::kMapWeights128 || k.kind == q4::kMapWeights128Prefill) {
-        // Q4_0 bytes as uint8 [rows = N, cols = K/32*18], box 144 bytes x 128 rows
+    if (k.kind == q4::kMapWeights128 || k.kind == q4::kMapWeights128Prefill || k.kind == q4::kMapWeights16 ||
+        k.kind == q4::kMapWeights32) {
+        // Q4_0 bytes as uint8 [rows = N, cols = K/32*18], box 144 bytes x 128 (16, 32) rows
         const cuuint64_t dims[2] = {static_cast<cuuint64_t>(k.cols), static_cast<cuuint64_t>(k.rows)};
         const cuuint64_t strides[1] = {static_cast<cuuint64_t>(k.cols)};
-        const cuuint32_t box[2] = {144, 128};
+        const cuuint32_t box_rows = k.kind == q4::kMapWeights16 ? 16 : k.kind == q4::kMapWeights32 ? 32 : 128;
+        const cuuint32_t box[2] = {144, box_rows};
         return enc(out, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(k.ptr), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;

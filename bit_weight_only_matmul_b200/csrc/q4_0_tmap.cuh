@@ -12,7 +12,9 @@ enum MapKind {
     kMapActivationsSw128 = 3,    // bf16 X, box 64 x 256, 128-byte swizzle
     kMapActivationsF16Sw128 = 4, // fp16 X, box 64 x 256, 128-byte swizzle
     kMapXDecode16 = 5,           // bf16 X, box 64 x 16, 128-byte swizzle (decode, M <= 16)
-    kMapXDecode32 = 6            // bf16 X, box 64 x 32, 128-byte swizzle (decode, M <= 32)
+    kMapXDecode32 = 6,           // bf16 X, box 64 x 32, 128-byte swizzle (decode, M <= 32)
+    kMapWeights16 = 7,           // Q4_0 bytes, box 144 bytes (256 k) x 16 rows
+    kMapWeights32 = 8            // Q4_0 bytes, box 144 bytes (256 k) x 32 rows
 };
 
 bool tensor_maps_available();
