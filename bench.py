@@ -51,7 +51,7 @@ DEFAULT_WORKLOAD = "cfg_decode"
 
 # kernel that dominates each workload, and the source file it lives in
 DOMINANT = {
-    "gemv": ("decode_m8_kernel", "q4_0_decode_m8.cu"),
+    "gemv": ("narrow_kernel", "q4_0_decode_m8.cu"),
     "layer": ("decode_m8_kernel", "q4_0_decode_m8.cu"),
     "cfg_decode": ("decode_m8_kernel", "q4_0_decode_m8.cu"),
     "concurrent": ("decode_mma_kernel", "q4_0_decode_mma.cu"),
