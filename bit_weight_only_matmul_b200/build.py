@@ -14,6 +14,7 @@ into _build_debug/ and libq4_0_b200_debug.so.
 from __future__ import annotations
 
 import argparse
+import concurrent.futures
 import glob
 import os
 import subprocess
@@ -48,7 +49,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False, 
     os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     newest_header = max((os.path.getmtime(h) for h in _headers()), default=0.0)
-    objs, relink = [], force or not os.path.exists(lib)
+    objs, relink, cmds = [], force or not os.path.exists(lib), []
     for src in srcs:
         obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
@@ -61,7 +62,13 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False, 
             cmd += ["-Xptxas", "-v"]
         if verbose:
             print(" ".join(cmd), flush=True)
-        subprocess.run(cmd, check=True)
+        cmds.append(cmd)
+    if cmds:
+        # the translation units compile independently: one nvcc per unit, a few at a time
+        with concurrent.futures.ThreadPoolExecutor(max_workers=min(len(cmds), os.cpu_count() or 4)) as pool:
+            for r in pool.map(lambda c: subprocess.run(c), cmds):
+                if r.returncode != 0:
+                    raise subprocess.CalledProcessError(r.returncode, r.args)
         relink = True
     if relink or any(os.path.getmtime(o) > os.path.getmtime(lib) for o in objs):
         tmp = lib + f".tmp{os.getpid()}"
