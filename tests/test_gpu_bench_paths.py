@@ -285,3 +285,33 @@ def test_prepared_pipeline_over_steps(q4):
     torch.cuda.synchronize()
     for k in range(6):
         assert torch.equal(ys[k], refs[k % 3]), f"step {k}"
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 256), (3, 2368, 512), (1, 2369, 512), (8, 4736, 768),
+                                   (2, 4737, 768), (5, 300, 6144), (1, 3072, 8192)])
+def test_one_problem_kernel_bounds(q4, M, N, K):
+    """A lone problem at M <= 8 runs the one-problem kernel when its rows fit
+    the SMs in CTAs of 16 rows (N <= 16 * 148), else of 32 (N <= 32 * 148),
+    and its CTA fits in shared memory; one row more, or a K too long, takes
+    the cluster path.  Both sides of each bound against the oracle, with and
+    without a residual (in place)."""
+    rng = np.random.default_rng(M * 7 + N + K)
+    codes, scales = _weights(rng, N, K)
+    X = _x(rng, M, K)
+    W, Xd = pack_on_gpu(q4, codes, scales), dev(X)
+    o = oracle.get()
+    ms = rng.integers(0, M, size=600)
+    ns = rng.integers(0, N, size=600)
+    ms[0], ns[0] = M - 1, N - 1
+    Y_or, B_or = o.gemm_sampled(o.pack(codes, scales), X, M, N, K, ms, ns)
+    Y = torch.full((M, N), float("nan"), device="cuda")
+    q4.q4_0_gemm(W, Xd, Y, M, N, K)
+    torch.cuda.synchronize()
+    check_gemm(Y.cpu().numpy()[ms, ns], Y_or, B_or, f"lone {M}x{N}x{K}")
+    R = rng.standard_normal((M, N)).astype(np.float32)
+    Rd = dev(R)
+    q4.q4_0_gemm_grouped_ex([(W, Xd, Rd, M, N, K, Rd, q4.Q4_0_EPI_RESIDUAL)])
+    torch.cuda.synchronize()
+    ref = Y_or + R[ms, ns]
+    check_gemm(Rd.cpu().numpy()[ms, ns] - R[ms, ns], Y_or, B_or + 1e3 * 2.0**-22 * np.abs(ref),
+               f"lone {M}x{N}x{K} + residual in place")
