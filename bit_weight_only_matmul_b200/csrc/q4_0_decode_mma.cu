@@ -16,9 +16,9 @@
 // B200, half of what HBM delivers.  The warp-level m16n8k16 has no such floor,
 // and its n=8 matches the few activation rows.
 //
-// Per CTA (one per SM): a producer warp, two X warps and two groups of 8
-// compute warps; X warp G and compute group G take the stages g with
-// g mod 2 == G, so that two stages are worked on at once.
+// Per CTA (one per SM): a producer warp and two groups of 8 compute warps;
+// compute group G takes the stages g with g mod 2 == G, so that two stages
+// are worked on at once.
 //  * stage = 256 k of an item (128 weight rows x 144 bytes, one TMA box) plus
 //    the same 256 k of every row of X (1-D bulk copies), in a ring of 4-6
 //    slots; for M <= 8 a slot holds two stages, so that every wait, arrival
@@ -33,9 +33,13 @@
 //  * for M > 8 the stage's X rows come as four TMA boxes (64 k x 8*NT rows,
 //    128-byte swizzle, rows past M zero-filled) instead of one 1-D copy per
 //    row: 32 copies per stage would cap the stream near 2.2 TB/s;
-//  * the X warps convert the stage's X rows to fp16 straight into the
-//    matching mma.sync B fragments (two buffers per group), one 8-byte shared
-//    load per fragment for the compute threads;
+//  * the compute warps of the group convert the stage's X rows to fp16
+//    straight into the matching mma.sync B fragments (two buffers per
+//    group), each warp one eighth of every row, and meet on the buffer's
+//    barrier before their MMAs: one 8-byte shared load per fragment for the
+//    compute threads.  (A separate conversion warp per group held the group
+//    back at M = 32: it alone issued as many instructions per stage as a
+//    compute warp's MMAs and dequantization together.)
 //  * fused epilogues (decode only): Y = sums + R, or, for a gate/up weight
 //    whose items hold 64 gate rows then the same 64 features' up rows,
 //    Y[m, f] = silu(gate) * up with the up tiles' sums handed to the gate
@@ -82,8 +86,8 @@ constexpr int kRawW = kItemRows * kStageRowBytes;   // 18432
 constexpr int kXRow = kStageK * 2;                  // 512 bytes of one bf16 X row per stage
 constexpr int kXPitch = kXRow + 16;                 // skews consecutive X rows by four banks
 constexpr int kXBufs = 4;                           // buffer g mod 4 belongs to group g mod 2
-constexpr int kWarpProd = 0, kWarpX0 = 1, kWarp0 = 3, kGroupWarps = 8;
-constexpr int kThreads = 32 * (kWarp0 + 2 * kGroupWarps);  // 608
+constexpr int kWarpProd = 0, kWarp0 = 1, kGroupWarps = 8;
+constexpr int kThreads = 32 * (kWarp0 + 2 * kGroupWarps);  // 544
 using q4split::kMaxItems;
 using q4split::kMaxSched;
 using q4split::kMaxSplitCtas;
@@ -120,7 +124,7 @@ struct Smem {
     uint2 xf[kXBufs][subs<NT>()][16][NT][32];               // B fragments: [stage][mma u][n tile][lane]
     float comb[8][NT][4][32];                   // group-1 sums handed to group 0 at an item's end
     uint64_t raw_full[ring<NT, CL>()], raw_empty[ring<NT, CL>()];
-    uint64_t xf_full[kXBufs], xf_empty[kXBufs];
+    uint64_t xf_full[kXBufs];
     uint64_t comb_full, comb_empty;
     float epi[4][NT][4][32];                    // SwiGLU: up-row sums handed to the gate rows
     uint64_t epi_full, epi_empty;
@@ -307,12 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
     if (threadIdx.x == 0) {
         for (int s = 0; s < RS; ++s) {
             mbar_init(&S.raw_full[s], 1);
-            mbar_init(&S.raw_empty[s], kGroupWarps + 1);
+            mbar_init(&S.raw_empty[s], kGroupWarps);
         }
-        for (int s = 0; s < kXBufs; ++s) {
-            mbar_init(&S.xf_full[s], 1);
-            mbar_init(&S.xf_empty[s], kGroupWarps);
-        }
+        for (int s = 0; s < kXBufs; ++s) mbar_init(&S.xf_full[s], kGroupWarps);
         mbar_init(&S.comb_full, kGroupWarps);
         mbar_init(&S.comb_empty, kGroupWarps);
         mbar_init(&S.epi_full, kGroupWarps / 2);
@@ -395,93 +396,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
             }
             ++prod_issued;
         }
-    } else if (warp < kWarp0) {
-        // ---------------------------------------------------------------- X rows -> fp16 B fragments
-        // X warp G fills all 16 MMAs of the stages of its parity: lane (gx, tx)
-        // -> X row 8j+gx, blocks 2tx and 2tx+1.  With the 528-byte pitch the
-        // 16-byte loads of a warp fall in eight distinct bank groups and the
-        // 8-byte stores in sixteen bank pairs.
-        const int G = warp - kWarpX0;
-        const int gx = lane >> 2, tx = lane & 3;
-        uint32_t g = 0, xbad = 0;
-        Walk<CL, SUB> q{};
-        q.start(D, rank);
-        for (; q.item >= 0; q.next(D, rank), ++g) {
-            if ((g & 1) != static_cast<uint32_t>(G)) continue;
-            const GroupProblem &pr = P.p[q.prob];
-            // every problem's X is range-checked once, by the CTA (or cluster)
-            // that works its first item
-            const bool check = q.row0 == 0;
-            const int slot = g % RS, xb = g % kXBufs;
-            bool ok = true;
-            if (lane == 0) {
-                ok = wait_or_abort(&S.raw_full[slot], (g / RS) & 1, &S.abort_flag, P.err);
-                if (ok) ok = wait_or_abort(&S.xf_empty[xb], ((g / kXBufs) & 1) ^ 1, &S.abort_flag, P.err);
-            }
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            if (check) {
-                // a separate pass, so that the conversion below stays as it is
-                // for every other item: this lane's 16-byte pieces of its rows
-                for (int i = 0; i < q.cnt && i < SUB; ++i) {
-                    const uint8_t *xr = S.raw[slot][i] + kRawW;
-                    for (int j = 0; j < NT; ++j) {
-                        const int m = 8 * j + gx;
-                        if (m >= pr.M) continue;
-                        for (int piece = 0; piece < 8; ++piece) {
-                            const int k = 64 * tx + 8 * piece;
-                            const uint8_t *src = xmap<NT>() ? xr + tx * xbox_bytes<NT>() + m * 128 +
-                                                                  ((((k & 63) >> 3) ^ (m & 7)) << 4)
-                                                            : xr + m * kXPitch + 2 * k;
-                            xbad |= x8_fp16_range_bad(*reinterpret_cast<const uint4 *>(src));
-                        }
-                    }
-                }
-            }
-            #pragma unroll
-            for (int i = 0; i < SUB; ++i) {
-                if (i >= q.cnt) break;
-                const uint8_t *xr = S.raw[slot][i] + kRawW;
-                #pragma unroll
-                for (int j = 0; j < NT; ++j) {
-                    const int m = 8 * j + gx;
-                    #pragma unroll
-                    for (int xw = 0; xw < 2; ++xw)
-                        #pragma unroll
-                        for (int h = 0; h < 2; ++h)
-                            #pragma unroll
-                            for (int wp = 0; wp < 2; ++wp) {
-                                uint4 o = make_uint4(0u, 0u, 0u, 0u);
-                                // TMA boxes (M > 8) zero-fill the rows past M, so every row
-                                // converts unconditionally (straight-line loads); 1-D copies
-                                // (M <= 8) leave those rows stale
-                                if (xmap<NT>() || m < pr.M) {
-                                    const int k = 32 * (2 * tx + xw) + 16 * h + 8 * wp;
-                                    // box tx holds k 64tx..64tx+63; its 16-byte chunk c of row m
-                                    // sits at chunk c ^ (m & 7) (128-byte swizzle)
-                                    const uint8_t *src =
-                                        xmap<NT>() ? xr + tx * xbox_bytes<NT>() + m * 128 +
-                                                         ((((k & 63) >> 3) ^ (m & 7)) << 4)
-                                                   : xr + m * kXPitch + 2 * k;
-                                    o = x8_to_fp16_permuted(*reinterpret_cast<const uint4 *>(src));
-                                }
-                                S.xf[xb][i][8 * xw + 4 * wp + h][j][lane] = make_uint2(o.x, o.y);
-                                S.xf[xb][i][8 * xw + 4 * wp + 2 + h][j][lane] = make_uint2(o.z, o.w);
-                            }
-                }
-            }
-            fence_proxy_async_smem();   // the producer's next copies may land in this slot
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&S.xf_full[xb]);
-                mbar_arrive(&S.raw_empty[slot]);
-            }
-        }
-        if (xbad) atomicOr(P.err, (unsigned)Q4_DEVERR_FP16_RANGE);
     } else {
         // ---------------------------------------------------------------- compute
         const int cw = warp - kWarp0;
         const int G = cw >> 3, tile = cw & 7;   // stage parity, rows 16*tile .. 16*tile+15
         const int gq = lane >> 2, t = lane & 3;
+        // X conversion: the B fragment of lane 4gx + tx holds X row 8j + gx at
+        // blocks 2tx and 2tx+1 of the stage.  Warp `tile` converts chunk
+        // (xw, h, wp) = (tile >> 2, (tile >> 1) & 1, tile & 1) -- k = 32(2tx + xw)
+        // + 16h + 8wp .. +7 -- of every row and stage, which feeds fragments
+        // 8xw + 4wp + h (low half) and 8xw + 4wp + 2 + h (high half).  Lane L
+        // works (gx, tx) = (L & 7, ((L >> 3) + 2 ((L >> 2) & 1)) & 3): each
+        // quarter-warp of its 16-byte loads covers the eight gx (eight bank
+        // groups, in the swizzled boxes and at the 528-byte pitch alike), and
+        // each half-warp of its 8-byte stores sixteen distinct bank pairs.
+        const int xw = tile >> 2, xh = (tile >> 1) & 1, xp = tile & 1;
+        const int gx = lane & 7, tx = ((lane >> 3) + 2 * ((lane >> 2) & 1)) & 3;
+        const int xl = 4 * gx + tx, xu = 8 * xw + 4 * xp + xh;
+        const int xk = 32 * (2 * tx + xw) + 16 * xh + 8 * xp;
+        uint32_t xbad = 0;
         float acc[2][NT][4];
         #pragma unroll
         for (int c = 0; c < 2; ++c)
@@ -494,6 +427,44 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
             if ((g & 1) == static_cast<uint32_t>(G)) {
                 const int slot = g % RS, xb = g % kXBufs;
                 if (!wait_or_abort(&S.raw_full[slot], (g / RS) & 1, &S.abort_flag, P.err)) break;
+                // this warp's share of the slot's X -> B fragments.  Buffer xb was
+                // last read by the group's slot g - 4; every warp of the group
+                // finished that before it arrived on the buffer barrier of slot
+                // g - 2, which this warp has passed.
+                {
+                    const GroupProblem &pr = P.p[q.prob];
+                    // every problem's X is range-checked once, by the CTA (or
+                    // cluster) that works its first item
+                    const bool check = q.row0 == 0;
+                    #pragma unroll
+                    for (int i = 0; i < SUB; ++i) {
+                        if (i >= q.cnt) break;
+                        const uint8_t *xr = S.raw[slot][i] + kRawW;
+                        #pragma unroll
+                        for (int j = 0; j < NT; ++j) {
+                            const int m = 8 * j + gx;
+                            uint4 o = make_uint4(0u, 0u, 0u, 0u);
+                            // TMA boxes (M > 8) zero-fill the rows past M, so every row
+                            // converts unconditionally (straight-line loads); 1-D copies
+                            // (M <= 8) leave those rows stale
+                            if (xmap<NT>() || m < pr.M) {
+                                // box tx holds k 64tx..64tx+63; its 16-byte chunk c of row m
+                                // sits at chunk c ^ (m & 7) (128-byte swizzle)
+                                const uint8_t *src = xmap<NT>()
+                                                         ? xr + tx * xbox_bytes<NT>() + m * 128 +
+                                                               ((((xk & 63) >> 3) ^ (m & 7)) << 4)
+                                                         : xr + m * kXPitch + 2 * xk;
+                                const uint4 v = *reinterpret_cast<const uint4 *>(src);
+                                if (check) xbad |= x8_fp16_range_bad(v);
+                                o = x8_to_fp16_permuted(v);
+                            }
+                            S.xf[xb][i][xu][j][xl] = make_uint2(o.x, o.y);
+                            S.xf[xb][i][xu + 2][j][xl] = make_uint2(o.z, o.w);
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.xf_full[xb]);
                 uint32_t rg[SUB][9], rg8[SUB][9];
                 #pragma unroll
                 for (int i = 0; i < SUB; ++i) {
@@ -518,8 +489,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
                     word_mma<NT, 1, 2>(rg[i], rg8[i], S.xf[xb][i], lane, acc);
                     word_mma<NT, 1, 3>(rg[i], rg8[i], S.xf[xb][i], lane, acc);
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&S.xf_empty[xb]);
             }
             if (q.stage + q.cnt == q.end) {
                 // end of the item: the two groups add their sums
@@ -639,6 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
                 ++items_done;
             }
         }
+        if (xbad) atomicOr(P.err, (unsigned)Q4_DEVERR_FP16_RANGE);
     }
 
     __syncthreads();
