@@ -121,7 +121,7 @@ struct XComb<NT, 1> {};
 template <int NT, int CL>
 struct Smem {
     uint8_t raw[ring<NT, CL>()][subs<NT>()][raw_bytes<NT>()];   // per stage: W rows (pitch 144), X rows (pitch 528)
-    uint2 xf[kXBufs][subs<NT>()][16][NT][32];               // B fragments: [stage][mma u][n tile][lane]
+    uint4 xf[kXBufs][subs<NT>()][8][NT][32];                // B fragments of MMAs 2v, 2v+1: [stage][v][n tile][lane]
     float comb[8][NT][4][32];                   // group-1 sums handed to group 0 at an item's end
     uint64_t raw_full[ring<NT, CL>()], raw_empty[ring<NT, CL>()];
     uint64_t xf_full[kXBufs];
@@ -165,7 +165,7 @@ __device__ __forceinline__ void block_word(const uint32_t (&r)[9], int w, uint32
 // MMAs u = 8B + 2w (low nibbles) and u + 1 (high nibbles) of the stage.
 template <int NT, int B, int W>
 __device__ __forceinline__ void word_mma(const uint32_t (&rg)[9], const uint32_t (&rg8)[9],
-                                         const uint2 (&xf)[16][NT][32], int lane, float (&acc)[2][NT][4]) {
+                                         const uint4 (&xf)[8][NT][32], int lane, float (&acc)[2][NT][4]) {
     uint32_t dg, dg8, qg, qg8;
     block_word<B>(rg, W, dg, qg);
     block_word<B>(rg8, W, dg8, qg8);
@@ -176,8 +176,9 @@ __device__ __forceinline__ void word_mma(const uint32_t (&rg)[9], const uint32_t
     #pragma unroll
     for (int j = 0; j < NT; ++j) {
         // a0/a1: k cols (2t, 2t+1) of rows g / g+8; a2/a3: k cols (2t+8, 2t+9)
-        mma_f16(acc[0][j], cg[0], cg8[0], cg[1], cg8[1], xf[u][j][lane]);
-        mma_f16(acc[1][j], cg[2], cg8[2], cg[3], cg8[3], xf[u + 1][j][lane]);
+        const uint4 b = xf[u >> 1][j][lane];   // one 16-byte load: the fragments of MMAs u and u + 1
+        mma_f16(acc[0][j], cg[0], cg8[0], cg[1], cg8[1], make_uint2(b.x, b.y));
+        mma_f16(acc[1][j], cg[2], cg8[2], cg[3], cg8[3], make_uint2(b.z, b.w));
     }
 }
 
@@ -409,7 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
         // works (gx, tx) = (L & 7, ((L >> 3) + 2 ((L >> 2) & 1)) & 3): each
         // quarter-warp of its 16-byte loads covers the eight gx (eight bank
         // groups, in the swizzled boxes and at the 528-byte pitch alike), and
-        // each half-warp of its 8-byte stores sixteen distinct bank pairs.
+        // its 8-byte stores into the fragment pairs meet at most two to a bank
+        // pair per half-warp.
         const int xw = tile >> 2, xh = (tile >> 1) & 1, xp = tile & 1;
         const int gx = lane & 7, tx = ((lane >> 3) + 2 * ((lane >> 2) & 1)) & 3;
         const int xl = 4 * gx + tx, xu = 8 * xw + 4 * xp + xh;
@@ -458,8 +460,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
                                 if (check) xbad |= x8_fp16_range_bad(v);
                                 o = x8_to_fp16_permuted(v);
                             }
-                            S.xf[xb][i][xu][j][xl] = make_uint2(o.x, o.y);
-                            S.xf[xb][i][xu + 2][j][xl] = make_uint2(o.z, o.w);
+                            // fragment u is half u & 1 of pair u >> 1
+                            uint2 *f = reinterpret_cast<uint2 *>(&S.xf[xb][i][xu >> 1][j][xl]) + xh;
+                            f[0] = make_uint2(o.x, o.y);
+                            f[2 * NT * 32] = make_uint2(o.z, o.w);   // fragment xu + 2: the next pair
                         }
                     }
                 }

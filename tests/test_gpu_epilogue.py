@@ -51,7 +51,7 @@ def test_interleave_bit_exact(q4):
     assert np.array_equal(out.cpu().numpy(), want.reshape(-1))
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 3072, 3072), (2, 200, 1024), (32, 300, 512), (7, 129, 768),
+@pytest.mark.parametrize("M,N,K", [(1, 3072, 3072), (2, 200, 1024), (32, 300, 512), (7, 129, 768), (16, 257, 768),
                                    (33, 200, 512), (300, 129, 768), (600, 512, 1024)])
 @pytest.mark.parametrize("inplace", [False, True])
 def test_residual_epilogue(q4, M, N, K, inplace):
@@ -85,7 +85,7 @@ def _swiglu_case(q4, rng, M, F, K):
     return Wgu, X, ref, tol
 
 
-@pytest.mark.parametrize("M,F,K", [(1, 64, 256), (2, 512, 1024), (32, 256, 512), (1, 8192, 3072),
+@pytest.mark.parametrize("M,F,K", [(1, 64, 256), (2, 512, 1024), (32, 256, 512), (12, 192, 1024), (1, 8192, 3072),
                                    (33, 64, 256), (300, 320, 512), (513, 1024, 1024)])
 def test_swiglu_epilogue(q4, M, F, K):
     rng = np.random.default_rng(M * 3 + F + K)
@@ -93,6 +93,32 @@ def test_swiglu_epilogue(q4, M, F, K):
     Y = torch.full((M, F), float("nan"), device="cuda")
     q4.q4_0_gemm_grouped_ex([(Wgu, dev(X), Y, M, 2 * F, K, None, q4.Q4_0_EPI_SWIGLU)])
     _check(Y.cpu().numpy(), ref, tol, "swiglu")
+    no_device_error(q4)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 3072, 3072), (5, 1000, 768)])
+def test_epilogues_forced_256k_stage_kernel(q4, M, N, K):
+    """Residual and SwiGLU on the M <= 32 kernel forced for M <= 8 (one n
+    tile; cluster split mode for the few-item case)."""
+    rng = np.random.default_rng(M + N + K + 5)
+    o = oracle.get()
+    codes, scales = _weights(rng, N, K)
+    X = _x(rng, M, K)
+    R = rng.standard_normal((M, N)).astype(np.float32)
+    Y = torch.full((M, N), float("nan"), device="cuda")
+    Wgu, Xs, ref_s, tol_s = _swiglu_case(q4, rng, M, N // 2 // 64 * 64, K)
+    F = N // 2 // 64 * 64
+    Ys = torch.full((M, F), float("nan"), device="cuda")
+    q4.q4_0_force_path(q4.PATH_DECODE)
+    try:
+        q4.q4_0_gemm_grouped_ex([(pack_on_gpu(q4, codes, scales), dev(X), Y, M, N, K, dev(R), q4.Q4_0_EPI_RESIDUAL)])
+        q4.q4_0_gemm_grouped_ex([(Wgu, dev(Xs), Ys, M, 2 * F, K, None, q4.Q4_0_EPI_SWIGLU)])
+    finally:
+        q4.q4_0_force_path(q4.PATH_AUTO)
+    Y_or, B_or = o.gemm(o.pack(codes, scales), X, M, N, K)
+    ref = Y_or + R
+    _check(Y.cpu().numpy(), ref, _bound(B_or) + 2.0**-22 * np.abs(ref), "residual, 256-k stage kernel")
+    _check(Ys.cpu().numpy(), ref_s, tol_s, "swiglu, 256-k stage kernel")
     no_device_error(q4)
 
 

@@ -236,6 +236,30 @@ def test_forced_warp_mma_decode(q4, M, N, K):
     run_gemm(q4, M, N, K, path=q4.PATH_DECODE_EXACT)
 
 
+@pytest.mark.parametrize("M,N,K", [
+    (1, 3072, 3072),   # 24 items: clusters of 4-8 cut them into pieces
+    (2, 129, 3072),    # one 12-stage item in pieces
+    (8, 1000, 1792),   # eight 7-stage items
+    (5, 257, 768),     # ragged N, 3-stage items
+    (3, 20000, 512),   # more items than SMs: plain mode
+])
+def test_forced_decode_256k_stages(q4, M, N, K):
+    """The M <= 32 kernel (256-k stages) forced for M <= 8, where it runs one
+    n tile with two stages per ring slot, in plain and cluster split modes."""
+    run_gemm(q4, M, N, K, path=q4.PATH_DECODE)
+
+
+def test_forced_decode_256k_stages_layer(q4):
+    """A decoder layer (216 items) on the same kernel: split mode in pairs."""
+    b = build_workload(q4, workloads.workload("layer"), full_oracle=True)
+    q4.q4_0_force_path(q4.PATH_DECODE)
+    try:
+        q4.q4_0_gemm_grouped(b.problems())
+    finally:
+        q4.q4_0_force_path(0)
+    check_built(b, "layer, 256-k stage kernel")
+
+
 @pytest.mark.parametrize("name,layers", [("cfg_decode", [0, 13, 25]), ("concurrent", [0, 25]), ("flow_head", None)])
 def test_decode_workloads_sampled(q4, name, layers):
     b = build_workload(q4, workloads.workload(name, layers=layers), samples=400)
