@@ -36,10 +36,15 @@
 //  * the compute warps of the group convert the stage's X rows to fp16
 //    straight into the matching mma.sync B fragments (two buffers per
 //    group), each warp one eighth of every row, and meet on the buffer's
-//    barrier before their MMAs: one 8-byte shared load per fragment for the
-//    compute threads.  (A separate conversion warp per group held the group
-//    back at M = 32: it alone issued as many instructions per stage as a
-//    compute warp's MMAs and dequantization together.)
+//    barrier before their MMAs.  The fragments of a code word's two MMAs sit
+//    side by side: one 16-byte shared load per pair for the compute threads.
+//    (A separate conversion warp per group held the group back at M = 32: it
+//    alone issued as many instructions per stage as a compute warp's MMAs and
+//    dequantization together.  Warps of 32 rows over half the blocks, which
+//    halve the fragment traffic, need the stage's words live across the MMAs:
+//    with the producer warp the CTA has 96 registers a thread, and either the
+//    words spill or the slot is held until the MMAs end, which starves the
+//    ring; both measured slower.)
 //  * fused epilogues (decode only): Y = sums + R, or, for a gate/up weight
 //    whose items hold 64 gate rows then the same 64 features' up rows,
 //    Y[m, f] = silu(gate) * up with the up tiles' sums handed to the gate
@@ -403,17 +408,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
         const int G = cw >> 3, tile = cw & 7;   // stage parity, rows 16*tile .. 16*tile+15
         const int gq = lane >> 2, t = lane & 3;
         // X conversion: the B fragment of lane 4gx + tx holds X row 8j + gx at
-        // blocks 2tx and 2tx+1 of the stage.  Warp `tile` converts chunk
-        // (xw, h, wp) = (tile >> 2, (tile >> 1) & 1, tile & 1) -- k = 32(2tx + xw)
-        // + 16h + 8wp .. +7 -- of every row and stage, which feeds fragments
-        // 8xw + 4wp + h (low half) and 8xw + 4wp + 2 + h (high half).  Lane L
-        // works (gx, tx) = (L & 7, ((L >> 3) + 2 ((L >> 2) & 1)) & 3): each
-        // quarter-warp of its 16-byte loads covers the eight gx (eight bank
-        // groups, in the swizzled boxes and at the 528-byte pitch alike), and
-        // its 8-byte stores into the fragment pairs meet at most two to a bank
-        // pair per half-warp.
-        const int xw = tile >> 2, xh = (tile >> 1) & 1, xp = tile & 1;
-        const int gx = lane & 7, tx = ((lane >> 3) + 2 * ((lane >> 2) & 1)) & 3;
+        // blocks 2tx and 2tx+1 of the stage.  The 16-byte chunk (xw, h, wp) of
+        // a row -- k = 32(2tx + xw) + 16h + 8wp .. +7 -- feeds fragments
+        // 8xw + 4wp + h (low half) and 8xw + 4wp + 2 + h (high half), i.e. half h
+        // of fragment pairs 4xw + 2wp and 4xw + 2wp + 1.  Warp `tile` takes
+        // (xw, wp) = (tile >> 2, (tile >> 1) & 1) and the fragment lanes of half
+        // s = tile & 1; lane L takes h = L & 1 and, with i = (L >> 1) & 3,
+        // c = (L >> 3) & 1 and k = 2s + (L >> 4), gx = (i & 1) + 4 (i >> 1) + 2c
+        // and tx = (k + (i >> 1) + 2c) & 3.  Then the eight lanes of each
+        // quarter-warp load from eight distinct bank groups (in the swizzled
+        // boxes and at the 528-byte pitch alike), and the two lanes of each
+        // fragment pair fill it whole, eight pairs with distinct bank groups per
+        // half-warp: both the loads and the stores are free of bank conflicts.
+        const int xw = tile >> 2, xp = (tile >> 1) & 1, xh = lane & 1;
+        const int xi = (lane >> 1) & 3, xc = (lane >> 3) & 1, xq = 2 * (tile & 1) + (lane >> 4);
+        const int gx = (xi & 1) + 4 * (xi >> 1) + 2 * xc, tx = (xq + (xi >> 1) + 2 * xc) & 3;
         const int xl = 4 * gx + tx, xu = 8 * xw + 4 * xp + xh;
         const int xk = 32 * (2 * tx + xw) + 16 * xh + 8 * xp;
         uint32_t xbad = 0;
