@@ -88,7 +88,8 @@ def source_sha(fname: str) -> str:
 
 def recorded_traffic(workload: str):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
-    summary, or None when absent or when the kernel source changed since."""
+    summary (the mean over a step's launches where a step has several), or
+    None when absent or when the kernel source changed since."""
     kernel, src = DOMINANT[workload] if workload in DOMINANT else UTIL_KERNELS[workload]
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.traffic.json")
     if not os.path.exists(path):
@@ -595,7 +596,9 @@ def build_record(name, wl, tensor, ms_total, steps, world, clock, launch, peaks,
         "roofline": {"bound": bound, "kernel": kernel, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
                      "frac": round(achieved / peak, 4), "peak_source": peak_src,
                      "spec_peak": spec, "frac_of_spec": round(achieved / spec, 4),
-                     "traffic": recorded_traffic(name), "algorithmic_per_launch": per_step},
+                     "traffic": recorded_traffic(name), "algorithmic_per_step": per_step,
+                     "dominant_launches_per_step": dominant_launches_per_step(wl),
+                     "algorithmic_per_launch": round(per_step / dominant_launches_per_step(wl))},
         "clocks": clock,
     }
 
@@ -639,7 +642,11 @@ def run_ours(args, rank: int, world: int):
     q4.q4_0_device_error(clear=True)
     for name in names:
         headline = name == args.workload
-        wl = workloads.workload(name)
+        if args.layers and headline:
+            wl = workloads.workload(name, layers=list(range(args.layers)))
+            wl.description += f" -- first {args.layers} layer(s) only, a profiling case"
+        else:
+            wl = workloads.workload(name)
         tensor = name in TENSOR_WORKLOADS
         copies = rotating_copies(wl)
         log(f"[rank {rank}] building {wl.name}: {len(wl.linears)} GEMMs x {copies} copies, "
@@ -916,11 +923,31 @@ def whole_job_rate(units_per_rank_step: float, steps: int, world: int, max_ms: f
     return world * steps * units_per_rank_step / (max_ms * 1e-3)
 
 
+def dominant_launches_per_step(wl) -> int:
+    """Launches of the step's dominant kernel: the decode launches of a
+    decode step (see launches_per_step), or one tensor-core GEMM per M > 32
+    problem.  `achieved` is the step's algorithmic work over the step's
+    time, i.e. the mean over these launches, which run back to back."""
+    big = sum(1 for l in wl.linears if l.M > 32)
+    if big:
+        return big
+    n8 = sum(1 for l in wl.linears if l.M <= 8)
+    n32 = sum(1 for l in wl.linears if 8 < l.M <= 32)
+    return -(-n8 // 128) + -(-n32 // 64)
+
+
+LAYERED_WORKLOADS = ("cfg_decode", "concurrent", "flow_head")
+
+
 def launches_per_step(name, wl) -> int:
-    # all M <= 32 problems of a step share one launch; each M > 32 problem is
-    # two (the fp16 conversion of X, then the tensor-core GEMM)
-    small = any(l.M <= 32 for l in wl.linears)
-    return int(small) + 2 * sum(1 for l in wl.linears if l.M > 32)
+    """Kernel launches of one step.  A grouped call runs its M <= 8 problems
+    in launches of up to 128 (one alone: the one-problem kernel) and its
+    8 < M <= 32 problems in launches of up to 64 (their X tensor maps fill
+    the kernel parameters); each M > 32 problem is two launches (the fp16
+    conversion of X, then the tensor-core GEMM)."""
+    n8 = sum(1 for l in wl.linears if l.M <= 8)
+    n32 = sum(1 for l in wl.linears if 8 < l.M <= 32)
+    return -(-n8 // 128) + -(-n32 // 64) + 2 * sum(1 for l in wl.linears if l.M > 32)
 
 
 # --------------------------------------------------------------------------- the oracle as a baseline
@@ -1079,7 +1106,12 @@ def main(argv=None):
     ap.add_argument("--soak", type=float, default=1.0,
                     help="seconds of untimed load after warm-up, so the clock sampler sees the GPU busy "
                          "(0 for short profiling runs)")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="with --only: keep the first N layers of a 26-layer workload (small cases for ncu "
+                         "captures; the line then describes that case, not the configuration)")
     args = ap.parse_args(argv)
+    if args.layers and (not args.only or args.workload not in LAYERED_WORKLOADS):
+        ap.error("--layers needs --only and one of " + ", ".join(LAYERED_WORKLOADS))
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
