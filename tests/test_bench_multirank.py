@@ -91,3 +91,31 @@ def test_cpu_baselines_single_and_all_cores():
     assert one["unit"] == two["unit"] == "GB/s"
     assert one["value"] > 0 and two["value"] > 0
     assert one["kind"] == two["kind"] == "oracle"
+
+
+def test_launch_counts_follow_the_library_chunks():
+    """gpu_launches: a grouped call runs its M <= 8 problems in launches of up
+    to 128 and its 8 < M <= 32 problems in launches of up to 64 (the X tensor
+    maps fill the kernel parameters); an M > 32 problem is the X conversion
+    plus the tensor-core GEMM.  The M = 32 decode step (104 GEMMs) is two
+    launches, and `achieved` is the mean over them."""
+    import bench
+    import workloads
+    want = {"gemv": (1, 1), "layer": (1, 1), "layer_fused": (1, 1), "cfg_decode": (1, 1),
+            "concurrent": (2, 2), "flow_head": (1, 1), "adapter": (2, 1), "qkv_prefill": (2, 1)}
+    for name, (launches, dominant) in want.items():
+        wl = workloads.workload(name)
+        assert bench.launches_per_step(name, wl) == launches, name
+        assert bench.dominant_launches_per_step(wl) == dominant, name
+    # mixed shapes: 130 problems at M = 2 and 65 at M = 16 -> 2 + 2 launches
+    mixed = workloads.Workload("mixed", "test", [workloads.Linear("a", 256, 256, 0, 0, 2)] * 130 +
+                               [workloads.Linear("b", 256, 256, 0, 1, 16)] * 65)
+    assert bench.launches_per_step("mixed", mixed) == 4
+
+
+def test_layers_option_needs_a_layered_workload():
+    import bench
+    with pytest.raises(SystemExit):
+        bench.main(["--workload", "gemv", "--only", "--layers", "2"])
+    with pytest.raises(SystemExit):
+        bench.main(["--workload", "concurrent", "--layers", "2"])
