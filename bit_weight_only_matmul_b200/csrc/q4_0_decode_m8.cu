@@ -673,12 +673,15 @@ __global__ void __launch_bounds__(kNarrowThreads, 1) narrow_kernel(const __grid_
         fence_mbar_init();
     }
     __syncthreads();
-    // programmatic dependent launch: the weights are asked into L2 before the
-    // previous grid is waited for, everything is read after it
+    // programmatic dependent launch: the weights and X are asked into L2
+    // before the previous grid is waited for, everything is read after it
+    // (CTA m < M asks for row m of X)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0) {
         prefetch_tensormap(&P.wmap);
         for (int st = 0; st < S; ++st) tma_prefetch_l2_2d(&P.wmap, st * kStageRowBytes, row0);
+    } else if (threadIdx.x == 32 && static_cast<int>(blockIdx.x) < P.M) {
+        bulk_prefetch_l2(P.X + static_cast<int64_t>(blockIdx.x) * P.K, static_cast<uint32_t>(P.K * 2));
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (threadIdx.x == 0) {

@@ -35,6 +35,13 @@ __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int x
 }
 
 // Fetch a tensor map (kernel parameter) into the descriptor cache.
+// L2 prefetch of `bytes` (a multiple of 16) from a 16-byte aligned global
+// address: no shared memory, no completion to wait for.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+                 : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
