@@ -624,8 +624,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_m8_kernel(const __grid_con
 // its time is latency, not bandwidth.  Here each CTA takes 16*NR weight rows
 // over all of K, requests all of its weights at once (one TMA box of
 // 16*NR rows x 144 bytes per 256-k stage, each on its own barrier), and its
-// 16 warps split the work into NR row tiles x 16/NR k-groups (k-group j takes
-// stages j, j + 16/NR, ...).  X is converted once per CTA into the B
+// NW warps (16 or 32) split the work into NR row tiles x NW/NR k-groups
+// (k-group j takes stages j, j + NW/NR, ...).  X is converted once per CTA into the B
 // fragments of every stage.  The k-groups' partial sums meet in shared memory
 // and are added in k-group order by the first k-group's warps, which store
 // Y.  No clusters, no ring, no hand-over between CTAs.
@@ -639,31 +639,39 @@ struct NarrowParams {
     int M, N, K, S, epi;  // S = K / 256 stages
 };
 
-constexpr int kNarrowWarps = 16;
-constexpr int kNarrowThreads = 32 * kNarrowWarps;
-
 template <int NR>
 constexpr int narrow_rows() { return 16 * NR; }
 
+// Warps of a CTA: 32 where 16 would give a k-group (16 / NR of them) more
+// than one stage and the CTA's weights are few (at most 24 stage-row-tiles,
+// 55 KB): twice the k-groups then halve the longest chain of stages, which
+// paces such latency-bound launches.  Else 16: with one stage per k-group
+// anyway, or with more weights per SM, where the stream paces the launch, the
+// larger CTA only adds its own cost.  Back to back: 3072^2 at M = 1 5.15 ->
+// 4.03 us with 32 warps (12 stages over 8 or 16 k-groups), M = 8 7.37 ->
+// 5.22 us; 4096^2 4.84 against 5.02 us and 2368 x 3072 (16 rows a CTA) 3.08
+// against 3.45 us with 16.
+constexpr int narrow_warps(int S, int NR) { return NR > 0 && S > 16 / NR && S * NR <= 24 ? 32 : 16; }
+
 // dynamic shared memory of a CTA: weights, fragments, partial sums, barriers
-template <int NR>
+template <int NR, int NW>
 constexpr size_t narrow_smem(int S) {
     return static_cast<size_t>(S) * narrow_rows<NR>() * kStageRowBytes   // weight boxes
            + static_cast<size_t>(S) * 4096                               // B fragment pairs per stage
-           + static_cast<size_t>(kNarrowWarps) * 4 * 32 * 4               // partial sums
+           + static_cast<size_t>(NW) * 4 * 32 * 4                         // partial sums
            + static_cast<size_t>(S) * 8 + 16 + 128;                      // barriers, abort flag, alignment
 }
 
-template <int NR>
-__global__ void __launch_bounds__(kNarrowThreads, 1) narrow_kernel(const __grid_constant__ NarrowParams P) {
-    constexpr int KG = kNarrowWarps / NR, ROWS = narrow_rows<NR>();
+template <int NR, int NW>
+__global__ void __launch_bounds__(32 * NW, 1) narrow_kernel(const __grid_constant__ NarrowParams P) {
+    constexpr int KG = NW / NR, ROWS = narrow_rows<NR>();
     constexpr int kBox = ROWS * kStageRowBytes;
     const int S = P.S;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *const wsm = align_smem<128>(smem_raw);
     uint8_t *const fsm = wsm + S * kBox;                                    // kBox is a multiple of 16
     float *const red = reinterpret_cast<float *>(fsm + S * 4096);
-    uint64_t *const bar = reinterpret_cast<uint64_t *>(red + kNarrowWarps * 4 * 32);
+    uint64_t *const bar = reinterpret_cast<uint64_t *>(red + NW * 4 * 32);
     int *const abort_flag = reinterpret_cast<int *>(bar + S);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row0 = blockIdx.x * ROWS;
@@ -698,7 +706,7 @@ __global__ void __launch_bounds__(kNarrowThreads, 1) narrow_kernel(const __grid_
     {
         const int cx = lane & 7;
         const uint32_t fl = (4 * (cx >> 2) + 2 * (cx & 1)) * 512 + (lane >> 3) * 16 + ((cx >> 1) & 1) * 8;
-        for (int pi = warp; pi < S * P.M; pi += kNarrowWarps) {
+        for (int pi = warp; pi < S * P.M; pi += NW) {
             const int st = pi / P.M, m = pi - st * P.M;
             if (Q4_DEBUG_BAD(st < S && m < P.M, P.err, abort_flag)) break;
             const uint4 v = __ldg(reinterpret_cast<const uint4 *>(P.X + static_cast<int64_t>(m) * P.K + st * kStageK) +
@@ -947,11 +955,12 @@ int narrow_rows_per_cta(const q4::Problem &p, const q4::DeviceInfo &dev) {
     const int S = static_cast<int>(p.K / kStageK);
     const int nr = p.N <= 16LL * dev.sm_count ? 1 : p.N <= 32LL * dev.sm_count ? 2 : 0;
     if (nr == 0) return 0;
-    const size_t smem = nr == 1 ? narrow_smem<1>(S) : narrow_smem<2>(S);
+    const size_t smem = narrow_warps(S, nr) == 32 ? (nr == 1 ? narrow_smem<1, 32>(S) : narrow_smem<2, 32>(S))
+                                              : (nr == 1 ? narrow_smem<1, 16>(S) : narrow_smem<2, 16>(S));
     return smem <= dev.smem_optin ? nr : 0;
 }
 
-template <int NR>
+template <int NR, int NW>
 cudaError_t launch_narrow(const q4::Problem &p, const q4::DeviceInfo &dev, cudaStream_t s) {
     NarrowParams P;
     if (!q4::get_tensor_map(&P.wmap, p.W, p.N, p.K / 32 * 18, NR == 1 ? q4::kMapWeights16 : q4::kMapWeights32))
@@ -966,10 +975,10 @@ cudaError_t launch_narrow(const q4::Problem &p, const q4::DeviceInfo &dev, cudaS
     P.K = static_cast<int>(p.K);
     P.S = static_cast<int>(p.K / kStageK);
     P.epi = p.epi;
-    const size_t smem = narrow_smem<NR>(P.S);
+    const size_t smem = narrow_smem<NR, NW>(P.S);
     static q4::DeviceOnce configured;
     cudaError_t e = configured.run(dev.device, [&] {
-        return cudaFuncSetAttribute(narrow_kernel<NR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        return cudaFuncSetAttribute(narrow_kernel<NR, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     static_cast<int>(dev.smem_optin));
     });
     if (e != cudaSuccess) return e;
@@ -978,12 +987,12 @@ cudaError_t launch_narrow(const q4::Problem &p, const q4::DeviceInfo &dev, cudaS
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>((p.N + narrow_rows<NR>() - 1) / narrow_rows<NR>()), 1, 1);
-    cfg.blockDim = dim3(kNarrowThreads, 1, 1);
+    cfg.blockDim = dim3(32 * NW, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, narrow_kernel<NR>, P);
+    return cudaLaunchKernelEx(&cfg, narrow_kernel<NR, NW>, P);
 }
 
 }  // namespace
@@ -1000,8 +1009,9 @@ cudaError_t launch_decode_m8(const Problem *probs, int count, const DeviceInfo &
     if (count <= 0) return cudaSuccess;
     if (count == 1) {   // a lone small problem: the one-problem kernel
         const int nr = narrow_rows_per_cta(probs[0], dev);
-        if (nr == 1) return launch_narrow<1>(probs[0], dev, s);
-        if (nr == 2) return launch_narrow<2>(probs[0], dev, s);
+        const bool wide = nr > 0 && narrow_warps(static_cast<int>(probs[0].K / kStageK), nr) == 32;
+        if (nr == 1) return wide ? launch_narrow<1, 32>(probs[0], dev, s) : launch_narrow<1, 16>(probs[0], dev, s);
+        if (nr == 2) return wide ? launch_narrow<2, 32>(probs[0], dev, s) : launch_narrow<2, 16>(probs[0], dev, s);
     }
     static thread_local std::vector<int> order;
     order.resize(count);
