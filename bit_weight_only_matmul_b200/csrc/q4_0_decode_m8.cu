@@ -624,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_m8_kernel(const __grid_con
 // its time is latency, not bandwidth.  Here each CTA takes 16*NR weight rows
 // over all of K, requests all of its weights at once (one TMA box of
 // 16*NR rows x 144 bytes per 256-k stage, each on its own barrier), and its
-// NW warps (16 or 32) split the work into NR row tiles x NW/NR k-groups
+// NW warps (16, 24 or 32) split the work into NR row tiles x NW/NR k-groups
 // (k-group j takes stages j, j + NW/NR, ...).  X is converted once per CTA into the B
 // fragments of every stage.  The k-groups' partial sums meet in shared memory
 // and are added in k-group order by the first k-group's warps, which store
@@ -642,18 +642,21 @@ struct NarrowParams {
 template <int NR>
 constexpr int narrow_rows() { return 16 * NR; }
 
-// Warps of a CTA: 32 where 16 would give a k-group (16 / NR of them) more
-// than one stage and the CTA's weights are few (at most 24 stage-row-tiles,
-// 55 KB): twice the k-groups then halve the longest chain of stages, which
-// paces such latency-bound launches.  Else 16: with one stage per k-group
-// anyway, or with more weights per SM, where the stream paces the launch, the
-// larger CTA only adds its own cost.  Back to back: 3072^2 at M = 1 5.15 ->
-// 4.03 us with 32 warps (12 stages over 8 or 16 k-groups), M = 8 7.37 ->
-// 5.22 us; 4096^2 4.84 against 5.02 us and 2368 x 3072 (16 rows a CTA) 3.08
-// against 3.45 us with 16.
-constexpr int narrow_warps(int S, int NR) { return NR > 0 && S > 16 / NR && S * NR <= 24 ? 32 : 16; }
+// Warps of a CTA.  Where 16 would give a k-group (16 / NR of them) more than
+// one stage and the CTA's weights are few (at most 24 stage-row-tiles,
+// 55 KB), 24 warps give every k-group at most one stage, which halves the
+// longest chain of stages that paces such latency-bound launches; 32 when
+// M > 4, where the X conversion (S * M rows of 256 k) wants the extra warps.
+// Else 16: with one stage per k-group anyway, or with more weights per SM,
+// where the stream paces the launch, a larger CTA only adds its own cost.
+// Back to back, 3072^2: M = 1 5.15 -> 3.87 us (24 warps; 4.05 with 32),
+// M = 2 5.72 -> 4.01 us, M = 8 7.37 -> 5.26 us (32 warps; 5.40 with 24); with
+// 16 warps kept: 4096^2 4.84 against 5.02 us and 2368 x 3072 (16 rows a CTA)
+// 3.08 against 3.45 us with 32.
+constexpr int narrow_warps(int S, int NR, int M) {
+    return NR > 0 && S > 16 / NR && S * NR <= 24 ? (M <= 4 ? 24 : 32) : 16;
+}
 
-// dynamic shared memory of a CTA: weights, fragments, partial sums, barriers
 template <int NR, int NW>
 constexpr size_t narrow_smem(int S) {
     return static_cast<size_t>(S) * narrow_rows<NR>() * kStageRowBytes   // weight boxes
@@ -955,8 +958,10 @@ int narrow_rows_per_cta(const q4::Problem &p, const q4::DeviceInfo &dev) {
     const int S = static_cast<int>(p.K / kStageK);
     const int nr = p.N <= 16LL * dev.sm_count ? 1 : p.N <= 32LL * dev.sm_count ? 2 : 0;
     if (nr == 0) return 0;
-    const size_t smem = narrow_warps(S, nr) == 32 ? (nr == 1 ? narrow_smem<1, 32>(S) : narrow_smem<2, 32>(S))
-                                              : (nr == 1 ? narrow_smem<1, 16>(S) : narrow_smem<2, 16>(S));
+    const int nw = narrow_warps(S, nr, static_cast<int>(p.M));
+    const size_t smem = nw == 32   ? (nr == 1 ? narrow_smem<1, 32>(S) : narrow_smem<2, 32>(S))
+                        : nw == 24 ? (nr == 1 ? narrow_smem<1, 24>(S) : narrow_smem<2, 24>(S))
+                                   : (nr == 1 ? narrow_smem<1, 16>(S) : narrow_smem<2, 16>(S));
     return smem <= dev.smem_optin ? nr : 0;
 }
 
@@ -1009,9 +1014,15 @@ cudaError_t launch_decode_m8(const Problem *probs, int count, const DeviceInfo &
     if (count <= 0) return cudaSuccess;
     if (count == 1) {   // a lone small problem: the one-problem kernel
         const int nr = narrow_rows_per_cta(probs[0], dev);
-        const bool wide = nr > 0 && narrow_warps(static_cast<int>(probs[0].K / kStageK), nr) == 32;
-        if (nr == 1) return wide ? launch_narrow<1, 32>(probs[0], dev, s) : launch_narrow<1, 16>(probs[0], dev, s);
-        if (nr == 2) return wide ? launch_narrow<2, 32>(probs[0], dev, s) : launch_narrow<2, 16>(probs[0], dev, s);
+        const int nw = narrow_warps(static_cast<int>(probs[0].K / kStageK), nr, static_cast<int>(probs[0].M));
+        if (nr == 1)
+            return nw == 32   ? launch_narrow<1, 32>(probs[0], dev, s)
+                   : nw == 24 ? launch_narrow<1, 24>(probs[0], dev, s)
+                              : launch_narrow<1, 16>(probs[0], dev, s);
+        if (nr == 2)
+            return nw == 32   ? launch_narrow<2, 32>(probs[0], dev, s)
+                   : nw == 24 ? launch_narrow<2, 24>(probs[0], dev, s)
+                              : launch_narrow<2, 16>(probs[0], dev, s);
     }
     static thread_local std::vector<int> order;
     order.resize(count);

@@ -288,13 +288,18 @@ def test_prepared_pipeline_over_steps(q4):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 1, 256), (3, 2368, 512), (1, 2369, 512), (8, 4736, 768),
-                                   (2, 4737, 768), (5, 300, 6144), (1, 3072, 8192)])
+                                   (2, 4737, 768), (5, 300, 6144), (1, 3072, 8192),
+                                   (1, 2000, 5120), (4, 3000, 2304), (6, 3000, 3072), (1, 3072, 4096)])
 def test_one_problem_kernel_bounds(q4, M, N, K):
     """A lone problem at M <= 8 runs the one-problem kernel when its rows fit
     the SMs in CTAs of 16 rows (N <= 16 * 148), else of 32 (N <= 32 * 148),
     and its CTA fits in shared memory; one row more, or a K too long, takes
-    the cluster path.  Both sides of each bound against the oracle, with and
-    without a residual (in place)."""
+    the cluster path.  The CTA has 24 warps (M <= 4) or 32 (M > 4) where 16
+    would leave a k-group two stages of at most 24 stage-row-tiles: here
+    2000 x 5120 (16 rows a CTA, 20 stages) and 3000 x 2304 with 24, 300 x 6144
+    and 3000 x 3072 with 32, 3072 x 4096 (32 stage-row-tiles) with 16.  Both
+    sides of each bound against the oracle, with and without a residual (in
+    place)."""
     rng = np.random.default_rng(M * 7 + N + K)
     codes, scales = _weights(rng, N, K)
     X = _x(rng, M, K)
