@@ -168,9 +168,17 @@ __device__ __forceinline__ void block_word(const uint32_t (&r)[9], int w, uint32
 }
 
 // MMAs u = 8B + 2w (low nibbles) and u + 1 (high nibbles) of the stage.
+// Accumulator chains per n-tile: with one n-tile, the low- and high-nibble
+// MMAs of a code word go to two chains so that they do not wait on each
+// other; with 2 or 4 n-tiles one chain each, the low-nibble MMAs of all
+// n-tiles issued before the high-nibble ones (a chain's MMAs NT apart), which
+// frees NT * 4 registers (M = 32: 2.09 -> 2.21 TB/s).
+template <int NT> constexpr int chains() { return NT == 1 ? 2 : 1; }
+
 template <int NT, int B, int W>
 __device__ __forceinline__ void word_mma(const uint32_t (&rg)[9], const uint32_t (&rg8)[9],
-                                         const uint4 (&xf)[8][NT][32], int lane, float (&acc)[2][NT][4]) {
+                                         const uint4 (&xf)[8][NT][32], int lane,
+                                         float (&acc)[chains<NT>()][NT][4]) {
     uint32_t dg, dg8, qg, qg8;
     block_word<B>(rg, W, dg, qg);
     block_word<B>(rg8, W, dg8, qg8);
@@ -178,12 +186,23 @@ __device__ __forceinline__ void word_mma(const uint32_t (&rg)[9], const uint32_t
     q4_word_to_fp16(qg, dg, cg);
     q4_word_to_fp16(qg8, dg8, cg8);
     constexpr int u = 8 * B + 2 * W;
+    constexpr int C = chains<NT>();
+    // one 16-byte load per n-tile: the fragments of MMAs u and u + 1
+    uint4 b[NT];
     #pragma unroll
-    for (int j = 0; j < NT; ++j) {
-        // a0/a1: k cols (2t, 2t+1) of rows g / g+8; a2/a3: k cols (2t+8, 2t+9)
-        const uint4 b = xf[u >> 1][j][lane];   // one 16-byte load: the fragments of MMAs u and u + 1
-        mma_f16(acc[0][j], cg[0], cg8[0], cg[1], cg8[1], make_uint2(b.x, b.y));
-        mma_f16(acc[1][j], cg[2], cg8[2], cg[3], cg8[3], make_uint2(b.z, b.w));
+    for (int j = 0; j < NT; ++j) b[j] = xf[u >> 1][j][lane];
+    // a0/a1: k cols (2t, 2t+1) of rows g / g+8; a2/a3: k cols (2t+8, 2t+9)
+    if constexpr (C == 2) {
+        #pragma unroll
+        for (int j = 0; j < NT; ++j) {
+            mma_f16(acc[0][j], cg[0], cg8[0], cg[1], cg8[1], make_uint2(b[j].x, b[j].y));
+            mma_f16(acc[1][j], cg[2], cg8[2], cg[3], cg8[3], make_uint2(b[j].z, b[j].w));
+        }
+    } else {
+        #pragma unroll
+        for (int j = 0; j < NT; ++j) mma_f16(acc[0][j], cg[0], cg8[0], cg[1], cg8[1], make_uint2(b[j].x, b[j].y));
+        #pragma unroll
+        for (int j = 0; j < NT; ++j) mma_f16(acc[0][j], cg[2], cg8[2], cg[3], cg8[3], make_uint2(b[j].z, b[j].w));
     }
 }
 
@@ -426,9 +445,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
         const int xl = 4 * gx + tx, xu = 8 * xw + 4 * xp + xh;
         const int xk = 32 * (2 * tx + xw) + 16 * xh + 8 * xp;
         uint32_t xbad = 0;
-        float acc[2][NT][4];
+        constexpr int C = chains<NT>();
+        float acc[C][NT][4];
         #pragma unroll
-        for (int c = 0; c < 2; ++c)
+        for (int c = 0; c < C; ++c)
             #pragma unroll
             for (int j = 0; j < NT; ++j) acc[c][j][0] = acc[c][j][1] = acc[c][j][2] = acc[c][j][3] = 0.f;
         uint32_t g = 0, items_done = 0, split_done = 0, swiglu_done = 0;
@@ -512,7 +532,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
                     #pragma unroll
                     for (int j = 0; j < NT; ++j)
                         #pragma unroll
-                        for (int e = 0; e < 4; ++e) S.comb[tile][j][e][lane] = acc[0][j][e] + acc[1][j][e];
+                        for (int e = 0; e < 4; ++e)
+                            S.comb[tile][j][e][lane] = C == 2 ? acc[0][j][e] + acc[C - 1][j][e] : acc[0][j][e];
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S.comb_full);
                 } else {
@@ -522,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
                     for (int j = 0; j < NT; ++j)
                         #pragma unroll
                         for (int e = 0; e < 4; ++e)
-                            sum[j][e] = acc[0][j][e] + acc[1][j][e] + S.comb[tile][j][e][lane];
+                            sum[j][e] = (C == 2 ? acc[0][j][e] + acc[C - 1][j][e] : acc[0][j][e]) + S.comb[tile][j][e][lane];
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S.comb_empty);
                     if constexpr (CL > 1) {
@@ -615,7 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(const __grid_co
                     }
                 }
                 #pragma unroll
-                for (int c = 0; c < 2; ++c)
+                for (int c = 0; c < C; ++c)
                     #pragma unroll
                     for (int j = 0; j < NT; ++j) acc[c][j][0] = acc[c][j][1] = acc[c][j][2] = acc[c][j][3] = 0.f;
                 ++items_done;
