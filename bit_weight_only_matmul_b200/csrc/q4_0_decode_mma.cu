@@ -49,9 +49,10 @@
 //    whose items hold 64 gate rows then the same 64 features' up rows,
 //    Y[m, f] = silu(gate) * up with the up tiles' sums handed to the gate
 //    tiles through shared memory -- the intermediate never reaches HBM;
-//  * the accumulators (two chains per n-tile) live across the whole item; at
-//    its end the group-1 warp hands its sums through shared memory to the
-//    group-0 warp of the same rows, which stores Y[m, n].
+//  * the accumulators (one chain per n-tile, two for a single n-tile) live
+//    across the whole item; at its end the group-1 warp hands its sums
+//    through shared memory to the group-0 warp of the same rows, which
+//    stores Y[m, n].
 // Split mode (M <= 8, up to kMaxItems items): when a launch has few items,
 // whole items leave a tail -- one decoder layer at M=1 has 24 items of 32
 // stages next to 192 of 12, so the busiest CTA works 32 stages against a
