@@ -338,12 +338,33 @@ def test_split_mode_few_items_grouped(q4):
 
 
 def test_grouped_many_problems_mixed_m(q4):
-    """70 problems, one of them at M = 16: the launcher sends M > 8 calls in
-    chunks of 64 problems, and sorted by K the first chunk here holds only
-    M <= 8 problems (which then run in split mode), the second the rest."""
+    """70 problems, one of them at M = 16: the M <= 8 problems go to the
+    M <= 8 kernel in one launch (split mode: fewer than 1024 items), the
+    M = 16 problem to the M <= 32 kernel."""
     o = oracle.get()
     rng = np.random.default_rng(53)
     shapes = [(1 + i % 8, 8 + (7 * i) % 33, 256 * (2 + i % 3)) for i in range(69)] + [(16, 24, 256)]
+    probs, refs, Ys = [], [], []
+    for (M, N, K) in shapes:
+        codes, scales, X = rand_inputs(rng, M, N, K)
+        Y = torch.full((M, N), float("nan"), device="cuda")
+        probs.append((pack_on_gpu(q4, codes, scales), dev(X), Y, M, N, K))
+        refs.append(o.gemm(o.pack(codes, scales), X, M, N, K))
+        Ys.append(Y)
+    q4.q4_0_gemm_grouped(probs)
+    for (M, N, K), Y, (Y_or, B_or) in zip(shapes, Ys, refs):
+        check_gemm(Y.cpu().numpy(), Y_or, B_or, f"many problems M={M} N={N} K={K}")
+    no_device_error(q4)
+
+
+def test_grouped_many_problems_m_over_8(q4):
+    """70 problems at 8 < M <= 32 in one grouped call: their X tensor maps fill
+    the kernel parameters at 64 problems, so the call runs as two launches of
+    the M <= 32 kernel (64 and 6 problems, sorted by K), each at the n-tile
+    count of its largest M."""
+    o = oracle.get()
+    rng = np.random.default_rng(59)
+    shapes = [(9 + (5 * i) % 24, 8 + (7 * i) % 41, 256 * (1 + i % 3)) for i in range(70)]
     probs, refs, Ys = [], [], []
     for (M, N, K) in shapes:
         codes, scales, X = rand_inputs(rng, M, N, K)
